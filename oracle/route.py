@@ -1,0 +1,301 @@
+"""Oracle for the router: block pooling, block scores, row softmax, Top-p cut, forced
+blocks and frame-level top-k. float64 NumPy, one plain step per function.
+
+Test infrastructure only (see the package docstring); never used by the product path.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import numpy as np
+
+EPS_GAP = 1e-6    # probability gap under which two blocks count as tied
+EPS_MASS = 1e-5   # distance of a cumulative mass from p under which the cut counts as tied
+
+
+@dataclasses.dataclass
+class RouteCfg:
+    """Routing configuration.
+
+    mode         "topp" (FVAttn Top-p) or "frame_topk" (Sol-Attn frame-level top-k).
+    p            Top-p mass threshold; p >= 1 selects every key block.
+    block        tokens per block (the pages use 32 or 64; the library supports 64).
+    force_diag   always keep key block i for query block i.
+    local_window w > 0 forces the band |i - j| <= w (wzjinhao notes §5.2 "邻近块保底").
+    frame_len    tokens per frame (0: no frame structure).
+    topk_frames  k for frame mode.
+    frame_window fw >= 0 forces the frames within +-fw of the query's frames; < 0 disables.
+    force_first_frame  always keep the blocks of frame 0.
+    scale        softmax scale; None means 1/sqrt(d).
+    """
+    mode: str = "topp"
+    p: float = 0.9
+    block: int = 64
+    force_diag: bool = True
+    local_window: int = 0
+    frame_len: int = 0
+    topk_frames: int = 0
+    frame_window: int = -1
+    force_first_frame: bool = False
+    scale: Optional[float] = None
+
+
+def _f64(x) -> np.ndarray:
+    if hasattr(x, "detach"):          # a torch tensor: bf16/fp32 -> fp64 is exact
+        x = x.detach().to("cpu").double().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def pool_blocks(X, block: int) -> np.ndarray:
+    """Mean of each block of `block` consecutive tokens, over the valid tokens only.
+
+    X: [BH, S, d]. Returns [BH, nb, d], nb = ceil(S / block). The last block, when S is not a
+    multiple of `block`, averages its S - (nb-1)*block real tokens (wzjinhao notes §5.2 pools
+    block means; padding tokens are not data, so they are not averaged in).
+    """
+    X = _f64(X)
+    BH, S, d = X.shape
+    nb = -(-S // block)
+    out = np.empty((BH, nb, d), dtype=np.float64)
+    for i in range(nb):
+        lo, hi = i * block, min(S, (i + 1) * block)
+        out[:, i, :] = X[:, lo:hi, :].sum(axis=1) / (hi - lo)
+    return out
+
+
+def pool_frames(X, frame_len: int) -> np.ndarray:
+    """Mean of each frame's tokens (Sol-Attn §2.1: a frame is represented by the average
+    pool of its patch tokens). X: [BH, S, d] -> [BH, F, d]."""
+    X = _f64(X)
+    BH, S, d = X.shape
+    F = -(-S // frame_len)
+    out = np.empty((BH, F, d), dtype=np.float64)
+    for f in range(F):
+        lo, hi = f * frame_len, min(S, (f + 1) * frame_len)
+        out[:, f, :] = X[:, lo:hi, :].sum(axis=1) / (hi - lo)
+    return out
+
+
+def block_scores(qbar: np.ndarray, kbar: np.ndarray, scale: float) -> np.ndarray:
+    """Sc[bh, i, j] = <qbar[bh, i], kbar[bh, j]> * scale (wzjinhao notes §5.2: einsum of
+    the block means divided by sqrt(d))."""
+    return np.matmul(qbar, np.swapaxes(kbar, -1, -2)) * scale
+
+
+def row_softmax(sc: np.ndarray) -> np.ndarray:
+    """Softmax over the key-block axis: the distribution whose cumulative mass the Top-p
+    cut compares with p."""
+    m = sc.max(axis=-1, keepdims=True)
+    e = np.exp(sc - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def topp_row(pi: np.ndarray, p: float):
+    """Top-p cut of one row (FVAttn summary, "AI视频生成的阿喀琉斯之踵": sort blocks by
+    importance, descending, and take them in turn until the cumulative importance reaches p).
+
+    Ties in pi go to the lower block index. Returns (order, k_star, csum): `order` is the
+    descending order, `csum[k-1]` the mass of the first k blocks, and the selection is
+    order[:k_star] with k_star the smallest k whose mass is >= p (all blocks when p >= 1 or
+    when rounding keeps the total just under p).
+    """
+    nb = pi.shape[0]
+    order = np.argsort(-pi, kind="stable")
+    csum = np.cumsum(pi[order])
+    if p >= 1.0:
+        return order, nb, csum
+    reach = np.nonzero(csum >= p)[0]
+    k_star = int(reach[0]) + 1 if reach.size else nb
+    return order, k_star, csum
+
+
+def _frames_of_block(j: int, S: int, block: int, frame_len: int):
+    lo = j * block
+    hi = min(S, (j + 1) * block) - 1
+    return lo // frame_len, hi // frame_len
+
+
+def frame_incidence(S: int, block: int, frame_len: int) -> np.ndarray:
+    """Boolean [F, nb]: entry (f, j) is true when key block j holds a valid token of frame f."""
+    nb = -(-S // block)
+    F = -(-S // frame_len)
+    inc = np.zeros((F, nb), dtype=bool)
+    for j in range(nb):
+        f0, f1 = _frames_of_block(j, S, block, frame_len)
+        inc[f0:f1 + 1, j] = True
+    return inc
+
+
+def _blocks_touching_frames(frames_sel: np.ndarray, inc: np.ndarray) -> np.ndarray:
+    """Key blocks whose valid tokens intersect any selected frame (boolean [nb])."""
+    return inc[np.asarray(frames_sel, dtype=bool)].any(axis=0)
+
+
+def forced_blocks(S: int, cfg: RouteCfg) -> np.ndarray:
+    """Mandatory key blocks for every query block, boolean [nb, nb] (same for all heads).
+
+    Union of: the diagonal; the band |i-j| <= local_window (wzjinhao notes §5.2); the blocks
+    of the frames within +-frame_window of the query block's frames, and of frame 0
+    (Sol-Attn §2.2: neighbouring frames and the first frame are always kept).
+    """
+    bs = cfg.block
+    nb = -(-S // bs)
+    forced = np.zeros((nb, nb), dtype=bool)
+    inc = frame_incidence(S, bs, cfg.frame_len) if cfg.frame_len > 0 else None
+    for i in range(nb):
+        if cfg.force_diag:
+            forced[i, i] = True
+        if cfg.local_window > 0:
+            lo, hi = max(0, i - cfg.local_window), min(nb - 1, i + cfg.local_window)
+            forced[i, lo:hi + 1] = True
+        if cfg.frame_len > 0 and (cfg.frame_window >= 0 or cfg.force_first_frame):
+            F = -(-S // cfg.frame_len)
+            fsel = np.zeros(F, dtype=bool)
+            f0, f1 = _frames_of_block(i, S, bs, cfg.frame_len)
+            if cfg.frame_window >= 0:
+                fsel[max(0, f0 - cfg.frame_window):min(F - 1, f1 + cfg.frame_window) + 1] = True
+            if cfg.force_first_frame:
+                fsel[0] = True
+            forced[i] |= _blocks_touching_frames(fsel, inc)
+    return forced
+
+
+def frame_topk_select(qf: np.ndarray, kf: np.ndarray, S: int, cfg: RouteCfg, scale: float):
+    """Frame-level top-k (Sol-Attn §2.1/§2.2): score every key frame against each query
+    frame with the frame means, keep the k best (ties to the lower frame index), and expand
+    to key blocks. A query block takes the union over the frames its tokens touch.
+
+    qf, kf: [BH, F, d]. Returns (mask [BH, nb, nb] bool without forcing, frame_scores
+    [BH, F, F], chosen [BH, F, F] bool).
+    """
+    BH, F, _ = qf.shape
+    bs = cfg.block
+    nb = -(-S // bs)
+    fs = np.matmul(qf, np.swapaxes(kf, -1, -2)) * scale
+    k = min(cfg.topk_frames, F)
+    chosen = np.zeros((BH, F, F), dtype=bool)
+    for bh in range(BH):
+        for f in range(F):
+            order = np.argsort(-fs[bh, f], kind="stable")
+            chosen[bh, f, order[:k]] = True
+    inc = frame_incidence(S, bs, cfg.frame_len)
+    mask = np.zeros((BH, nb, nb), dtype=bool)
+    for bh in range(BH):
+        for i in range(nb):
+            f0, f1 = _frames_of_block(i, S, bs, cfg.frame_len)
+            fsel = chosen[bh, f0:f1 + 1].any(axis=0)
+            mask[bh, i] = _blocks_touching_frames(fsel, inc)
+    return mask, fs, chosen
+
+
+def route(Q, K, cfg: RouteCfg):
+    """The whole router on [BH, S, d] inputs. Returns a dict with
+    mask [BH, nb, nb] (the final selection: routed set union forced set), routed (the set
+    before forcing), forced [nb, nb], pi or frame scores, and near_tie [BH, nb]."""
+    Q = _f64(Q)
+    K = _f64(K)
+    BH, S, d = Q.shape
+    bs = cfg.block
+    nb = -(-S // bs)
+    scale = cfg.scale if cfg.scale is not None else 1.0 / math.sqrt(d)
+    forced = forced_blocks(S, cfg)
+    out = {"forced": forced, "nb": nb, "scale": scale}
+    if cfg.mode == "topp":
+        qbar, kbar = pool_blocks(Q, bs), pool_blocks(K, bs)
+        pi = row_softmax(block_scores(qbar, kbar, scale))
+        routed = np.zeros((BH, nb, nb), dtype=bool)
+        kstar = np.zeros((BH, nb), dtype=np.int64)
+        for bh in range(BH):
+            for i in range(nb):
+                order, ks, _ = topp_row(pi[bh, i], cfg.p)
+                routed[bh, i, order[:ks]] = True
+                kstar[bh, i] = ks
+        out.update(pi=pi, kstar=kstar, qbar=qbar, kbar=kbar)
+    elif cfg.mode == "frame_topk":
+        qf, kf = pool_frames(Q, cfg.frame_len), pool_frames(K, cfg.frame_len)
+        routed, fs, chosen = frame_topk_select(qf, kf, S, cfg, scale)
+        out.update(frame_scores=fs, chosen=chosen)
+    else:
+        raise ValueError(cfg.mode)
+    out["routed"] = routed
+    out["mask"] = routed | forced[None]
+    out["near_tie"] = near_tie_rows(out, S, cfg)
+    return out
+
+
+def near_tie_rows(r: dict, S: int, cfg: RouteCfg) -> np.ndarray:
+    """Rows whose selection is decided by a difference below the stated resolution:
+    a cumulative mass within EPS_MASS of p at the cut (k* or k*-1 blocks), or a probability
+    gap under EPS_GAP between the last block kept and the first block left out. In frame
+    mode: a score gap under EPS_GAP at the top-k boundary of any frame the row touches."""
+    mask = r["mask"]
+    BH, nb, _ = mask.shape
+    near = np.zeros((BH, nb), dtype=bool)
+    if cfg.mode == "topp":
+        if cfg.p >= 1.0:
+            return near
+        pi = r["pi"]
+        for bh in range(BH):
+            for i in range(nb):
+                order, ks, csum = topp_row(pi[bh, i], cfg.p)
+                srt = pi[bh, i][order]
+                t = abs(csum[ks - 1] - cfg.p) < EPS_MASS
+                if ks >= 2:
+                    t |= abs(csum[ks - 2] - cfg.p) < EPS_MASS
+                if ks < srt.shape[0]:
+                    t |= (srt[ks - 1] - srt[ks]) < EPS_GAP
+                near[bh, i] = t
+        return near
+    fs = r["frame_scores"]
+    F = fs.shape[1]
+    k = min(cfg.topk_frames, F)
+    ftie = np.zeros((BH, F), dtype=bool)
+    if k < F:
+        for bh in range(BH):
+            for f in range(F):
+                srt = np.sort(fs[bh, f])[::-1]
+                ftie[bh, f] = (srt[k - 1] - srt[k]) < EPS_GAP
+    for i in range(nb):
+        f0, f1 = _frames_of_block(i, S, cfg.block, cfg.frame_len)
+        near[:, i] = ftie[:, f0:f1 + 1].any(axis=1)
+    return near
+
+
+def valid_near_tie_set(r: dict, bh: int, i: int, gpu_row: np.ndarray, S: int, cfg: RouteCfg) -> bool:
+    """Is `gpu_row` (boolean [nb]) an acceptable selection for a near-tie row?
+
+    It must hold every forced block and every block clearly above the cut, hold nothing
+    clearly below it, and (Top-p) reach mass p - EPS_MASS."""
+    forced = r["forced"][i]
+    gpu_row = np.asarray(gpu_row, dtype=bool)
+    if np.any(forced & ~gpu_row):
+        return False
+    if cfg.mode == "topp":
+        pi = r["pi"][bh, i]
+        order, ks, csum = topp_row(pi, cfg.p)
+        srt = pi[order]
+        hi_cut = srt[ks - 1]
+        lo_cut = srt[ks] if ks < pi.shape[0] else -np.inf
+        must = (pi > hi_cut + EPS_GAP) | forced
+        may = (pi >= lo_cut - EPS_GAP) | forced
+        if pi[gpu_row].sum() < cfg.p - EPS_MASS:
+            return False
+    else:
+        fs = r["frame_scores"][bh]
+        F = fs.shape[0]
+        k = min(cfg.topk_frames, F)
+        f0, f1 = _frames_of_block(i, S, cfg.block, cfg.frame_len)
+        fm = np.zeros(F, dtype=bool)
+        fy = np.zeros(F, dtype=bool)
+        for f in range(f0, f1 + 1):
+            srt = np.sort(fs[f])[::-1]
+            hi_cut = srt[k - 1]
+            lo_cut = srt[k] if k < F else -np.inf
+            fm |= fs[f] > hi_cut + EPS_GAP
+            fy |= fs[f] >= lo_cut - EPS_GAP
+        inc = frame_incidence(S, cfg.block, cfg.frame_len)
+        must = _blocks_touching_frames(fm, inc) | forced
+        may = _blocks_touching_frames(fy, inc) | forced
+    return bool(np.all(gpu_row[must]) and not np.any(gpu_row & ~may))

@@ -1,0 +1,289 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself: closed forms,
+hand-computed golden cases, brute force over all subsets, invariants and a library
+routine (torch's scaled_dot_product_attention). CPU only."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.route import EPS_GAP, EPS_MASS
+from workloads import get_workload, make_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- pooling (closed forms)
+
+def test_pool_ramp_closed_form_with_ragged_tail():
+    # X[t, c] = t + 1000 c: the mean of tokens lo..hi-1 is (lo + hi - 1)/2 + 1000 c.
+    S, d = 200, 3
+    X = (np.arange(S)[:, None] + 1000.0 * np.arange(d)[None, :])[None]
+    m = oracle.pool_blocks(X, 64)
+    assert m.shape == (1, 4, d)
+    for i, (lo, hi) in enumerate([(0, 64), (64, 128), (128, 192), (192, 200)]):
+        np.testing.assert_array_equal(m[0, i], (lo + hi - 1) / 2 + 1000.0 * np.arange(d))
+
+
+def test_pool_constant_blocks():
+    S, d = 64 * 5, 8
+    X = np.repeat(np.arange(5, dtype=np.float64), 64)[None, :, None] * np.ones((2, 1, d))
+    np.testing.assert_array_equal(oracle.pool_blocks(X, 64)[1, :, 0], np.arange(5.0))
+
+
+def test_pool_frames_closed_form():
+    S, fl = 250, 100
+    X = np.arange(S, dtype=np.float64)[None, :, None]
+    m = oracle.pool_frames(X, fl)[0, :, 0]
+    np.testing.assert_array_equal(m, [49.5, 149.5, 224.5])
+
+
+# ---------------------------------------------------------------- scores and softmax
+
+def test_block_scores_hand():
+    q = np.zeros((1, 2, 4)); k = np.zeros((1, 3, 4))
+    q[0, 0, 0] = 2.0; q[0, 1, 1] = -1.0
+    k[0, 0, 0] = 3.0; k[0, 1, 1] = 5.0; k[0, 2] = 1.0
+    sc = oracle.block_scores(q, k, 0.5)
+    np.testing.assert_array_equal(sc[0], [[3.0, 0.0, 1.0], [0.0, -2.5, -0.5]])
+
+
+def test_softmax_closed_form():
+    pi = oracle.row_softmax(np.log(np.array([[1.0, 2.0, 3.0, 4.0], [1.0, 3.0, 0.0 + 1e-300, 4.0]])))
+    np.testing.assert_allclose(pi[0], [0.1, 0.2, 0.3, 0.4], rtol=1e-15)
+    np.testing.assert_allclose(pi[1], [0.125, 0.375, 0.0, 0.5], atol=1e-15)
+    # shift invariance of the logits
+    x = np.random.default_rng(0).normal(size=(3, 7)) * 50
+    np.testing.assert_allclose(oracle.row_softmax(x), oracle.row_softmax(x + 1234.5), rtol=1e-12)
+
+
+# ---------------------------------------------------------------- Top-p cut
+
+def test_topp_golden_hand_cases():
+    cases = json.load(open(os.path.join(GOLDEN, "topp_hand_cases.json")))["cases"]
+    for c in cases:
+        pi = oracle.row_softmax(np.log(np.array(c["w"], dtype=np.float64))[None])[0]
+        order, ks, _ = oracle.topp_row(pi, c["p"])
+        assert sorted(order[:ks].tolist()) == c["expect"], c
+
+
+def _brute_force_min_set(pi, p):
+    """Smallest cardinality of any subset with mass >= p, and the best mass at that size."""
+    n = pi.shape[0]
+    for k in range(1, n + 1):
+        best = max(sum(pi[list(s)]) for s in itertools.combinations(range(n), k))
+        if best >= p:
+            return k, best
+    return n, pi.sum()
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topp_minimal_prefix_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(2, 11))
+    pi = oracle.row_softmax(rng.normal(size=n) * rng.uniform(0.3, 3.0))
+    for p in (0.2, 0.5, 0.8, 0.9, 0.97):
+        order, ks, csum = oracle.topp_row(pi, p)
+        kmin, best = _brute_force_min_set(pi, p)
+        if abs(csum[ks - 1] - p) < 1e-12 or abs(best - p) < 1e-12:
+            continue
+        assert ks == kmin
+        assert abs(pi[order[:ks]].sum() - best) < 1e-12     # the prefix is a best set of that size
+
+
+def test_topp_degenerate_rows():
+    nb = 16
+    one_hot = np.zeros(nb); one_hot[5] = 1.0
+    order, ks, _ = oracle.topp_row(one_hot, 0.9)
+    assert ks == 1 and order[0] == 5
+    uni = np.full(nb, 1.0 / nb)
+    assert oracle.topp_row(uni, 0.5)[1] == nb // 2
+    assert oracle.topp_row(uni, 1.0)[1] == nb
+    assert oracle.topp_row(uni, 1e-9)[1] == 1
+
+
+def test_topp_nested_in_p():
+    rng = np.random.default_rng(7)
+    pi = oracle.row_softmax(rng.normal(size=40) * 2.0)
+    prev = set()
+    for p in (0.1, 0.3, 0.5, 0.8, 0.9, 0.95, 0.99, 1.0):
+        order, ks, _ = oracle.topp_row(pi, p)
+        cur = set(order[:ks].tolist())
+        assert prev <= cur
+        prev = cur
+    assert prev == set(range(40))
+
+
+def test_near_tie_flags():
+    cfg = oracle.RouteCfg(p=0.9)
+    # cut exactly at p: masses .5 .4 .1 -> c_2 = .9 (within EPS_MASS of p)
+    r = {"pi": np.array([[[0.5, 0.4, 0.1]]]), "mask": np.ones((1, 1, 3), bool), "forced": np.eye(1, 3, dtype=bool)}
+    assert oracle.near_tie_rows(r, 64 * 3, cfg)[0, 0]
+    # clear cut, no tie
+    r["pi"] = np.array([[[0.7, 0.05, 0.25]]])
+    assert not oracle.near_tie_rows(r, 64 * 3, cfg)[0, 0]
+    # probability gap below EPS_GAP at the boundary
+    r["pi"] = np.array([[[0.85, 0.075 + 0.4 * EPS_GAP, 0.075 - 0.4 * EPS_GAP]]])
+    assert oracle.near_tie_rows(r, 64 * 3, cfg)[0, 0]
+
+
+# ---------------------------------------------------------------- forced blocks
+
+def test_forced_diag_and_band_hand():
+    f = oracle.forced_blocks(6 * 64, oracle.RouteCfg(force_diag=True, local_window=1))
+    expect = np.zeros((6, 6), bool)
+    for i in range(6):
+        for j in range(max(0, i - 1), min(5, i + 1) + 1):
+            expect[i, j] = True
+    np.testing.assert_array_equal(f, expect)
+    f0 = oracle.forced_blocks(6 * 64 - 10, oracle.RouteCfg(force_diag=True))
+    np.testing.assert_array_equal(f0, np.eye(6, dtype=bool))
+
+
+def test_forced_frames_golden():
+    cases = json.load(open(os.path.join(GOLDEN, "frame_hand_cases.json")))["cases"]
+    for c in cases:
+        cfg = oracle.RouteCfg(force_diag=False, frame_len=c["frame_len"], frame_window=c["frame_window"],
+                              force_first_frame=c["first"])
+        f = oracle.forced_blocks(c["S"], cfg)
+        assert np.nonzero(f[c["query_block"]])[0].tolist() == c["expect_blocks"], c
+
+
+# ---------------------------------------------------------------- whole router invariants
+
+def _small(name="single", **kw):
+    w = get_workload(name, **kw)
+    x = make_inputs(w)
+    BH = w.B * w.H
+    return w, x["q"].reshape(BH, w.S, w.d), x["k"].reshape(BH, w.S, w.d), x["v"].reshape(BH, w.S, w.d)
+
+
+def test_route_invariants_and_p1_dense():
+    w, Q, K, _ = _small(H=3, S=1000, frame_len=500, region_len=128, seed=11)
+    for cfg in (oracle.RouteCfg(p=0.8, force_diag=True), oracle.RouteCfg(p=0.5, force_diag=False, local_window=2),
+                oracle.RouteCfg(p=0.7, force_diag=True, frame_len=500, frame_window=0, force_first_frame=True)):
+        r = oracle.route(Q, K, cfg)
+        m = r["mask"]
+        assert m.shape == (3, 16, 16)
+        assert (m.sum(axis=2) >= 1).all()
+        assert (m | ~r["forced"][None]).all()                      # forced subset of selected
+        np.testing.assert_array_equal(m, r["routed"] | r["forced"][None])
+        # the routed part has mass >= p in every row
+        mass = (r["pi"] * r["routed"]).sum(axis=2)
+        assert (mass >= cfg.p - 1e-12).all()
+    r1 = oracle.route(Q, K, oracle.RouteCfg(p=1.0, force_diag=False))
+    assert r1["mask"].all()
+
+
+def test_route_selection_nested_in_p():
+    w, Q, K, _ = _small(H=2, S=768, frame_len=256, region_len=64, seed=3, alpha=("const", 0.7))
+    prev = None
+    for p in (0.5, 0.8, 0.9, 0.95, 0.99, 1.0):
+        m = oracle.route(Q, K, oracle.RouteCfg(p=p, force_diag=True))["mask"]
+        if prev is not None:
+            assert (m | ~prev).all()
+        prev = m
+
+
+def test_frame_mode_topk_ge_frames_is_dense():
+    w, Q, K, _ = _small(H=2, S=900, frame_len=300, region_len=100, seed=5)
+    r = oracle.route(Q, K, oracle.RouteCfg(mode="frame_topk", topk_frames=3, frame_len=300, force_diag=False))
+    assert r["mask"].all()
+
+
+def test_frame_mode_aligned_direct_construction():
+    # Frames of 128 tokens = 2 blocks each: a key block is selected iff its frame is one of
+    # the k frames whose mean key scores highest against the query block's frame mean.
+    w, Q, K, _ = _small(H=2, S=1024, frame_len=128, region_len=64, seed=9)
+    cfg = oracle.RouteCfg(mode="frame_topk", topk_frames=2, frame_len=128, force_diag=False)
+    r = oracle.route(Q, K, cfg)
+    Qd, Kd = Q.double().numpy(), K.double().numpy()
+    F, nb = 8, 16
+    for bh in range(2):
+        qm = [Qd[bh, f * 128:(f + 1) * 128].mean(axis=0) for f in range(F)]
+        km = [Kd[bh, f * 128:(f + 1) * 128].mean(axis=0) for f in range(F)]
+        for i in range(nb):
+            f = i // 2
+            s = [float(np.dot(qm[f], km[g])) for g in range(F)]
+            top = sorted(range(F), key=lambda g: (-s[g], g))[:2]
+            expect = np.array([(j // 2) in top for j in range(nb)])
+            np.testing.assert_array_equal(r["mask"][bh, i], expect)
+
+
+def test_valid_near_tie_set_accepts_neighbours_and_rejects_far():
+    cfg = oracle.RouteCfg(p=0.9, force_diag=True)
+    pi = np.array([0.5, 0.4 + 2e-6, 0.1 - 2e-6, 0.0])
+    r = {"pi": pi[None, None], "forced": np.eye(4, dtype=bool)[:1], "mask": None}
+    assert oracle.valid_near_tie_set(r, 0, 0, np.array([1, 1, 0, 0], bool), 256, cfg)
+    assert oracle.valid_near_tie_set(r, 0, 0, np.array([1, 1, 1, 0], bool), 256, cfg)
+    assert not oracle.valid_near_tie_set(r, 0, 0, np.array([1, 0, 1, 0], bool), 256, cfg)
+    assert not oracle.valid_near_tie_set(r, 0, 0, np.array([0, 1, 1, 0], bool), 256, cfg)
+
+
+# ---------------------------------------------------------------- attention
+
+def test_attention_full_coverage_equals_dense_sdpa():
+    # The pages' own check (wzjinhao notes §5.3): b,h,l,d = 2,4,512,64, fp32, full coverage
+    # must equal dense attention to max-abs < 1e-4.
+    g = torch.Generator().manual_seed(0)
+    q, k, v = (torch.randn(8, 512, 64, generator=g) for _ in range(3))
+    mask = np.ones((8, 8, 8), bool)
+    o = oracle.attention_sets(q, k, v, mask, 1 / 8.0)
+    dense = torch.nn.functional.scaled_dot_product_attention(q.double(), k.double(), v.double()).numpy()
+    assert np.abs(o - dense).max() < 1e-12
+    dense32 = torch.nn.functional.scaled_dot_product_attention(q, k, v).numpy()
+    assert np.abs(o - dense32).max() < 1e-4
+
+
+def test_attention_single_block_and_tail_equal_sdpa_on_slice():
+    g = torch.Generator().manual_seed(1)
+    S = 200                                   # blocks 0..3, the last with 8 tokens
+    q, k, v = (torch.randn(1, S, 32, dtype=torch.float64, generator=g) for _ in range(3))
+    mask = np.zeros((1, 4, 4), bool)
+    mask[0, 1, 3] = True                      # query block 1 sees only the ragged block 3
+    mask[0, 3, [0, 3]] = True                 # query block 3 sees blocks 0 and 3
+    mask[0, 0, 0] = mask[0, 2, 2] = True
+    o = oracle.attention_sets(q, k, v, mask, 0.3)
+    sd = torch.nn.functional.scaled_dot_product_attention
+    ref1 = sd(q[:, 64:128], k[:, 192:200], v[:, 192:200], scale=0.3)
+    np.testing.assert_allclose(o[0, 64:128], ref1[0].numpy(), atol=1e-13)
+    cols = torch.cat([torch.arange(0, 64), torch.arange(192, 200)])
+    ref3 = sd(q[:, 192:200], k[:, cols], v[:, cols], scale=0.3)
+    np.testing.assert_allclose(o[0, 192:200], ref3[0].numpy(), atol=1e-13)
+
+
+def test_attention_gather_equals_token_mask():
+    w, Q, K, V = _small(H=2, S=700, frame_len=350, region_len=64, seed=2)
+    rng = np.random.default_rng(4)
+    nb = 11
+    mask = rng.random((2, nb, nb)) < 0.3
+    mask[:, np.arange(nb), np.arange(nb)] = True
+    a = oracle.attention_sets(Q, K, V, mask, 0.1)
+    b = oracle.attention_token_mask(Q, K, V, mask, 0.1)
+    assert np.abs(a - b).max() < 1e-12
+
+
+# ---------------------------------------------------------------- bookkeeping
+
+def test_csr_loads_tiles_lpt_hand():
+    m = np.zeros((2, 3, 3), bool)
+    m[0, 0, [0, 2]] = True; m[0, 1, [1]] = True; m[0, 2, [0, 1, 2]] = True
+    m[1, 0, [0]] = True; m[1, 1, [0, 1]] = True; m[1, 2, [2]] = True
+    rp, ci = oracle.csr_from_mask(m)
+    assert rp.tolist() == [0, 2, 3, 6, 7, 9, 10]
+    assert ci.tolist() == [0, 2, 1, 0, 1, 2, 0, 0, 1, 2]
+    assert oracle.head_loads(m).tolist() == [6, 4]
+    c = oracle.tile_costs(m)                  # tiles: (0,1) and (2,) per head
+    assert c.tolist() == [[3, 3], [2, 1]]
+    assert oracle.lpt_order(c).tolist() == [0, 1, 2, 3]
+    assert oracle.lpt_order(np.array([[1, 5], [5, 2]])).tolist() == [1, 2, 3, 0]
+
+
+def test_selected_flops_hand():
+    m = np.zeros((1, 2, 2), bool)
+    m[0, 0, 1] = True; m[0, 1, 1] = True     # S = 100: block 0 = 64 tokens, block 1 = 36
+    assert oracle.selected_flops(m, 100, 64, 16) == 4 * 16 * (64 * 36 + 36 * 36)
