@@ -1,0 +1,383 @@
+"""Benchmark of one video-DiT attention layer: Top-p block routing + block-sparse attention.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dit] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one synthetic layer already resident in HBM:
+fvattn_route (pool -> fp64 scores/softmax/Top-p -> CSR, loads, tile order) followed by
+fvattn_sparse_attn. The layer is B=1, H=40, S=32760 (21 frames x 1560 tokens), d=128, bf16,
+block 64, p=0.9 with the diagonal forced; inputs (1 GB of Q, K, V) are larger than L2.
+
+`value` is the effective TFLOPS of the step: attention FLOPs of the selected blocks only
+(4*d per selected query/key token pair) divided by the step time. With N GPUs every rank runs
+its own layer (weak scaling, no collective on the data path); the time is the max over ranks.
+
+--impl reference times the CPU oracle (fp64 NumPy) on a bounded sample of the same layer.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "block-sparse attn effective TFLOPS & ms per layer at S=32760,H=40,p=0.9; % bf16 peak"
+UNIT = "TFLOPS"
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in FALLBACK}, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def env_rank():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def workload_desc(w) -> str:
+    return (f"{w.name}: B={w.B},H={w.H},S={w.S} ({w.frames} frames x {w.frame_len} tokens),d={w.d},{w.dtype},"
+            f"block=64,p={w.p},diag forced")
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(suffix=".csv")
+        self.proc = None
+        self.gpu = gpu_index
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ FLOP / byte accounting
+
+def selected_flops_from_csr(csr, S: int, d: int):
+    """4*d*sum over selected (query block i, key block j) of valid-token counts n_i*n_j."""
+    import torch
+    nb = csr.nb
+    n = torch.full((nb,), 64, dtype=torch.int64, device=csr.row_ptr.device)
+    n[-1] = S - 64 * (nb - 1)
+    rp = csr.row_ptr.long()
+    nnz = int(csr.nnz.item())
+    counts = rp[1:] - rp[:-1]
+    rows = torch.repeat_interleave(torch.arange(counts.numel(), device=rp.device), counts)
+    qi = rows % nb
+    kj = csr.col_idx[:nnz].long()
+    pairs = int((n[qi] * n[kj]).sum().item())
+    padded = int(counts.sum().item()) * 64 * 64
+    kv_tokens = int(n[kj].sum().item())
+    return 4 * d * pairs, nnz, 4 * d * padded, kv_tokens
+
+
+def router_bytes(BH: int, S: int, d: int, esize: int, nb: int, nnz: int) -> int:
+    nt = BH * ((nb + 1) // 2)
+    return 2 * BH * S * d * esize + 4 * (BH * nb + 1) + 4 * nnz + 8 * BH + 8 * nt + 8
+
+
+def traffic_from_profile(kernel_src: str):
+    """dram bytes per launch of the attention kernel from the committed ncu summary, if it was
+    taken on the current source of the kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", "attn_tc_dit_layer.traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    h = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    if d.get("source_sha256_16") != h:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+def cpu_oracle_run(w, q_cpu, k_cpu, v_cpu, n_items: int, seed: int = 0):
+    """Time the oracle (as it stands) on a bounded sample of the layer: the full router on
+    `heads` heads and exact attention for `n_items` query blocks of those heads. Returns
+    (estimated seconds for the whole layer, sample description, threads used, sample FLOPs)."""
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    BH = w.B * w.H
+    heads = min(BH, 4)
+    Q = q_cpu.reshape(BH, w.S, w.d)[:heads]
+    K = k_cpu.reshape(BH, w.S, w.d)[:heads]
+    V = v_cpu.reshape(BH, w.S, w.d)[:heads]
+    cfg = oracle.RouteCfg(p=w.p, force_diag=True)
+    t0 = time.perf_counter()
+    r = oracle.route(Q, K, cfg)
+    t_route = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    items = [(int(b), int(i)) for b, i in zip(rng.integers(0, heads, n_items), rng.integers(0, w.nb, n_items))]
+    t0 = time.perf_counter()
+    oracle.attention_rows(Q, K, V, r["mask"], 1.0 / math.sqrt(w.d), items)
+    t_attn = time.perf_counter() - t0
+    # scale: router time per head x BH; attention time per sampled block x all blocks of the layer,
+    # weighted by the selected-FLOP share of the sample
+    flops_heads = oracle.selected_flops(r["mask"], w.S, 64, w.d)
+    nrow = np.array([min(w.S, (i + 1) * 64) - i * 64 for i in range(w.nb)])
+    f_items = sum(4 * w.d * int(nrow[i]) * int(nrow[r["mask"][b, i]].sum()) for b, i in items)
+    est_layer_flops = flops_heads * BH / heads
+    t_layer = t_route * BH / heads + t_attn * (est_layer_flops / max(f_items, 1))
+    desc = (f"oracle router on {heads}/{BH} heads ({t_route:.1f} s) + exact attention of {n_items} sampled query "
+            f"blocks ({t_attn:.1f} s), scaled to the whole layer by heads and by selected-FLOP share")
+    return t_layer, desc, threads, est_layer_flops
+
+
+def run_reference(args, w):
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return 0
+    import torch
+    from workloads import make_inputs
+    x = make_inputs(w.replace(H=4), device="cpu")      # the sample's heads (same per-head generator)
+    times = []
+    flops = None
+    desc = threads = None
+    for s in range(args.warmup + args.steps):
+        t_layer, desc, threads, flops = cpu_oracle_run(w.replace(H=4), x["q"], x["k"], x["v"], n_items=8, seed=s)
+        t_layer *= w.H / 4
+        if s >= args.warmup:
+            times.append(t_layer)
+    flops = flops * w.H / 4
+    t = statistics.median(times)
+    value = flops / t / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(w), "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_ours(args, w):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_top_fvattn_b200 as fv
+    from workloads import make_inputs
+
+    rank, world, local = env_rank()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    fv.load()
+    pk, pk_src = peaks()
+
+    # every rank draws its own layer (weak scaling): seed offset by rank
+    x = make_inputs(w, device=dev, seed=w.seed + 1000 * rank)
+    q, k, v = x["q"], x["k"], x["v"]
+    B, H, S, d = q.shape
+    BH = B * H
+    cfg = fv.RouteConfig(p=w.p, force_diag=True)
+    csr = fv.alloc_csr(B, H, S, dev)
+    ws = torch.empty(fv.workspace_bytes(q, cfg), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        fv.route(q, k, cfg, csr=csr, workspace=ws)
+        fv.sparse_attn(q, k, v, csr, out=out)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if fv.read_status(csr) != 0:
+        raise RuntimeError(f"device status {fv.read_status(csr)}")
+    flops, nnz, flops_padded, kv_tokens = selected_flops_from_csr(csr, S, d)
+    density = nnz / (BH * csr.nb * csr.nb)
+
+    # timed region: K steps; per-kernel events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        ev[s][0].record(stream)
+        fv.route(q, k, cfg, csr=csr, workspace=ws)
+        ev[s][1].record(stream)
+        fv.sparse_attn(q, k, v, csr, out=out)
+        ev[s][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    route_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.steps)]
+    attn_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(args.steps)]
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+        ft = torch.tensor([float(flops)], device=dev, dtype=torch.float64)
+        dist.all_reduce(ft, op=dist.ReduceOp.SUM)
+        flops_all = float(ft.item())
+    else:
+        flops_all = float(flops)
+    ms_step = total_ms / args.steps
+    value = flops_all * args.steps / (total_ms * 1e-3) / 1e12
+    attn_avg = statistics.mean(attn_ms)
+    route_avg = statistics.mean(route_ms)
+    attn_tflops = flops / (attn_avg * 1e-3) / 1e12
+    rbytes = router_bytes(BH, S, d, q.element_size(), csr.nb, nnz)
+    router_gbs = rbytes / (route_avg * 1e-3) / 1e9
+    traffic = traffic_from_profile(os.path.join(ROOT, "block_sparse_top_fvattn_b200", "csrc", "attn_tc.cu"))
+
+    # end to end through the public API with host buffers (pinned), copies inside the region
+    e2e = None
+    if rank == 0 or world > 1:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        n_e2e = max(2, min(5, args.steps))
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            fv.route(dq, dk, cfg, csr=csr, workspace=ws)
+            fv.sparse_attn(dq, dk, dv, csr, out=out)
+            ho.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / n_e2e
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": flops_all / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+               "d2h_bytes_per_step": out.numel() * out.element_size()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_layer, desc, threads, _ = cpu_oracle_run(w, q.cpu(), k.cpu(), v.cpu(), n_items=12)
+        cpu = {"value": flops / t_layer / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    bf16_peak = pk["bf16_tflops_sustained"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "l2": "inputs larger than L2 (Q,K,V = 1.0 GB per layer)",
+                   "parallelism": f"independent layer per GPU x{world}"},
+        "route_ms": route_avg, "attn_ms": attn_avg, "attn_tflops": attn_tflops,
+        "pct_bf16_peak": 100.0 * value / pk["bf16_tflops"],
+        "pct_bf16_peak_attn": 100.0 * attn_tflops / pk["bf16_tflops"],
+        "density": density, "selected_flops_per_layer": flops, "padded_tile_flops_per_layer": flops_padded,
+        "selected_kv_tokens_per_s": kv_tokens / (attn_avg * 1e-3),
+        "query_tokens_per_s": BH * S / (ms_step * 1e-3),
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": attn_tflops, "peak": bf16_peak,
+                     "unit": "TFLOP/s", "frac": attn_tflops / bf16_peak, "traffic": traffic,
+                     "peak_kind": f"bf16 sustained ({pk_src})",
+                     "frac_of_burst": attn_tflops / pk["bf16_tflops"]},
+        "roofline_router": {"bound": "hbm", "achieved": router_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                            "frac": router_gbs / pk["hbm_gbs"], "algorithmic_bytes": rbytes,
+                            "peak_kind": f"hbm copy ({pk_src})"},
+        "e2e": e2e, "cpu_baseline": cpu,
+        "gpu_launches": 5 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="dit")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    from workloads import get_workload
+    w = get_workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

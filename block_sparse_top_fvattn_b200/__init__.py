@@ -1,0 +1,179 @@
+"""Top-p block routing and block-sparse attention for video-DiT layers on B200 (sm_100a).
+
+Thin Python binding of libfvattn.so (include/fvattn.h). PyTorch supplies device memory and
+the current stream; every step of the computation runs in the library's CUDA kernels.
+There is no CPU or library fallback: if the library is missing, the first call raises.
+
+    csr = route(q, k, p=0.9)                 # q, k: [B, H, S, d] CUDA tensors
+    o = sparse_attn(q, k, v, csr)
+
+Method (FVAttn blog summary, section "AI视频生成的阿喀琉斯之踵"): per 64-token query block,
+keep the smallest descending-importance set of key blocks whose cumulative softmax mass of
+mean-pooled block scores reaches p, then attend exactly over the kept blocks only.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import (FVATTN_BF16, FVATTN_F32, FVATTN_MODE_FRAME_TOPK, FVATTN_MODE_TOPP, FvattnError, check,
+                   load, status_string)
+
+__all__ = ["RouteConfig", "CsrBuffers", "alloc_csr", "route", "sparse_attn", "block_means", "read_status",
+           "workspace_bytes", "shape_of", "load", "FvattnError", "status_string"]
+
+BLOCK = 64
+
+
+@dataclasses.dataclass
+class RouteConfig:
+    """Mirror of fvattn_route_cfg (see include/fvattn.h for the meaning of each field)."""
+    mode: str = "topp"            # "topp" | "frame_topk"
+    p: float = 0.9
+    force_diag: bool = True
+    local_window: int = 0
+    frame_len: int = 0
+    topk_frames: int = 0
+    frame_window: int = -1
+    force_first_frame: bool = False
+
+    def to_c(self) -> _lib.RouteCfg:
+        mode = {"topp": FVATTN_MODE_TOPP, "frame_topk": FVATTN_MODE_FRAME_TOPK}[self.mode]
+        return _lib.RouteCfg(mode, float(self.p), int(self.force_diag), int(self.local_window), int(self.frame_len),
+                             int(self.topk_frames), int(self.frame_window), int(self.force_first_frame))
+
+
+@dataclasses.dataclass
+class CsrBuffers:
+    """Router outputs (device tensors) in the layout of fvattn_csr."""
+    row_ptr: torch.Tensor      # int32 [BH*nb + 1]
+    col_idx: torch.Tensor      # int32 [BH*nb*nb]
+    head_load: torch.Tensor    # int64 [BH]
+    tile_cost: torch.Tensor    # int32 [BH*ceil(nb/2)]
+    tile_order: torch.Tensor   # int32 [BH*ceil(nb/2)]
+    nnz: torch.Tensor          # int64 [1]
+    status: torch.Tensor       # int32 [4]
+    B: int
+    H: int
+    S: int
+
+    @property
+    def nb(self) -> int:
+        return -(-self.S // BLOCK)
+
+    def to_c(self) -> _lib.Csr:
+        return _lib.Csr(self.row_ptr.data_ptr(), self.col_idx.data_ptr(), self.col_idx.numel(),
+                        self.head_load.data_ptr(), self.tile_cost.data_ptr(), self.tile_order.data_ptr(),
+                        self.nnz.data_ptr(), self.status.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return FVATTN_BF16
+    if t.dtype == torch.float32:
+        return FVATTN_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; bf16 or fp32")
+
+
+def shape_of(q: torch.Tensor, scale: float = 0.0) -> _lib.Shape:
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, S, d]")
+    B, H, S, d = q.shape
+    return _lib.Shape(B, H, S, d, BLOCK, _dtype_code(q), float(scale))
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_tensor(t: torch.Tensor, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous [B, H, S, d]")
+
+
+def alloc_csr(B: int, H: int, S: int, device="cuda") -> CsrBuffers:
+    nb = -(-S // BLOCK)
+    nt = B * H * (-(-nb // 2))
+    i32, i64 = torch.int32, torch.int64
+    return CsrBuffers(
+        row_ptr=torch.empty(B * H * nb + 1, dtype=i32, device=device),
+        col_idx=torch.empty(B * H * nb * nb, dtype=i32, device=device),
+        head_load=torch.empty(B * H, dtype=i64, device=device),
+        tile_cost=torch.empty(nt, dtype=i32, device=device),
+        tile_order=torch.empty(nt, dtype=i32, device=device),
+        nnz=torch.empty(1, dtype=i64, device=device),
+        status=torch.zeros(4, dtype=i32, device=device),
+        B=B, H=H, S=S)
+
+
+def workspace_bytes(q: torch.Tensor, cfg: RouteConfig) -> int:
+    n = load().fvattn_route_workspace_bytes(ctypes.byref(shape_of(q)), ctypes.byref(cfg.to_c()))
+    if n == 0:
+        raise FvattnError(_lib.FVATTN_ERR_INVALID, "fvattn_route_workspace_bytes")
+    return int(n)
+
+
+def route(q: torch.Tensor, k: torch.Tensor, cfg: Optional[RouteConfig] = None, *, p: Optional[float] = None,
+          csr: Optional[CsrBuffers] = None, workspace: Optional[torch.Tensor] = None,
+          stream: Optional[torch.cuda.Stream] = None, scale: float = 0.0) -> CsrBuffers:
+    """Run fvattn_route on the current (or given) stream. Returns the CSR buffers."""
+    cfg = cfg or RouteConfig()
+    if p is not None:
+        cfg = dataclasses.replace(cfg, p=p)
+    _check_tensor(q, "q")
+    _check_tensor(k, "k")
+    if k.shape != q.shape or k.dtype != q.dtype:
+        raise ValueError("q and k must have the same shape and dtype")
+    B, H, S, _ = q.shape
+    if csr is None:
+        csr = alloc_csr(B, H, S, q.device)
+    shp = shape_of(q, scale)
+    c_cfg = cfg.to_c()
+    nws = workspace_bytes(q, cfg)
+    if workspace is None or workspace.numel() < nws:
+        workspace = torch.empty(nws, dtype=torch.uint8, device=q.device)
+    c_csr = csr.to_c()
+    check(load().fvattn_route(q.data_ptr(), k.data_ptr(), ctypes.byref(shp), ctypes.byref(c_cfg),
+                              ctypes.byref(c_csr), workspace.data_ptr(), nws, _stream(stream)), "fvattn_route")
+    csr._workspace = workspace      # keep the scratch alive until the kernels have run
+    return csr
+
+
+def sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, csr: CsrBuffers, *,
+                out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None, scale: float = 0.0) -> torch.Tensor:
+    """Run fvattn_sparse_attn: exact attention over the routed key blocks. Returns O."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_tensor(t, n)
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k, v must have the same shape and dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    shp = shape_of(q, scale)
+    c_csr = csr.to_c()
+    check(load().fvattn_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(shp), ctypes.byref(c_csr),
+                                    out.data_ptr(), lse.data_ptr() if lse is not None else None, _stream(stream)),
+          "fvattn_sparse_attn")
+    return out
+
+
+def block_means(x: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """fp64 means of every 64-token block of x ([B, H, S, d]) over its valid tokens."""
+    _check_tensor(x, "x")
+    B, H, S, d = x.shape
+    out = torch.empty((B, H, -(-S // BLOCK), d), dtype=torch.float64, device=x.device)
+    check(load().fvattn_block_means(x.data_ptr(), ctypes.byref(shape_of(x)), out.data_ptr(), _stream(stream)),
+          "fvattn_block_means")
+    return out
+
+
+def read_status(csr: CsrBuffers, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronise the stream and return the device status word (0 = ok)."""
+    return int(load().fvattn_read_status(ctypes.byref(csr.to_c()), _stream(stream)))

@@ -1,0 +1,87 @@
+"""ctypes view of libfvattn.so (the C ABI of include/fvattn.h). Marshalling only."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfvattn.so")
+
+FVATTN_OK = 0
+FVATTN_ERR_INVALID = -1
+FVATTN_ERR_UNSUPPORTED = -2
+FVATTN_ERR_CAPACITY = -3
+FVATTN_ERR_CUDA = -4
+FVATTN_ERR_TIMEOUT = -5
+
+FVATTN_BF16 = 0
+FVATTN_F32 = 1
+FVATTN_MODE_TOPP = 0
+FVATTN_MODE_FRAME_TOPK = 1
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("S", ctypes.c_int64), ("d", ctypes.c_int64),
+                ("block", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class RouteCfg(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int32), ("p", ctypes.c_float), ("force_diag", ctypes.c_int32),
+                ("local_window", ctypes.c_int32), ("frame_len", ctypes.c_int32), ("topk_frames", ctypes.c_int32),
+                ("frame_window", ctypes.c_int32), ("force_first_frame", ctypes.c_int32)]
+
+
+class Csr(ctypes.Structure):
+    _fields_ = [("row_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p), ("col_capacity", ctypes.c_int64),
+                ("head_load", ctypes.c_void_p), ("tile_cost", ctypes.c_void_p), ("tile_order", ctypes.c_void_p),
+                ("nnz", ctypes.c_void_p), ("status", ctypes.c_void_p)]
+
+
+class FvattnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+        self.code = code
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load the in-tree library. Raises if it has not been built: there is no other path."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with `python -m block_sparse_top_fvattn_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER
+    vp = ctypes.c_void_p
+    lib.fvattn_version.restype = ctypes.c_int
+    lib.fvattn_version.argtypes = []
+    lib.fvattn_status_string.restype = ctypes.c_char_p
+    lib.fvattn_status_string.argtypes = [ctypes.c_int]
+    lib.fvattn_csr_max_nnz.restype = ctypes.c_int64
+    lib.fvattn_csr_max_nnz.argtypes = [P(Shape)]
+    lib.fvattn_num_tiles.restype = ctypes.c_int64
+    lib.fvattn_num_tiles.argtypes = [P(Shape)]
+    lib.fvattn_route_workspace_bytes.restype = ctypes.c_size_t
+    lib.fvattn_route_workspace_bytes.argtypes = [P(Shape), P(RouteCfg)]
+    lib.fvattn_route.restype = ctypes.c_int
+    lib.fvattn_route.argtypes = [vp, vp, P(Shape), P(RouteCfg), P(Csr), vp, ctypes.c_size_t, vp]
+    lib.fvattn_sparse_attn.restype = ctypes.c_int
+    lib.fvattn_sparse_attn.argtypes = [vp, vp, vp, P(Shape), P(Csr), vp, vp, vp]
+    lib.fvattn_block_means.restype = ctypes.c_int
+    lib.fvattn_block_means.argtypes = [vp, P(Shape), vp, vp]
+    lib.fvattn_read_status.restype = ctypes.c_int
+    lib.fvattn_read_status.argtypes = [P(Csr), vp]
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().fvattn_status_string(int(code)).decode()
+
+
+def check(code: int, what: str) -> None:
+    if code != FVATTN_OK:
+        raise FvattnError(code, what)

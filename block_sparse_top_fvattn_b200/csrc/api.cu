@@ -1,0 +1,221 @@
+// Host side of the C ABI declared in include/fvattn.h: argument validation, workspace
+// layout, and the launch sequence of the router and the attention kernels.
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "route.cuh"
+
+using namespace fv;
+
+namespace {
+
+constexpr int kVersion = (1 << 16) | 0;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int validate_shape(const fvattn_shape* s) {
+  if (s == nullptr) return FVATTN_ERR_INVALID;
+  if (s->B < 1 || s->H < 1 || s->S < 1 || s->d < 1) return FVATTN_ERR_INVALID;
+  if (s->dtype != FVATTN_BF16 && s->dtype != FVATTN_F32) return FVATTN_ERR_INVALID;
+  if (!(s->scale >= 0.f) && !(s->scale <= 0.f)) return FVATTN_ERR_INVALID;   // NaN
+  if (isinf(s->scale)) return FVATTN_ERR_INVALID;
+  if (s->block != kBlock) return FVATTN_ERR_UNSUPPORTED;
+  if (s->d != 64 && s->d != 128) return FVATTN_ERR_UNSUPPORTED;
+  if (s->S > (int64_t)1 << 30 || s->B * s->H > 65535) return FVATTN_ERR_UNSUPPORTED;
+  const int64_t nb = (s->S + kBlock - 1) / kBlock;
+  // CSR offsets are int32: the densest selection must fit.
+  if (s->B * s->H * nb * nb >= ((int64_t)1 << 31)) return FVATTN_ERR_UNSUPPORTED;
+  return FVATTN_OK;
+}
+
+int validate_cfg(const fvattn_shape* s, const fvattn_route_cfg* c) {
+  if (c == nullptr) return FVATTN_ERR_INVALID;
+  if (c->mode != FVATTN_MODE_TOPP && c->mode != FVATTN_MODE_FRAME_TOPK) return FVATTN_ERR_INVALID;
+  if (!(c->p > 0.f) || isinf(c->p)) return FVATTN_ERR_INVALID;        // rejects p <= 0 and NaN
+  if (c->local_window < 0 || c->frame_len < 0 || c->frame_window < -1) return FVATTN_ERR_INVALID;
+  if (c->force_diag != 0 && c->force_diag != 1) return FVATTN_ERR_INVALID;
+  if (c->force_first_frame != 0 && c->force_first_frame != 1) return FVATTN_ERR_INVALID;
+  if ((c->frame_window >= 0 || c->force_first_frame) && c->frame_len == 0) return FVATTN_ERR_INVALID;
+  if (c->mode == FVATTN_MODE_FRAME_TOPK) {
+    if (c->frame_len < kBlock || c->topk_frames < 1) return FVATTN_ERR_INVALID;
+    const int64_t F = (s->S + c->frame_len - 1) / c->frame_len;
+    if (F > 128) return FVATTN_ERR_UNSUPPORTED;
+  }
+  return FVATTN_OK;
+}
+
+struct WsLayout {
+  size_t qlo, klo, qhi, khi, qf, kf, bits, counts, total;
+};
+
+size_t take(size_t& off, size_t bytes) {
+  const size_t o = off;
+  off += (bytes + 255) & ~(size_t)255;
+  return o;
+}
+
+WsLayout ws_layout(const Dims& m, int mode) {
+  WsLayout L{};
+  size_t off = 0;
+  const size_t means = (size_t)m.BH * m.nb * m.d * sizeof(double);
+  L.qlo = take(off, means);
+  L.klo = take(off, means);
+  if (mode == FVATTN_MODE_FRAME_TOPK) {
+    L.qhi = take(off, means);
+    L.khi = take(off, means);
+    const size_t fm = (size_t)m.BH * m.F * m.d * sizeof(double);
+    L.qf = take(off, fm);
+    L.kf = take(off, fm);
+  }
+  L.bits = take(off, (size_t)m.BH * m.nb * m.nw * sizeof(uint32_t));
+  L.counts = take(off, (size_t)m.BH * m.nb * sizeof(int32_t));
+  L.total = off;
+  return L;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+double softmax_scale(const fvattn_shape* s) {
+  return s->scale > 0.f ? (double)s->scale : 1.0 / sqrt((double)s->d);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fvattn_version(void) { return kVersion; }
+
+const char* fvattn_status_string(int status) {
+  switch (status) {
+    case FVATTN_OK: return "ok";
+    case FVATTN_ERR_INVALID: return "invalid argument";
+    case FVATTN_ERR_UNSUPPORTED: return "unsupported shape or configuration";
+    case FVATTN_ERR_CAPACITY: return "buffer too small";
+    case FVATTN_ERR_CUDA: return "CUDA error";
+    case FVATTN_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int64_t fvattn_csr_max_nnz(const fvattn_shape* shape) {
+  const int st = validate_shape(shape);
+  if (st != FVATTN_OK) return st;
+  const int64_t nb = (shape->S + kBlock - 1) / kBlock;
+  return shape->B * shape->H * nb * nb;
+}
+
+int64_t fvattn_num_tiles(const fvattn_shape* shape) {
+  const int st = validate_shape(shape);
+  if (st != FVATTN_OK) return st;
+  const int64_t nb = (shape->S + kBlock - 1) / kBlock;
+  return shape->B * shape->H * ((nb + 1) / 2);
+}
+
+size_t fvattn_route_workspace_bytes(const fvattn_shape* shape, const fvattn_route_cfg* cfg) {
+  if (validate_shape(shape) != FVATTN_OK || validate_cfg(shape, cfg) != FVATTN_OK) return 0;
+  const Dims m = make_dims(*shape, cfg->frame_len);
+  return ws_layout(m, cfg->mode).total;
+}
+
+int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const fvattn_route_cfg* cfg,
+                 const fvattn_csr* out, void* workspace, size_t workspace_bytes, fvattn_stream_t stream) {
+  int st = validate_shape(shape);
+  if (st != FVATTN_OK) return st;
+  st = validate_cfg(shape, cfg);
+  if (st != FVATTN_OK) return st;
+  if (Q == nullptr || K == nullptr || out == nullptr || workspace == nullptr) return FVATTN_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(workspace, 256)) return FVATTN_ERR_INVALID;
+  if (!out->row_ptr || !out->col_idx || !out->head_load || !out->tile_cost || !out->tile_order || !out->nnz ||
+      !out->status)
+    return FVATTN_ERR_INVALID;
+  const Dims m = make_dims(*shape, cfg->frame_len);
+  const WsLayout L = ws_layout(m, cfg->mode);
+  if (workspace_bytes < L.total) return FVATTN_ERR_CAPACITY;
+  if (out->col_capacity < m.BH * m.nb * m.nb) return FVATTN_ERR_CAPACITY;
+  const int nsm = num_sms();
+  if (nsm <= 0) return FVATTN_ERR_CUDA;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  double* qlo = reinterpret_cast<double*>(ws + L.qlo);
+  double* klo = reinterpret_cast<double*>(ws + L.klo);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(ws + L.bits);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  const double scale = softmax_scale(shape);
+  ForceCfg fc{cfg->force_diag, cfg->local_window, cfg->frame_len, cfg->frame_window, cfg->force_first_frame};
+
+  if (cudaMemsetAsync(out->status, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
+  cudaError_t e;
+  if (cfg->mode == FVATTN_MODE_TOPP) {
+    e = launch_pool(Q, K, 2, shape->dtype, m, 0, qlo, klo, nullptr, nullptr, nsm, s);
+    if (e == cudaSuccess)
+      e = launch_topp(qlo, klo, m, cfg->p >= 1.f ? 1.0 : (double)cfg->p, scale, fc, bits, counts, out->tile_cost, s);
+  } else {
+    double* qhi = reinterpret_cast<double*>(ws + L.qhi);
+    double* khi = reinterpret_cast<double*>(ws + L.khi);
+    double* qf = reinterpret_cast<double*>(ws + L.qf);
+    double* kf = reinterpret_cast<double*>(ws + L.kf);
+    e = launch_pool(Q, K, 2, shape->dtype, m, cfg->frame_len, qlo, klo, qhi, khi, nsm, s);
+    if (e == cudaSuccess)
+      e = launch_frame(qlo, qhi, klo, khi, qf, kf, m, cfg->frame_len, cfg->topk_frames, scale, fc, bits, counts,
+                       out->tile_cost, s);
+  }
+  if (e == cudaSuccess)
+    e = launch_schedule(counts, out->tile_cost, m, out->row_ptr, out->head_load, out->nnz, out->tile_order,
+                        out->col_capacity, out->status, s);
+  if (e == cudaSuccess) e = launch_csr(bits, out->row_ptr, m, out->col_idx, out->col_capacity, nsm, s);
+  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
+int fvattn_sparse_attn(const void* Q, const void* K, const void* V, const fvattn_shape* shape,
+                       const fvattn_csr* csr, void* O, float* lse, fvattn_stream_t stream) {
+  int st = validate_shape(shape);
+  if (st != FVATTN_OK) return st;
+  if (!Q || !K || !V || !O || !csr || !csr->row_ptr || !csr->col_idx || !csr->tile_order || !csr->status)
+    return FVATTN_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) || (lse && !aligned(lse, 4)))
+    return FVATTN_ERR_INVALID;
+  const Dims m = make_dims(*shape, 0);
+  const float scale = (float)softmax_scale(shape);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (shape->dtype == FVATTN_F32) {
+    e = launch_attn_f32(static_cast<const float*>(Q), static_cast<const float*>(K), static_cast<const float*>(V), m,
+                        scale, csr->row_ptr, csr->col_idx, static_cast<float*>(O), lse, s);
+  } else {
+    const int nsm = num_sms();
+    if (nsm <= 0) return FVATTN_ERR_CUDA;
+    if (cudaMemsetAsync(csr->status + 2, 0, sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
+    e = launch_attn_tc(Q, K, V, m, scale, csr->row_ptr, csr->col_idx, csr->tile_order, csr->status, O, lse, nsm, s);
+  }
+  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
+int fvattn_block_means(const void* X, const fvattn_shape* shape, double* out, fvattn_stream_t stream) {
+  const int st = validate_shape(shape);
+  if (st != FVATTN_OK) return st;
+  if (!X || !out || !aligned(X, 16) || !aligned(out, 8)) return FVATTN_ERR_INVALID;
+  const Dims m = make_dims(*shape, 0);
+  const int nsm = num_sms();
+  if (nsm <= 0) return FVATTN_ERR_CUDA;
+  cudaError_t e = launch_pool(X, nullptr, 1, shape->dtype, m, 0, out, nullptr, nullptr, nullptr, nsm,
+                              reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
+int fvattn_read_status(const fvattn_csr* csr, fvattn_stream_t stream) {
+  if (csr == nullptr || csr->status == nullptr) return FVATTN_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FVATTN_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, csr->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return FVATTN_ERR_CUDA;
+  return v;
+}
+
+}  // extern "C"

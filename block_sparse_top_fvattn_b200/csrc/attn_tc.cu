@@ -1,0 +1,454 @@
+// Block-sparse flash attention on the B200 tensor cores (tcgen05, TMEM, TMA), bf16 inputs,
+// fp32 accumulation.
+//
+// What it computes (FVAttn blog summary, section "AI视频生成的阿喀琉斯之踵"; the masked
+// attention of the wzjinhao.cn notes §5.2): for every query token, exact softmax attention
+// over the tokens (< S) of the key blocks that the router kept for its query block.
+//
+// How: a persistent CTA per SM takes 128-row query tiles (query blocks 2t and 2t+1 of one
+// head) in the router's longest-first order. A tile walks the ascending union of its two
+// block lists; for each key block j:
+//   S = Q K_j^T          tcgen05.mma M=128 N=64 K=d, A and B K-major from shared memory,
+//                        fp32 accumulator in TMEM (double-buffered)
+//   P = exp2(S*c - m)    one thread per row reads its TMEM lane, masks the half-tile whose
+//                        list lacks j and the keys >= S, keeps a running max m that is only
+//                        raised (with a rescale of O in TMEM) when it grows by more than
+//                        2^8, and writes P as bf16 into shared memory in the MMA's layout
+//   O += P V_j           tcgen05.mma M=128 N=d K=64, V MN-major, O accumulated in TMEM
+// Warp roles: warp 0 issues TMA loads (Q once per tile, K_j and V_j into a 4-stage ring),
+// warp 1 allocates TMEM and issues the MMAs, warps 2-5 do softmax and the epilogue.
+// Every mbarrier wait is bounded; a wait that runs out sets an abort flag, every role
+// unwinds, TMEM is freed and FVATTN_ERR_TIMEOUT is written to the device status word.
+#include <cuda.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "route.cuh"
+#include "tc_ptx.cuh"
+
+namespace fv {
+
+namespace {
+
+constexpr int NS = 4;                        // K/V pipeline stages
+constexpr uint32_t kWaitLimit = 1u << 22;    // polls of a bounded wait (seconds, not minutes)
+constexpr float kRescaleLog2 = 8.0f;         // raise the running max only when it grows by > 2^8
+
+template <int D>
+struct TcLayout {
+  static constexpr int kQChunk = kTileRows * 128;     // [128 rows x 64 dims] bf16 = 16 KB
+  static constexpr int kQBytes = (D / 64) * kQChunk;
+  static constexpr int kKVChunk = kBlock * 128;       // [64 rows x 64 dims] bf16 = 8 KB
+  static constexpr int kKBytes = (D / 64) * kKVChunk;
+  static constexpr int kStage = 2 * kKBytes;          // K_j and V_j
+  static constexpr int kPBytes = kTileRows * 128;     // [128 rows x 64 keys] bf16 = 16 KB
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = kQBytes;
+  static constexpr int kOffP = kOffKV + NS * kStage;
+  static constexpr int kOffBar = kOffP + 2 * kPBytes;
+  static constexpr int kBytes = kOffBar + 512;
+  static constexpr uint32_t kTmemCols = 256;          // S[2] at columns 0 and 64, O at 128
+  static constexpr uint32_t kColO = 128;
+};
+
+struct TcBars {
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[NS], kv_empty[NS];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full[2], pv_done[2];
+  uint64_t o_full, o_empty;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Ascending union of the key-block lists of query blocks 2t and 2t+1 of one head, with a
+// 2-bit membership mask (bit 0: block 2t keeps j, bit 1: block 2t+1 keeps j).
+struct PairMerge {
+  const int32_t* ci;
+  int a, ae, b, be;
+  __device__ PairMerge(const int32_t* row_ptr, const int32_t* col_idx, int64_t bh, int t, int nb) {
+    ci = col_idx;
+    const int64_t r0 = bh * nb + 2 * t;
+    a = row_ptr[r0];
+    ae = row_ptr[r0 + 1];
+    if (2 * t + 1 < nb) {
+      b = ae;
+      be = row_ptr[r0 + 2];
+    } else {
+      b = be = 0;
+    }
+  }
+  __device__ __forceinline__ bool next(int& j, int& mask) {
+    if (a >= ae && b >= be) return false;
+    const int ja = a < ae ? ci[a] : 0x7fffffff;
+    const int jb = b < be ? ci[b] : 0x7fffffff;
+    j = min(ja, jb);
+    mask = (ja == j ? 1 : 0) | (jb == j ? 2 : 0);
+    a += (ja == j);
+    b += (jb == j);
+    return true;
+  }
+};
+
+__device__ __forceinline__ void fail(TcBars* bars, int code) {
+  atomicCAS(&bars->abort, 0, code);
+}
+
+// A bounded wait taken by a whole warp with one outcome for all lanes.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+  const bool ok = tc::mbar_wait(bar, parity, abort, kWaitLimit);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// 2^x by the SFU's ex2.approx instruction (flush-to-zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, Dims m, float scale_log2,
+                   const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                   const int32_t* __restrict__ tile_order, int32_t* __restrict__ control,
+                   __nv_bfloat16* __restrict__ O, float* __restrict__ lse) {
+  using L = TcLayout<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  TcBars* bars = reinterpret_cast<TcBars*>(smem + L::kOffBar);
+  unsigned char* sQ = smem + L::kOffQ;
+  unsigned char* sKV = smem + L::kOffKV;
+  unsigned char* sP = smem + L::kOffP;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ntiles = m.BH * m.nt;
+  volatile int* abort = &bars->abort;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bars->q_full, 1);
+    tc::mbar_init(&bars->q_empty, 1);
+    for (int s = 0; s < NS; ++s) {
+      tc::mbar_init(&bars->kv_full[s], 1);
+      tc::mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&bars->s_full[s], 1);
+      tc::mbar_init(&bars->s_empty[s], 4);
+      tc::mbar_init(&bars->p_full[s], 4);
+      tc::mbar_init(&bars->pv_done[s], 1);
+    }
+    tc::mbar_init(&bars->o_full, 1);
+    tc::mbar_init(&bars->o_empty, 4);
+    bars->abort = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&bars->tmem_base, L::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::prefetch_tmap(&tmQ);
+    tc::prefetch_tmap(&tmK);
+    tc::prefetch_tmap(&tmV);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t g = 0, tcount = 0;
+      for (int64_t k = blockIdx.x; k < ntiles && !*abort; k += gridDim.x, ++tcount) {
+        const int tile = tile_order[k];
+        if (tile < 0 || tile >= ntiles) { fail(bars, 11); break; }
+        const int64_t bh = tile / m.nt;
+        const int t = (int)(tile - bh * m.nt);
+        if (!tc::mbar_wait(&bars->q_empty, (tcount & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 1); break; }
+        tc::mbar_expect_tx(&bars->q_full, L::kQBytes);
+        for (int c = 0; c < D / 64; ++c)
+          for (int h = 0; h < 2; ++h)
+            tc::tma_load_3d(sQ + c * L::kQChunk + h * L::kKVChunk, &tmQ, &bars->q_full, c * 64,
+                            t * kTileRows + h * kBlock, (int)bh);
+        PairMerge mg(row_ptr, col_idx, bh, t, m.nb);
+        int j, mask;
+        while (mg.next(j, mask)) {
+          const int st = g % NS;
+          if (!tc::mbar_wait(&bars->kv_empty[st], ((g / NS) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 2); break; }
+          unsigned char* sK = sKV + st * L::kStage;
+          unsigned char* sV = sK + L::kKBytes;
+          tc::mbar_expect_tx(&bars->kv_full[st], L::kStage);
+          for (int c = 0; c < D / 64; ++c) {
+            tc::tma_load_3d(sK + c * L::kKVChunk, &tmK, &bars->kv_full[st], c * 64, j * kBlock, (int)bh);
+            tc::tma_load_3d(sV + c * L::kKVChunk, &tmV, &bars->kv_full[st], c * 64, j * kBlock, (int)bh);
+          }
+          ++g;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = tc::idesc_bf16_f32(kTileRows, kBlock, 0, 0);
+      constexpr uint32_t idO = tc::idesc_bf16_f32(kTileRows, D, 0, 1);
+      const uint32_t qaddr = tc::smem_u32(sQ), kvaddr = tc::smem_u32(sKV), paddr = tc::smem_u32(sP);
+      uint32_t g = 0, tcount = 0;
+      bool ok = true;
+      // O += P_gs V_gs for step gs; `first` = first step of the tile (overwrites O).
+      auto pv = [&](uint32_t gs, bool first) -> bool {
+        const int pb = gs & 1;
+        if (!tc::mbar_wait(&bars->p_full[pb], (gs >> 1) & 1, abort, kWaitLimit)) return false;
+        if (first && !tc::mbar_wait(&bars->o_empty, (tcount & 1) ^ 1, abort, kWaitLimit)) return false;
+        tc::fence_after_sync();
+        const uint32_t vaddr = kvaddr + (gs % NS) * L::kStage + L::kKBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk) {
+          const uint64_t a = tc::smem_desc_sw128(paddr + pb * L::kPBytes + kk * 32, 16, 1024);
+          const uint64_t b = tc::smem_desc_sw128(vaddr + kk * 16 * 128, L::kKVChunk, 1024);
+          tc::mma_f16(tbase + L::kColO, a, b, idO, (first && kk == 0) ? 0u : 1u);
+        }
+        tc::mma_commit(&bars->pv_done[pb]);
+        tc::mma_commit(&bars->kv_empty[gs % NS]);
+        return true;
+      };
+      for (int64_t k = blockIdx.x; k < ntiles && ok; k += gridDim.x, ++tcount) {
+        const int tile = tile_order[k];
+        if (tile < 0 || tile >= ntiles) { fail(bars, 11); break; }
+        const int64_t bh = tile / m.nt;
+        const int t = (int)(tile - bh * m.nt);
+        if (!tc::mbar_wait(&bars->q_full, tcount & 1, abort, kWaitLimit)) { fail(bars, 3); ok = false; break; }
+        PairMerge mg(row_ptr, col_idx, bh, t, m.nb);
+        int j, mask, i = 0;
+        while (mg.next(j, mask)) {
+          const uint32_t gi = g + i;
+          const int st = gi % NS, sb = gi & 1;
+          if (!tc::mbar_wait(&bars->kv_full[st], (gi / NS) & 1, abort, kWaitLimit) ||
+              !tc::mbar_wait(&bars->s_empty[sb], ((gi >> 1) & 1) ^ 1, abort, kWaitLimit)) {
+            fail(bars, 4);
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t kaddr = kvaddr + st * L::kStage;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int c = kk >> 2, off = (kk & 3) * 32;
+            const uint64_t a = tc::smem_desc_sw128(qaddr + c * L::kQChunk + off, 16, 1024);
+            const uint64_t b = tc::smem_desc_sw128(kaddr + c * L::kKVChunk + off, 16, 1024);
+            tc::mma_f16(tbase + sb * kBlock, a, b, idS, kk > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&bars->s_full[sb]);
+          if (i > 0 && !pv(gi - 1, i == 1)) { fail(bars, 5); ok = false; break; }
+          ++i;
+        }
+        if (!ok) break;
+        tc::mma_commit(&bars->q_empty);          // every S of this tile issued: Q may be replaced
+        if (i > 0 && !pv(g + i - 1, i == 1)) { fail(bars, 6); ok = false; break; }
+        tc::mma_commit(&bars->o_full);
+        g += i;
+      }
+      // Drain: every MMA issued so far has completed before TMEM can be released.
+      if (ok && tcount > 0) tc::mbar_wait(&bars->o_full, (tcount - 1) & 1, abort, kWaitLimit);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int q = warp & 3;                  // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;             // tile row == TMEM lane
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const bool lo_half = r < kBlock;
+    uint32_t g = 0, tcount = 0;
+    for (int64_t k = blockIdx.x; k < ntiles; k += gridDim.x, ++tcount) {
+      const int tile = tile_order[k];
+      if (tile < 0 || tile >= ntiles) { fail(bars, 11); break; }
+      const int64_t bh = tile / m.nt;
+      const int t = (int)(tile - bh * m.nt);
+      float mrow = -INFINITY, lrow = 0.f;
+      PairMerge mg(row_ptr, col_idx, bh, t, m.nb);
+      int j, mask, i = 0;
+      bool ok = true;
+      while (mg.next(j, mask)) {
+        const uint32_t gi = g + i;
+        const int sb = gi & 1;
+        if (!warp_wait(&bars->s_full[sb], (gi >> 1) & 1, abort)) { fail(bars, 7); ok = false; break; }
+        tc::fence_after_sync();
+        uint32_t sraw[64];
+        {
+          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]);
+          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]);
+          tc::tmem_ld32(tbase + lane_off + sb * kBlock, lo);
+          tc::tmem_ld32(tbase + lane_off + sb * kBlock + 32, hi);
+          tc::tmem_ld_wait();
+        }
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bars->s_empty[sb]);
+
+        const bool sel = lo_half ? (mask & 1) : (mask & 2);
+        const int nk = (int)imin<int64_t>(kBlock, m.S - (int64_t)j * kBlock);
+        float x[64];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          x[c] = (sel && c < nk) ? __uint_as_float(sraw[c]) * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, x[c]);
+        }
+        // Raise the running max only when it grows by more than 2^8 (or on the row's first
+        // kept block); rows whose O already holds earlier blocks then scale O in TMEM.
+        const bool raise = sel && (mrow == -INFINITY || mx > mrow + kRescaleLog2);
+        const bool scale_o = raise && i > 0 && mrow != -INFINITY;
+        if (__any_sync(0xffffffffu, scale_o)) {
+          // tcgen05.ld/st are warp-collective: the whole warp takes part, each lane with its
+          // own factor (1 for rows that keep their max).
+          const uint32_t gp = gi - 1;
+          if (!warp_wait(&bars->pv_done[gp & 1], (gp >> 1) & 1, abort)) { fail(bars, 8); ok = false; break; }
+          tc::fence_after_sync();
+          const float alpha = scale_o ? ex2(mrow - mx) : 1.f;
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tc::tmem_ld32(tbase + lane_off + L::kColO + cc * 32, o);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tc::tmem_st32(tbase + lane_off + L::kColO + cc * 32, o);
+          }
+          tc::tmem_st_wait();
+          lrow *= alpha;
+        }
+        if (raise) mrow = mx;
+        uint32_t packed[32];
+        if (sel) {
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const float p0 = ex2(x[c] - mrow);
+            const float p1 = ex2(x[c + 1] - mrow);
+            lrow += p0 + p1;
+            packed[c >> 1] = pack_bf16(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) packed[c] = 0u;
+        }
+        if (gi >= 2) {       // P buffer sb was last read by the P.V of step gi-2
+          const uint32_t gp = gi - 2;
+          if (!warp_wait(&bars->pv_done[sb], (gp >> 1) & 1, abort)) { fail(bars, 9); ok = false; break; }
+        }
+        // Row r of P in the 128-byte-swizzled K-major layout: 16-byte chunk c of the row goes
+        // to chunk position c ^ (r mod 8).
+        unsigned char* prow = sP + sb * L::kPBytes + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 v = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = v;
+        }
+        tc::fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bars->p_full[sb]);
+        ++i;
+      }
+      if (__any_sync(0xffffffffu, !ok || *abort)) break;
+      // ---------------------------------------------------------- epilogue
+      if (!warp_wait(&bars->o_full, tcount & 1, abort)) { fail(bars, 10); break; }
+      tc::fence_after_sync();
+      const int64_t trow = (int64_t)t * kTileRows + r;
+      const bool valid = trow < m.S;
+      const float inv = 1.f / lrow;
+      __nv_bfloat16* orow = O + (bh * m.S + trow) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tc::tmem_ld32(tbase + lane_off + L::kColO + cc * 32, o);
+        tc::tmem_ld_wait();
+        if (valid) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(o[8 * v4 + 0]) * inv, __uint_as_float(o[8 * v4 + 1]) * inv);
+            w.y = pack_bf16(__uint_as_float(o[8 * v4 + 2]) * inv, __uint_as_float(o[8 * v4 + 3]) * inv);
+            w.z = pack_bf16(__uint_as_float(o[8 * v4 + 4]) * inv, __uint_as_float(o[8 * v4 + 5]) * inv);
+            w.w = pack_bf16(__uint_as_float(o[8 * v4 + 6]) * inv, __uint_as_float(o[8 * v4 + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + cc * 32 + v4 * 8) = w;
+          }
+        }
+      }
+      if (valid && lse != nullptr) lse[bh * m.S + trow] = (mrow + log2f(lrow)) * 0.69314718055994531f;
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bars->o_empty);
+      g += i;
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(tbase, L::kTmemCols);
+  if (threadIdx.x == 0 && bars->abort) report_error(control, FVATTN_ERR_TIMEOUT, bars->abort);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [BH, S, d] bf16 viewed as a 3-D tensor (d innermost); 64 x 64 boxes with the 128-byte
+// swizzle; rows past S read as zeros and never reach the next head.
+bool make_map(CUtensorMap* map, const void* base, const Dims& m) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)m.d, (cuuint64_t)m.S, (cuuint64_t)m.BH};
+  cuuint64_t strides[2] = {(cuuint64_t)m.d * 2, (cuuint64_t)m.S * (cuuint64_t)m.d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)kBlock, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_tc_d(const void* Q, const void* K, const void* V, const Dims& m, float scale,
+                        const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_order,
+                        int32_t* control, void* O, float* lse, int nsm, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, m) || !make_map(&mk, K, m) || !make_map(&mv, V, m)) return cudaErrorInvalidValue;
+  const size_t smem = TcLayout<D>::kBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t ntiles = m.BH * m.nt;
+  const int grid = (int)imin<int64_t>(ntiles, (int64_t)nsm);
+  attn_tc_kernel<D><<<grid, 192, smem, st>>>(mq, mk, mv, m, scale * 1.4426950408889634f, row_ptr, col_idx,
+                                             tile_order, control, static_cast<__nv_bfloat16*>(O), lse);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const Dims& m, float scale,
+                           const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_order,
+                           int32_t* control, void* O, float* lse, int nsm, cudaStream_t st) {
+  if (m.d == 128)
+    return launch_tc_d<128>(Q, K, V, m, scale, row_ptr, col_idx, tile_order, control, O, lse, nsm, st);
+  return launch_tc_d<64>(Q, K, V, m, scale, row_ptr, col_idx, tile_order, control, O, lse, nsm, st);
+}
+
+}  // namespace fv

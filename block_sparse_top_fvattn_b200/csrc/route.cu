@@ -1,0 +1,783 @@
+// Router kernels: block pooling, fp64 block scores, row softmax, Top-p cut, frame-level
+// top-k, forced blocks, CSR rows, per-head loads, tile costs and the longest-first order.
+//
+// Method: FVAttn blog summary ("腾讯+中山大学新作：视频生成提速2.11×，靠的是RLB和SASA"), section
+// "AI视频生成的阿喀琉斯之踵" (Top-p: smallest descending-importance prefix reaching p) and
+// section "RLB…" (per-head load = selected block count, heaviest first); video-generation
+// acceleration notes (wzjinhao.cn) §5.2 (block means, score = mean(Q)·mean(K)/sqrt(d), local
+// band); vLLM-Omni Sol-Attn article §2.1/§2.2 (frame top-k, neighbour and first frames).
+#include <math.h>
+
+#include "common.cuh"
+#include "route.cuh"
+
+namespace fv {
+
+// ------------------------------------------------------------------ warp helpers
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ double warp_max(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_incl_scan(T v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    T u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  return v;
+}
+
+// ------------------------------------------------------------------ K1: block pooling
+//
+// One 64-token block of one tensor per loop iteration. Every thread streams 16-byte vectors
+// of PASSES rows (all loads issued before any use), sums them in AccT (fp32 for bf16 input:
+// a sum of four bf16 values is exact unless their exponents are 16+ apart; fp64 for fp32
+// input), and the row groups are combined in fp64 in a fixed order. Output: fp64 means over
+// the valid tokens, or (frame mode) fp64 sums of the tokens before / after the block's first
+// frame boundary.
+
+template <typename T> struct Acc;
+template <> struct Acc<__nv_bfloat16> { using type = float; static constexpr int kVec = 8; };
+template <> struct Acc<float> { using type = double; static constexpr int kVec = 4; };
+
+__device__ __forceinline__ void unpack(const uint4& v, float (&o)[8], const __nv_bfloat16*) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float2 f = __bfloat1622float2(h[q]);
+    o[2 * q] = f.x;
+    o[2 * q + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void unpack(const uint4& v, double (&o)[4], const float*) {
+  o[0] = __uint_as_float(v.x);
+  o[1] = __uint_as_float(v.y);
+  o[2] = __uint_as_float(v.z);
+  o[3] = __uint_as_float(v.w);
+}
+
+template <typename T, int D, bool FRAME>
+__global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ Q, const T* __restrict__ K,
+                                                   int ntensors, Dims m, int frame_len,
+                                                   double* __restrict__ qlo, double* __restrict__ klo,
+                                                   double* __restrict__ qhi, double* __restrict__ khi) {
+  using AccT = typename Acc<T>::type;
+  constexpr int VEC = Acc<T>::kVec;
+  constexpr int CPR = D / VEC;         // 16-byte chunks per row
+  constexpr int RPP = 256 / CPR;       // rows per pass
+  constexpr int PASSES = kBlock / RPP;
+  __shared__ double red[FRAME ? 2 : 1][RPP][D];
+
+  const int tid = threadIdx.x;
+  const int c = tid % CPR, r0 = tid / CPR;
+  const int64_t per = m.BH * m.nb;
+  const int64_t units = per * ntensors;
+  for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+    const bool isK = u >= per;
+    const int64_t row = isK ? u - per : u;       // bh * nb + blk
+    const int64_t bh = row / m.nb;
+    const int blk = (int)(row - bh * m.nb);
+    const int64_t t0 = (int64_t)blk * kBlock;
+    const int nvalid = (int)imin<int64_t>(kBlock, m.S - t0);
+    const T* X = (isK ? K : Q) + (bh * m.S + t0) * D;
+    int boundary = kBlock;
+    if (FRAME) boundary = (int)imin<int64_t>(kBlock, (t0 / frame_len + 1) * frame_len - t0);
+
+    uint4 v[PASSES];
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) {
+      const int r = r0 + p * RPP;
+      if (r < nvalid)
+        v[p] = __ldg(reinterpret_cast<const uint4*>(X + (int64_t)r * D + c * VEC));
+      else
+        v[p] = make_uint4(0, 0, 0, 0);
+    }
+    AccT lo[VEC], hi[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) lo[e] = hi[e] = 0;
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) {
+      AccT x[VEC];
+      unpack(v[p], x, (const T*)nullptr);
+      const bool in_lo = !FRAME || (r0 + p * RPP) < boundary;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        if (in_lo) lo[e] += x[e];
+        else hi[e] += x[e];
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      red[0][r0][c * VEC + e] = (double)lo[e];
+      if (FRAME) red[FRAME ? 1 : 0][r0][c * VEC + e] = (double)hi[e];
+    }
+    __syncthreads();
+    if (tid < D) {
+      double s = 0.0;
+#pragma unroll
+      for (int rr = 0; rr < RPP; ++rr) s += red[0][rr][tid];
+      double* out = (isK ? klo : qlo) + row * D + tid;
+      if (FRAME) {
+        double h = 0.0;
+#pragma unroll
+        for (int rr = 0; rr < RPP; ++rr) h += red[FRAME ? 1 : 0][rr][tid];
+        *out = s;
+        (isK ? khi : qhi)[row * D + tid] = h;
+      } else {
+        *out = s / (double)nvalid;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ forced blocks
+
+// Up to four inclusive block ranges that every row of query block i keeps: the diagonal,
+// the band |i-j| <= w, the frames within +-fw of the block's frames, frame 0. An empty
+// range has a > b.
+__device__ __forceinline__ void forced_ranges(int i, const Dims& m, const ForceCfg& fc, int (&a)[4],
+                                              int (&b)[4]) {
+#pragma unroll
+  for (int r = 0; r < 4; ++r) { a[r] = 1; b[r] = 0; }
+  if (fc.force_diag) { a[0] = i; b[0] = i; }
+  if (fc.local_window > 0) {
+    a[1] = max(0, i - fc.local_window);
+    b[1] = min(m.nb - 1, i + fc.local_window);
+  }
+  if (fc.frame_len > 0) {
+    const int64_t fl = fc.frame_len;
+    if (fc.frame_window >= 0) {
+      const int64_t t0 = (int64_t)i * kBlock, t1 = min(m.S, t0 + kBlock) - 1;
+      const int64_t f0 = imax<int64_t>(0, t0 / fl - fc.frame_window);
+      const int64_t f1 = imin<int64_t>(m.F - 1, t1 / fl + fc.frame_window);
+      a[2] = (int)(f0 * fl / kBlock);
+      b[2] = (int)((min(m.S, (f1 + 1) * fl) - 1) / kBlock);
+    }
+    if (fc.force_first) { a[3] = 0; b[3] = (int)((min(m.S, fl) - 1) / kBlock); }
+  }
+}
+
+// OR the forced ranges into the row's bitmask (shared memory), store it and its count.
+__device__ __forceinline__ int finalize_row(uint32_t* w, int i, const Dims& m, const ForceCfg& fc, int lane,
+                                            uint32_t* __restrict__ gbits, int32_t* __restrict__ gcount) {
+  int a[4], b[4];
+  forced_ranges(i, m, fc, a, b);
+  int cnt = 0;
+  for (int q = lane; q < m.nw; q += 32) {
+    uint32_t x = w[q];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) x |= range_bits(a[r], b[r], q);
+    x &= range_bits(0, m.nb - 1, q);
+    w[q] = x;
+    gbits[q] = x;
+    cnt += __popc(x);
+  }
+  cnt = warp_sum(cnt);
+  if (lane == 0) *gcount = cnt;
+  __syncwarp();
+  return cnt;
+}
+
+// ------------------------------------------------------------------ K2: Top-p
+
+constexpr int RT = 16;      // query blocks per CTA
+constexpr int KT = 256;     // key blocks per pass of the score tile
+constexpr int KC = 16;      // head-dim chunk staged in shared memory
+constexpr int NWARP = 8;
+
+// In-place softmax of a row of n logits (fp64): pi_j = exp(s_j - max) / sum.
+__device__ void softmax_row(double* L, int n, int lane) {
+  double mx = -INFINITY;
+  for (int j = lane; j < n; j += 32) mx = fmax(mx, L[j]);
+  mx = warp_max(mx);
+  double z = 0.0;
+  for (int j = lane; j < n; j += 32) {
+    const double e = exp(L[j] - mx);
+    L[j] = e;
+    z += e;
+  }
+  z = warp_sum(z);
+  for (int j = lane; j < n; j += 32) L[j] = L[j] / z;
+  __syncwarp();
+}
+
+// Probability mass as a 62-bit fixed-point integer, so that every sum below is exact and
+// independent of summation order (rounding: 2^-63 per block).
+__device__ __forceinline__ uint64_t fixmass(double x) {
+  return (uint64_t)__double2ull_rn(x * 4611686018427387904.0);
+}
+
+// Top-p cut of one row of probabilities (one warp). The kept set is the descending prefix
+// (ties: lower index first) of minimal length whose mass reaches p. Positive doubles order
+// like their bit patterns, so the cut is found as the largest key T with
+//   mass{ j : key_j >= T } >= P
+// by an MSB-first radix select over 8-bit digits of the keys (histograms of exact
+// fixed-point mass); then every key > T is kept and as many keys == T, in ascending index,
+// as are needed to reach P. Writes the bitmask words w[0..nw).
+__device__ void topp_select(const double* pi, int n, double p, uint64_t* hm, uint32_t* hc, uint32_t* w,
+                            int lane) {
+  const int nw = (n + 31) / 32;
+  bool all = p >= 1.0;
+  const uint64_t P = fixmass(p);
+  if (!all) {
+    uint64_t tot = 0;
+    for (int j = lane; j < n; j += 32) tot += fixmass(pi[j]);
+    tot = warp_sum(tot);
+    all = tot < P;      // the whole row falls short of p by rounding: keep everything
+  }
+  if (all) {
+    for (int q = lane; q < nw; q += 32) w[q] = range_bits(0, n - 1, q);
+    __syncwarp();
+    return;
+  }
+  uint64_t prefix = 0, pmask = 0, above = 0;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) { hm[b] = 0; hc[b] = 0; }
+    __syncwarp();
+    for (int j = lane; j < n; j += 32) {
+      const uint64_t key = (uint64_t)__double_as_longlong(pi[j]);
+      if ((key & pmask) == prefix) {
+        const int dg = (int)((key >> shift) & 255);
+        atomicAdd(reinterpret_cast<unsigned long long*>(&hm[dg]), (unsigned long long)fixmass(pi[j]));
+        atomicAdd(&hc[dg], 1u);
+      }
+    }
+    __syncwarp();
+    // Lane l holds bins 255-8l .. 248-8l, so scanning lanes upward walks the digits downward.
+    uint64_t lsum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) lsum += hm[255 - 8 * lane - q];
+    const uint64_t incl = warp_incl_scan(lsum, lane);
+    uint64_t cum = above + (incl - lsum);
+    int found = -1;
+    uint64_t before = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int dg = 255 - 8 * lane - q;
+      const uint64_t nc = cum + hm[dg];
+      if (found < 0 && nc >= P) { found = dg; before = cum; }
+      cum = nc;
+    }
+    const uint32_t bal = __ballot_sync(0xffffffffu, found >= 0);
+    const int src = __ffs(bal) - 1;     // invariant: above < P <= above + candidates' mass
+    const int dg = __shfl_sync(0xffffffffu, found, src);
+    above = __shfl_sync(0xffffffffu, before, src);
+    prefix |= (uint64_t)dg << shift;
+    pmask |= (uint64_t)0xff << shift;
+    const uint32_t cnt = hc[dg];
+    __syncwarp();
+    if (cnt == 1) {      // a single candidate left: it is T
+      uint64_t T = 0;
+      for (int j = lane; j < n; j += 32) {
+        const uint64_t key = (uint64_t)__double_as_longlong(pi[j]);
+        if ((key & pmask) == prefix) T = key;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t u = __shfl_xor_sync(0xffffffffu, T, o);
+        T = u > T ? u : T;
+      }
+      prefix = T;
+      pmask = ~0ull;
+      break;
+    }
+  }
+  const uint64_t T = prefix;
+  const uint64_t mT = fixmass(__longlong_as_double((long long)T));
+  const uint64_t need = mT ? (P - above + mT - 1) / mT : 0;
+  uint32_t taken = 0;
+  for (int q = 0; q < nw; ++q) {
+    const int j = q * 32 + lane;
+    const uint64_t key = j < n ? (uint64_t)__double_as_longlong(pi[j]) : 0;
+    const bool gt = j < n && key > T;
+    const bool eq = j < n && key == T;
+    const uint32_t be = __ballot_sync(0xffffffffu, eq);
+    const uint32_t rank = taken + __popc(be & lanemask_lt());
+    const bool sel = gt || (eq && rank < need);
+    const uint32_t word = __ballot_sync(0xffffffffu, sel);
+    if (lane == 0) w[q] = word;
+    taken += __popc(be);
+  }
+  __syncwarp();
+}
+
+size_t topp_smem_bytes(const Dims& m) {
+  const size_t nbp = (size_t)m.nw * 32;
+  const size_t u = (size_t)KC * KT * 8 > (size_t)NWARP * 256 * 12 ? (size_t)KC * KT * 8 : (size_t)NWARP * 256 * 12;
+  return (size_t)KC * RT * 8 + (size_t)RT * nbp * 8 + u + (size_t)NWARP * 2 * m.nw * 4;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) topp_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
+                                                   Dims m, double p, double scale, ForceCfg fc,
+                                                   uint32_t* __restrict__ bits, int32_t* __restrict__ counts,
+                                                   int32_t* __restrict__ tile_cost) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int nbp = m.nw * 32;
+  double* sA = reinterpret_cast<double*>(smem_raw);      // [KC][RT]
+  double* sL = sA + KC * RT;                               // [RT][nbp] logits, then probabilities
+  double* sU = sL + (size_t)RT * nbp;                      // [KC][KT] key-mean chunk | histograms
+  uint32_t* sW = reinterpret_cast<uint32_t*>(sU + KC * KT); // [NWARP][2][nw] row bitmasks
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t bh = blockIdx.y;
+  const int row0 = blockIdx.x * RT;
+  const double* qb = qbar + bh * m.nb * D;
+  const double* kb = kbar + bh * m.nb * D;
+  const int lm = lane >> 3, ln = lane & 7;   // 4 x 8 lanes: 4 rows x 4 keys per lane
+
+  // Scores Sc[i][j] = <qbar_i, kbar_j> * scale, fp64 FMA in ascending head-dim order.
+  for (int kp = 0; kp < m.nb; kp += KT) {
+    double acc[4][4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[r][c] = 0.0;
+    for (int k0 = 0; k0 < D; k0 += KC) {
+      __syncthreads();
+      {
+        const int r = tid / KC, kk = tid % KC;
+        const int i = row0 + r;
+        sA[kk * RT + r] = (i < m.nb) ? qb[(int64_t)i * D + k0 + kk] : 0.0;
+      }
+      {
+        const int j = kp + tid;
+        if (j < m.nb) {
+          const double2* src = reinterpret_cast<const double2*>(kb + (int64_t)j * D + k0);
+#pragma unroll
+          for (int q = 0; q < KC / 2; ++q) {
+            const double2 v = src[q];
+            sU[(2 * q) * KT + tid] = v.x;
+            sU[(2 * q + 1) * KT + tid] = v.y;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < KC; ++q) sU[q * KT + tid] = 0.0;
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int kk = 0; kk < KC; ++kk) {
+        const double2 a01 = *reinterpret_cast<const double2*>(sA + kk * RT + lm * 4);
+        const double2 a23 = *reinterpret_cast<const double2*>(sA + kk * RT + lm * 4 + 2);
+        const double a[4] = {a01.x, a01.y, a23.x, a23.y};
+        double bq[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) bq[c] = sU[kk * KT + warp * 32 + ln + 8 * c];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[r][c] = fma(a[r], bq[c], acc[r][c]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int j = kp + warp * 32 + ln + 8 * c;
+        if (j < m.nb) sL[(lm * 4 + r) * nbp + j] = acc[r][c] * scale;
+      }
+  }
+  __syncthreads();
+
+  uint64_t* hm = reinterpret_cast<uint64_t*>(sU) + warp * 256;
+  uint32_t* hc = reinterpret_cast<uint32_t*>(reinterpret_cast<uint64_t*>(sU) + NWARP * 256) + warp * 256;
+  uint32_t* w0 = sW + warp * 2 * m.nw;
+#pragma unroll 1
+  for (int rr = 0; rr < 2; ++rr) {
+    const int r = 2 * warp + rr, i = row0 + r;
+    uint32_t* w = w0 + rr * m.nw;
+    if (i >= m.nb) {
+      for (int q = lane; q < m.nw; q += 32) w[q] = 0;
+      __syncwarp();
+      continue;
+    }
+    double* L = sL + (size_t)r * nbp;
+    softmax_row(L, m.nb, lane);
+    topp_select(L, m.nb, p, hm, hc, w, lane);
+    const int64_t grow = bh * m.nb + i;
+    finalize_row(w, i, m, fc, lane, bits + grow * m.nw, counts + grow);
+  }
+  const int t = (row0 >> 1) + warp;
+  if (2 * t < m.nb) {
+    int c = 0;
+    for (int q = lane; q < m.nw; q += 32) c += __popc(w0[q] | w0[m.nw + q]);
+    c = warp_sum(c);
+    if (lane == 0) tile_cost[bh * m.nt + t] = c;
+  }
+}
+
+// ------------------------------------------------------------------ frame mode
+
+// Frame means from the per-block segment sums: frame f gathers the "lo" sums of the blocks
+// that start inside f and the "hi" sums of the block that starts in f-1 and straddles into f
+// (frames are at least one block long, so a block touches at most two frames).
+template <int D>
+__global__ void __launch_bounds__(D) frame_means_kernel(const double* __restrict__ qlo, const double* __restrict__ qhi,
+                                                        const double* __restrict__ klo, const double* __restrict__ khi,
+                                                        Dims m, int frame_len, double* __restrict__ qf,
+                                                        double* __restrict__ kf) {
+  const int f = blockIdx.x;
+  const int64_t bh = blockIdx.y;
+  const bool isK = blockIdx.z != 0;
+  const double* lo = isK ? klo : qlo;
+  const double* hi = isK ? khi : qhi;
+  const int64_t t0 = (int64_t)f * frame_len, t1 = min(m.S, t0 + frame_len);
+  const int b0 = (int)(t0 / kBlock), b1 = (int)((t1 - 1) / kBlock);
+  double s = 0.0;
+  for (int b = b0; b <= b1; ++b) {
+    const int64_t fb = ((int64_t)b * kBlock) / frame_len;
+    const double* src = (fb == f) ? lo : hi;
+    s += src[(bh * m.nb + b) * D + threadIdx.x];
+  }
+  (isK ? kf : qf)[(bh * m.F + f) * D + threadIdx.x] = s / (double)(t1 - t0);
+}
+
+size_t frame_smem_bytes(const Dims& m) {
+  const int fwords = (m.F + 31) / 32;
+  return (size_t)m.F * m.F * 8 + (size_t)m.F * fwords * 4 + (size_t)NWARP * 2 * m.nw * 4;
+}
+
+// One CTA per head: frame scores s(f,g) = <qf_f, kf_g> * scale in fp64; per query frame the
+// top-k key frames (ties to the lower frame); per query block the union over the frames it
+// touches, expanded to the key blocks that hold tokens of a kept frame; then forced blocks.
+template <int D>
+__global__ void __launch_bounds__(256) frame_select_kernel(const double* __restrict__ qf, const double* __restrict__ kf,
+                                                           Dims m, int frame_len, int topk, double scale,
+                                                           ForceCfg fc, uint32_t* __restrict__ bits,
+                                                           int32_t* __restrict__ counts,
+                                                           int32_t* __restrict__ tile_cost) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int F = m.F, fwords = (F + 31) / 32;
+  double* sS = reinterpret_cast<double*>(smem_raw);                     // [F][F]
+  uint32_t* sCh = reinterpret_cast<uint32_t*>(sS + (size_t)F * F);      // [F][fwords]
+  uint32_t* sW = sCh + (size_t)F * fwords;                              // [NWARP][2][nw]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t bh = blockIdx.x;
+
+  for (int x = tid; x < F * F; x += blockDim.x) {
+    const int f = x / F, g = x - f * F;
+    const double* a = qf + (bh * F + f) * D;
+    const double* b = kf + (bh * F + g) * D;
+    double s = 0.0;
+#pragma unroll 8
+    for (int k = 0; k < D; ++k) s = fma(a[k], b[k], s);
+    sS[x] = s * scale;
+  }
+  for (int x = tid; x < F * fwords; x += blockDim.x) sCh[x] = 0;
+  __syncthreads();
+
+  const int k = min(topk, F);
+  for (int f = warp; f < F; f += NWARP) {
+    for (int r = 0; r < k; ++r) {
+      double best = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int g = lane; g < F; g += 32) {
+        const bool taken = (sCh[f * fwords + (g >> 5)] >> (g & 31)) & 1u;
+        const double v = sS[f * F + g];
+        if (!taken && (v > best || (v == best && g < bi))) { best = v; bi = g; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > best || (ov == best && oi < bi)) { best = ov; bi = oi; }
+      }
+      if (lane == 0) sCh[f * fwords + (bi >> 5)] |= 1u << (bi & 31);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+
+  uint32_t* w0 = sW + warp * 2 * m.nw;
+  for (int t = warp; t < m.nt; t += NWARP) {
+#pragma unroll 1
+    for (int rr = 0; rr < 2; ++rr) {
+      const int i = 2 * t + rr;
+      uint32_t* w = w0 + rr * m.nw;
+      if (i >= m.nb) {
+        for (int q = lane; q < m.nw; q += 32) w[q] = 0;
+        __syncwarp();
+        continue;
+      }
+      const int64_t ti0 = (int64_t)i * kBlock, ti1 = min(m.S, ti0 + kBlock) - 1;
+      const int f0 = (int)(ti0 / frame_len), f1 = (int)(ti1 / frame_len);
+      for (int q = lane; q < m.nw; q += 32) {
+        uint32_t x = 0;
+        for (int g = 0; g < F; ++g) {
+          const uint32_t kept = ((sCh[f0 * fwords + (g >> 5)] | sCh[f1 * fwords + (g >> 5)]) >> (g & 31)) & 1u;
+          if (kept) {
+            const int a = (int)(((int64_t)g * frame_len) / kBlock);
+            const int b = (int)((min(m.S, (int64_t)(g + 1) * frame_len) - 1) / kBlock);
+            x |= range_bits(a, b, q);
+          }
+        }
+        w[q] = x;
+      }
+      __syncwarp();
+      const int64_t grow = bh * m.nb + i;
+      finalize_row(w, i, m, fc, lane, bits + grow * m.nw, counts + grow);
+    }
+    if (2 * t < m.nb) {
+      int c = 0;
+      for (int q = lane; q < m.nw; q += 32) c += __popc(w0[q] | w0[m.nw + q]);
+      c = warp_sum(c);
+      if (lane == 0) tile_cost[bh * m.nt + t] = c;
+    }
+    __syncwarp();
+  }
+}
+
+// ------------------------------------------------------------------ K3: schedule
+
+size_t schedule_smem_bytes(const Dims& m, int* groups) {
+  const size_t nb1 = (size_t)m.nb + 1;
+  int g = 32;
+  while (g > 1 && (size_t)(g + 1) * nb1 * 4 > 200 * 1024) g >>= 1;
+  *groups = g;
+  return (size_t)(g + 1) * nb1 * 4;
+}
+
+// One CTA: CSR row offsets (exclusive scan of the row counts), nnz, per-head loads, and the
+// tile order: a stable counting sort of tile costs, largest first, ties by ascending tile id.
+// Tiles are split into `groups` contiguous segments with one histogram each, so the sort
+// stays stable while the segments are placed in parallel.
+__global__ void __launch_bounds__(1024) schedule_kernel(const int32_t* __restrict__ counts,
+                                                        const int32_t* __restrict__ tile_cost, Dims m,
+                                                        int groups, int32_t* __restrict__ row_ptr,
+                                                        int64_t* __restrict__ head_load,
+                                                        int64_t* __restrict__ nnz_out,
+                                                        int32_t* __restrict__ tile_order, int64_t capacity,
+                                                        int32_t* __restrict__ status) {
+  extern __shared__ __align__(16) int32_t shs[];
+  __shared__ int64_t wsum[32];
+  __shared__ int32_t wtot[32];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- row offsets
+  const int64_t N = m.BH * m.nb;
+  const int64_t per = (N + 1023) / 1024;
+  const int64_t r0 = min(N, (int64_t)tid * per), r1 = min(N, r0 + per);
+  int64_t s = 0;
+  for (int64_t r = r0; r < r1; ++r) s += counts[r];
+  const int64_t incl = warp_incl_scan(s, lane);
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int64_t v = wsum[lane];
+    const int64_t vi = warp_incl_scan(v, lane);
+    wsum[lane] = vi - v;
+  }
+  __syncthreads();
+  int64_t base = wsum[warp] + incl - s;
+  for (int64_t r = r0; r < r1; ++r) {
+    row_ptr[r] = (int32_t)base;
+    base += counts[r];
+  }
+  if (tid == 1023) {
+    row_ptr[N] = (int32_t)base;
+    *nnz_out = base;
+    if (base > capacity) report_error(status, FVATTN_ERR_CAPACITY, 1);
+  }
+  __syncthreads();
+  for (int64_t bh = tid; bh < m.BH; bh += 1024)
+    head_load[bh] = (int64_t)row_ptr[(bh + 1) * m.nb] - (int64_t)row_ptr[bh * m.nb];
+
+  // ---- tile order
+  const int nb1 = m.nb + 1;
+  int32_t* hist = shs;                    // [groups][nb1]: counts, then running offsets
+  int32_t* tot = shs + (size_t)groups * nb1;
+  for (int x = tid; x < groups * nb1; x += 1024) hist[x] = 0;
+  __syncthreads();
+  const int64_t NT = m.BH * m.nt;
+  const int64_t seg = (NT + groups - 1) / groups;
+  if (warp < groups) {
+    const int64_t s0 = min(NT, warp * seg), s1 = min(NT, s0 + seg);
+    for (int64_t t = s0 + lane; t < s1; t += 32) atomicAdd(&hist[warp * nb1 + tile_cost[t]], 1);
+  }
+  __syncthreads();
+  for (int c = tid; c < nb1; c += 1024) {
+    int run = 0;
+    for (int g = 0; g < groups; ++g) {
+      const int h = hist[g * nb1 + c];
+      hist[g * nb1 + c] = run;
+      run += h;
+    }
+    tot[c] = run;
+  }
+  __syncthreads();
+  // base[c] = number of tiles with cost > c: a suffix scan of tot, in chunks per thread.
+  {
+    const int chunk = (nb1 + 1023) / 1024;
+    const int c0 = min(nb1, tid * chunk), c1 = min(nb1, c0 + chunk);
+    int ls = 0;
+    for (int c = c0; c < c1; ++c) ls += tot[c];
+    const int li = warp_incl_scan(ls, lane);
+    if (lane == 31) wtot[warp] = li;
+    __syncthreads();
+    if (warp == 0) {
+      const int v = wtot[lane];
+      const int vi = warp_incl_scan(v, lane);
+      wtot[lane] = vi;   // inclusive over warps
+    }
+    __syncthreads();
+    const int total = wtot[31];
+    // tiles with cost >= c0 (all buckets from this thread's chunk upward):
+    const int before_incl = (warp ? wtot[warp - 1] : 0) + li;   // sum of buckets [0, c1)
+    int above = total - before_incl;                             // sum of buckets [c1, nb1)
+    for (int c = c1 - 1; c >= c0; --c) {
+      const int tc = tot[c];
+      for (int g = 0; g < groups; ++g) hist[g * nb1 + c] += above;
+      above += tc;
+    }
+  }
+  __syncthreads();
+  if (warp < groups) {
+    const int64_t s0 = min(NT, warp * seg), s1 = min(NT, s0 + seg);
+    for (int64_t t0 = s0; t0 < s1; t0 += 32) {
+      const int64_t t = t0 + lane;
+      const bool v = t < s1;
+      const int c = v ? tile_cost[t] : -1 - lane;
+      const uint32_t peers = __match_any_sync(0xffffffffu, c);
+      const uint32_t lower = peers & lanemask_lt();
+      int pos = 0;
+      if (v) pos = hist[warp * nb1 + c] + __popc(lower);
+      __syncwarp();
+      if (v) {
+        tile_order[pos] = (int32_t)t;
+        if (lower == 0) hist[warp * nb1 + c] += __popc(peers);
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// ------------------------------------------------------------------ K4: CSR columns
+
+__global__ void __launch_bounds__(256) csr_kernel(const uint32_t* __restrict__ bits,
+                                                  const int32_t* __restrict__ row_ptr, Dims m,
+                                                  int32_t* __restrict__ col_idx, int64_t capacity) {
+  const int lane = threadIdx.x & 31;
+  const int64_t N = m.BH * m.nb;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < N; row += nwarps) {
+    if ((int64_t)row_ptr[row + 1] > capacity) continue;     // reported by the schedule kernel
+    const uint32_t* w = bits + row * m.nw;
+    int64_t base = row_ptr[row];
+    for (int q0 = 0; q0 < m.nw; q0 += 32) {
+      const int q = q0 + lane;
+      uint32_t x = q < m.nw ? w[q] : 0u;
+      const int c = __popc(x);
+      const int incl = warp_incl_scan(c, lane);
+      int64_t pos = base + incl - c;
+      while (x) {
+        const int b = __ffs(x) - 1;
+        x &= x - 1;
+        col_idx[pos++] = q * 32 + b;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ launchers
+
+template <typename T>
+static cudaError_t launch_pool_t(const void* Q, const void* K, int ntensors, const Dims& m, int frame_len,
+                                 double* qlo, double* klo, double* qhi, double* khi, int nsm,
+                                 cudaStream_t st) {
+  const int64_t units = m.BH * m.nb * ntensors;
+  const int grid = (int)imin<int64_t>(units, (int64_t)nsm * 8);
+  const T* q = static_cast<const T*>(Q);
+  const T* k = static_cast<const T*>(K);
+  if (m.d == 128) {
+    if (frame_len > 0) pool_kernel<T, 128, true><<<grid, 256, 0, st>>>(q, k, ntensors, m, frame_len, qlo, klo, qhi, khi);
+    else pool_kernel<T, 128, false><<<grid, 256, 0, st>>>(q, k, ntensors, m, 0, qlo, klo, qhi, khi);
+  } else {
+    if (frame_len > 0) pool_kernel<T, 64, true><<<grid, 256, 0, st>>>(q, k, ntensors, m, frame_len, qlo, klo, qhi, khi);
+    else pool_kernel<T, 64, false><<<grid, 256, 0, st>>>(q, k, ntensors, m, 0, qlo, klo, qhi, khi);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int frame_len,
+                        double* qlo, double* klo, double* qhi, double* khi, int nsm, cudaStream_t st) {
+  if (dtype == FVATTN_BF16)
+    return launch_pool_t<__nv_bfloat16>(Q, K, ntensors, m, frame_len, qlo, klo, qhi, khi, nsm, st);
+  return launch_pool_t<float>(Q, K, ntensors, m, frame_len, qlo, klo, qhi, khi, nsm, st);
+}
+
+cudaError_t launch_topp(const double* qbar, const double* kbar, const Dims& m, double p, double scale,
+                        const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
+                        cudaStream_t st) {
+  const size_t smem = topp_smem_bytes(m);
+  dim3 grid((m.nb + RT - 1) / RT, (unsigned)m.BH);
+  cudaError_t e;
+  if (m.d == 128) {
+    e = cudaFuncSetAttribute(topp_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    topp_kernel<128><<<grid, 256, smem, st>>>(qbar, kbar, m, p, scale, fc, bits, counts, tile_cost);
+  } else {
+    e = cudaFuncSetAttribute(topp_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    topp_kernel<64><<<grid, 256, smem, st>>>(qbar, kbar, m, p, scale, fc, bits, counts, tile_cost);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,
+                         double* qf, double* kf, const Dims& m, int frame_len, int topk, double scale,
+                         const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
+                         cudaStream_t st) {
+  dim3 g1((unsigned)m.F, (unsigned)m.BH, 2);
+  const size_t smem = frame_smem_bytes(m);
+  cudaError_t e;
+  if (m.d == 128) {
+    frame_means_kernel<128><<<g1, 128, 0, st>>>(qlo, qhi, klo, khi, m, frame_len, qf, kf);
+    e = cudaFuncSetAttribute(frame_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    frame_select_kernel<128><<<(unsigned)m.BH, 256, smem, st>>>(qf, kf, m, frame_len, topk, scale, fc, bits, counts,
+                                                                tile_cost);
+  } else {
+    frame_means_kernel<64><<<g1, 64, 0, st>>>(qlo, qhi, klo, khi, m, frame_len, qf, kf);
+    e = cudaFuncSetAttribute(frame_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    frame_select_kernel<64><<<(unsigned)m.BH, 256, smem, st>>>(qf, kf, m, frame_len, topk, scale, fc, bits, counts,
+                                                               tile_cost);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_schedule(const int32_t* counts, const int32_t* tile_cost, const Dims& m, int32_t* row_ptr,
+                            int64_t* head_load, int64_t* nnz, int32_t* tile_order, int64_t capacity,
+                            int32_t* status, cudaStream_t st) {
+  int groups = 32;
+  const size_t smem = schedule_smem_bytes(m, &groups);
+  cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  schedule_kernel<<<1, 1024, smem, st>>>(counts, tile_cost, m, groups, row_ptr, head_load, nnz, tile_order,
+                                         capacity, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_csr(const uint32_t* bits, const int32_t* row_ptr, const Dims& m, int32_t* col_idx,
+                       int64_t capacity, int nsm, cudaStream_t st) {
+  const int64_t rows = m.BH * m.nb;
+  const int grid = (int)imin<int64_t>((rows + 7) / 8, (int64_t)nsm * 8);
+  csr_kernel<<<grid, 256, 0, st>>>(bits, row_ptr, m, col_idx, capacity);
+  return cudaGetLastError();
+}
+
+}  // namespace fv

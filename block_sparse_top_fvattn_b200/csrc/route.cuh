@@ -1,0 +1,40 @@
+// Launchers of the router kernels (route.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace fv {
+
+// Forced-block settings of fvattn_route_cfg, as the kernels use them.
+struct ForceCfg {
+  int force_diag, local_window, frame_len, frame_window, force_first;
+};
+
+size_t topp_smem_bytes(const Dims& m);
+size_t frame_smem_bytes(const Dims& m);
+size_t schedule_smem_bytes(const Dims& m, int* groups);
+
+cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int frame_len,
+                        double* qlo, double* klo, double* qhi, double* khi, int nsm, cudaStream_t st);
+cudaError_t launch_topp(const double* qbar, const double* kbar, const Dims& m, double p, double scale,
+                        const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
+                        cudaStream_t st);
+cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,
+                         double* qf, double* kf, const Dims& m, int frame_len, int topk, double scale,
+                         const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
+                         cudaStream_t st);
+cudaError_t launch_schedule(const int32_t* counts, const int32_t* tile_cost, const Dims& m, int32_t* row_ptr,
+                            int64_t* head_load, int64_t* nnz, int32_t* tile_order, int64_t capacity,
+                            int32_t* status, cudaStream_t st);
+cudaError_t launch_csr(const uint32_t* bits, const int32_t* row_ptr, const Dims& m, int32_t* col_idx,
+                       int64_t capacity, int nsm, cudaStream_t st);
+
+// Attention (attn_f32.cu, attn_tc.cu).
+cudaError_t launch_attn_f32(const float* Q, const float* K, const float* V, const Dims& m, float scale,
+                            const int32_t* row_ptr, const int32_t* col_idx, float* O, float* lse,
+                            cudaStream_t st);
+cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const Dims& m, float scale,
+                           const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_order,
+                           int32_t* control, void* O, float* lse, int nsm, cudaStream_t st);
+
+}  // namespace fv

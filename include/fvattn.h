@@ -1,0 +1,177 @@
+/*
+ * fvattn.h -- C ABI of libfvattn.so: Top-p block routing and block-sparse attention for
+ * video-DiT self-attention on NVIDIA B200 (sm_100a).
+ *
+ * The method (FVAttn blog summary "腾讯+中山大学新作：视频生成提速2.11×，靠的是RLB和SASA",
+ * section "AI视频生成的阿喀琉斯之踵"): split the key/value sequence into fixed blocks, score
+ * every key block for each query block, keep the smallest set of blocks, in descending
+ * importance, whose cumulative importance reaches p, and run exact softmax attention over
+ * the kept blocks only. Block scores are the scaled dot products of block-mean vectors
+ * (video-generation acceleration notes, wzjinhao.cn, §5.2 "块稀疏注意力的教学实现").
+ *
+ * Conventions for every entry point:
+ *  - Tensors Q, K, V, O are dense row-major [B, H, S, d] device arrays (the notes' [B,H,L,D]
+ *    layout, §5.2), element type given by fvattn_shape.dtype, base 16-byte aligned.
+ *  - The caller owns and allocates every buffer. The library never allocates or frees
+ *    memory and never synchronises, except fvattn_read_status. All work is enqueued on the
+ *    caller's stream, in order; the calls can be captured into a CUDA graph by the caller.
+ *  - Argument errors are detected on the host, before any launch, and returned as a negative
+ *    fvattn_status; nothing is enqueued then. A failed launch returns FVATTN_ERR_CUDA.
+ *    Errors found on the device (capacity exceeded, a bounded wait that ran out) are written
+ *    to the device status word (fvattn_csr.status[0]) and read with fvattn_read_status.
+ *  - Not thread-safe for concurrent calls that share output or workspace buffers.
+ */
+#ifndef FVATTN_H
+#define FVATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+struct CUstream_st;
+typedef struct CUstream_st* fvattn_stream_t;
+
+typedef enum {
+  FVATTN_OK = 0,
+  FVATTN_ERR_INVALID = -1,      /* bad argument: null pointer, size, range, alignment      */
+  FVATTN_ERR_UNSUPPORTED = -2,  /* valid but not implemented (block != 64, d not 64/128)   */
+  FVATTN_ERR_CAPACITY = -3,     /* an output or workspace buffer is too small              */
+  FVATTN_ERR_CUDA = -4,         /* a CUDA runtime call or launch failed                    */
+  FVATTN_ERR_TIMEOUT = -5       /* a bounded device-side wait ran out (device status only) */
+} fvattn_status;
+
+typedef enum { FVATTN_BF16 = 0, FVATTN_F32 = 1 } fvattn_dtype;
+
+typedef enum {
+  FVATTN_MODE_TOPP = 0,        /* FVAttn Top-p over key blocks                             */
+  FVATTN_MODE_FRAME_TOPK = 1   /* Sol-Attn frame-level top-k (vLLM-Omni article §2.1-§2.2) */
+} fvattn_mode;
+
+/* Problem shape. block must be 64; d must be 64 or 128; scale <= 0 means 1/sqrt(d). */
+typedef struct {
+  int64_t B, H, S, d;
+  int32_t block;
+  int32_t dtype;     /* fvattn_dtype */
+  float scale;
+} fvattn_shape;
+
+/*
+ * Routing configuration.
+ *  mode              fvattn_mode.
+ *  p                 Top-p threshold in (0, 1]; p >= 1 keeps every key block (dense).
+ *  force_diag        1: key block i is always kept for query block i.
+ *  local_window      w > 0 keeps the band |i - j| <= w (notes §5.2, "邻近块保底"); 0: none.
+ *  frame_len         tokens per latent frame; 0: no frame structure. Frame mode needs >= 64.
+ *  topk_frames       frame mode: frames kept per query frame by score (>= 1).
+ *  frame_window      fw >= 0 keeps the frames within +-fw of the query block's frames
+ *                    (Sol-Attn §2.2, neighbouring frames); -1 disables.
+ *  force_first_frame 1: the blocks of frame 0 are always kept (Sol-Attn §5.2).
+ * Forced blocks are added after the Top-p cut (a union); they do not count toward p.
+ */
+typedef struct {
+  int32_t mode;
+  float p;
+  int32_t force_diag;
+  int32_t local_window;
+  int32_t frame_len;
+  int32_t topk_frames;
+  int32_t frame_window;
+  int32_t force_first_frame;
+} fvattn_route_cfg;
+
+/*
+ * Router output, all device buffers owned by the caller. With nb = ceil(S/64), BH = B*H,
+ * ntiles = BH * ceil(nb/2) (a tile is 128 query rows: query blocks 2t and 2t+1 of one head):
+ *  row_ptr    int32 [BH*nb + 1]   CSR row offsets; row = bh*nb + i.
+ *  col_idx    int32 [col_capacity] selected key blocks of each row, ascending.
+ *  col_capacity                   must be >= fvattn_csr_max_nnz(shape).
+ *  head_load  int64 [BH]          selected (query block, key block) pairs per head: the unit
+ *                                 of the FVAttn runtime load balancer (blog section "RLB").
+ *  tile_cost  int32 [ntiles]      distinct key blocks a 128-row tile visits (union of its
+ *                                 two rows).
+ *  tile_order int32 [ntiles]      tile ids (bh*ceil(nb/2) + t) by cost, largest first, ties
+ *                                 by ascending id: the longest-processing-time order in which
+ *                                 the attention kernel's persistent CTAs take tiles.
+ *  nnz        int64 [1]           total selected pairs (= row_ptr[BH*nb]).
+ *  status     int32 [4]           control block: [0] device status (fvattn_status), [1] error
+ *                                 detail, [2] tile ticket of the attention scheduler, [3] 0.
+ */
+typedef struct {
+  int32_t* row_ptr;
+  int32_t* col_idx;
+  int64_t col_capacity;
+  int64_t* head_load;
+  int32_t* tile_cost;
+  int32_t* tile_order;
+  int64_t* nnz;
+  int32_t* status;
+} fvattn_csr;
+
+/* Library version, (major << 16) | minor. */
+int fvattn_version(void);
+
+/* Static text for a status code. Never NULL. */
+const char* fvattn_status_string(int status);
+
+/* BH * nb * nb: the largest possible nnz, hence the col_idx capacity to allocate.
+ * Returns a negative fvattn_status for an invalid shape. Host only, no CUDA call. */
+int64_t fvattn_csr_max_nnz(const fvattn_shape* shape);
+
+/* BH * ceil(nb/2): entries of tile_cost and tile_order. Negative status if invalid. */
+int64_t fvattn_num_tiles(const fvattn_shape* shape);
+
+/* Workspace bytes fvattn_route needs for this shape and configuration (block means in
+ * fp64, per-row selection bitmasks and counts). 0 on invalid arguments. Host only. */
+size_t fvattn_route_workspace_bytes(const fvattn_shape* shape, const fvattn_route_cfg* cfg);
+
+/*
+ * fvattn_route -- the router (FVAttn Top-p, or Sol-Attn frame top-k), all on the device:
+ *   1. block means of Q and K over the valid tokens of each 64-token block (notes §5.2),
+ *      accumulated exactly enough to be held in fp64;
+ *   2. Top-p: scores Sc[i][j] = <Qbar_i, Kbar_j> * scale in fp64, softmax over j, and the
+ *      smallest descending-probability prefix whose mass is >= p (ties: lower j first);
+ *      frame mode: frame means, frame scores, top-k frames per query frame, expanded to the
+ *      key blocks that hold tokens of a kept frame;
+ *   3. union with the forced blocks of cfg; CSR rows (ascending), per-head loads, tile
+ *      costs and the longest-first tile order.
+ * Q, K: device [B,H,S,d]; out: caller buffers as above; workspace: device, at least
+ * fvattn_route_workspace_bytes(shape, cfg) bytes, 256-byte aligned, contents need not be
+ * initialised. Returns FVATTN_OK once everything is enqueued on `stream`.
+ */
+int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape,
+                 const fvattn_route_cfg* cfg, const fvattn_csr* out,
+                 void* workspace, size_t workspace_bytes, fvattn_stream_t stream);
+
+/*
+ * fvattn_sparse_attn -- exact softmax attention over the selected key blocks:
+ *   O[t] = sum_u softmax_u(Q[t].K[u] * scale) V[u],  u over the tokens (< S) of the key
+ *   blocks listed in the CSR row of t's query block.
+ * csr: the output of fvattn_route on the same shape (row_ptr, col_idx, tile_order, status
+ * are read; status[2] is reset and used as the work ticket). O: device [B,H,S,d], same
+ * dtype as Q. lse: optional device float [B,H,S] receiving the natural-log softmax
+ * normaliser of each row (NULL to skip). bf16 runs on the tensor cores (tcgen05, fp32
+ * accumulation); f32 runs on the CUDA cores in fp32.
+ */
+int fvattn_sparse_attn(const void* Q, const void* K, const void* V, const fvattn_shape* shape,
+                       const fvattn_csr* csr, void* O, float* lse, fvattn_stream_t stream);
+
+/*
+ * fvattn_block_means -- step 1 of fvattn_route on its own: means of X [B,H,S,d] over the
+ * valid tokens of each 64-token block, written as fp64 [B,H,nb,d] to `out` (device).
+ */
+int fvattn_block_means(const void* X, const fvattn_shape* shape, double* out,
+                       fvattn_stream_t stream);
+
+/* Synchronises `stream`, then returns the device status word status[0] (FVATTN_OK or a
+ * negative fvattn_status written by a kernel). FVATTN_ERR_CUDA if the copy fails. */
+int fvattn_read_status(const fvattn_csr* csr, fvattn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FVATTN_H */
