@@ -293,7 +293,7 @@ def run_ours(args, w):
 
     # end to end through the public API with host buffers (pinned), copies inside the region
     e2e = None
-    if rank == 0 or world > 1:
+    if not args.no_e2e:
         hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
         ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -371,9 +371,13 @@ def main():
     ap.add_argument("--workload", default="dit")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling case)")
     args = ap.parse_args()
     from workloads import get_workload
     w = get_workload(args.workload)
+    if args.heads:
+        w = w.replace(H=args.heads)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)
