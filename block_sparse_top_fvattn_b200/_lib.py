@@ -74,6 +74,8 @@ def load() -> ctypes.CDLL:
     lib.fvattn_block_means.argtypes = [vp, P(Shape), vp, vp]
     lib.fvattn_read_status.restype = ctypes.c_int
     lib.fvattn_read_status.argtypes = [P(Csr), vp]
+    lib.fvattn_route_static_scratch.restype = ctypes.c_int
+    lib.fvattn_route_static_scratch.argtypes = [vp, vp, P(Shape), P(RouteCfg), P(Csr), vp]
     _lib = lib
     return lib
 

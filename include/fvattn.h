@@ -170,6 +170,26 @@ int fvattn_block_means(const void* X, const fvattn_shape* shape, double* out,
  * negative fvattn_status written by a kernel). FVATTN_ERR_CUDA if the copy fails. */
 int fvattn_read_status(const fvattn_csr* csr, fvattn_stream_t stream);
 
+/*
+ * fvattn_route_static_scratch -- fvattn_route without a caller workspace. The pages have no
+ * counterpart of this call; it exists for callers that cannot allocate device memory: hosts
+ * that own all device memory through their own fixed pool, or plugin interfaces that pass a
+ * library only its input and output pointers, leave no way to obtain a workspace.
+ *
+ * The router's scratch is a static device array of FVATTN_STATIC_SCRATCH_BYTES that every
+ * GPU loading the library holds until the process exits; nothing is allocated or freed.
+ * Sizes whose fvattn_route_workspace_bytes exceeds it return FVATTN_ERR_CAPACITY (8 MiB
+ * covers, e.g., B*H = 12 heads at S = 8192, d = 128 in Top-p mode). The first call on each
+ * device looks up the array's device address (cudaGetSymbolAddress, device current); make
+ * that first call before any stream capture. All calls share the one array: calls that
+ * overlap on the GPU (other streams, other threads) race and must be serialised by the
+ * caller. Q, K, shape, cfg, out and stream are as for fvattn_route.
+ */
+#define FVATTN_STATIC_SCRATCH_BYTES (8u << 20)
+int fvattn_route_static_scratch(const void* Q, const void* K, const fvattn_shape* shape,
+                                const fvattn_route_cfg* cfg, const fvattn_csr* out,
+                                fvattn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
