@@ -30,7 +30,7 @@ namespace fv {
 
 namespace {
 
-constexpr int NS = 4;                        // K/V pipeline stages
+constexpr int NS = 2;                        // K/V pipeline stages (two CTAs share an SM)
 constexpr uint32_t kWaitLimit = 1u << 22;    // polls of a bounded wait (seconds, not minutes)
 constexpr float kRescaleLog2 = 8.0f;         // raise the running max only when it grows by > 2^8
 
@@ -41,22 +41,23 @@ struct TcLayout {
   static constexpr int kKVChunk = kBlock * 128;       // [64 rows x 64 dims] bf16 = 8 KB
   static constexpr int kKBytes = (D / 64) * kKVChunk;
   static constexpr int kStage = 2 * kKBytes;          // K_j and V_j
-  static constexpr int kPBytes = kTileRows * 128;     // [128 rows x 64 keys] bf16 = 16 KB
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = kQBytes;
-  static constexpr int kOffP = kOffKV + NS * kStage;
-  static constexpr int kOffBar = kOffP + 2 * kPBytes;
+  static constexpr int kOffBar = kOffKV + NS * kStage;
   static constexpr int kBytes = kOffBar + 512;
-  static constexpr uint32_t kTmemCols = 256;          // S[2] at columns 0 and 64, O at 128
+  // TMEM: S double buffer at columns 0 and 64 (P, bf16, overwrites the first 32 columns of its
+  // S buffer), O at column 128.
+  static constexpr uint32_t kTmemCols = 256;
   static constexpr uint32_t kColO = 128;
 };
 
 struct TcBars {
   uint64_t q_full, q_empty;
   uint64_t kv_full[NS], kv_empty[NS];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], pv_done[2];
+  uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t o_full, o_empty;
+  uint64_t sched_full[2], sched_empty[2];
+  int sched_tile[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -107,13 +108,33 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Packed pairs of fp32 (one 64-bit register): two FMAs / adds per instruction.
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, Dims m, float scale_log2,
                    const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
@@ -126,7 +147,6 @@ __global__ void __launch_bounds__(192, 1)
   TcBars* bars = reinterpret_cast<TcBars*>(smem + L::kOffBar);
   unsigned char* sQ = smem + L::kOffQ;
   unsigned char* sKV = smem + L::kOffKV;
-  unsigned char* sP = smem + L::kOffP;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ntiles = m.BH * m.nt;
   volatile int* abort = &bars->abort;
@@ -140,9 +160,10 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->s_full[s], 1);
-      tc::mbar_init(&bars->s_empty[s], 4);
       tc::mbar_init(&bars->p_full[s], 4);
       tc::mbar_init(&bars->pv_done[s], 1);
+      tc::mbar_init(&bars->sched_full[s], 1);
+      tc::mbar_init(&bars->sched_empty[s], 5);    // the MMA thread and the four softmax warps
     }
     tc::mbar_init(&bars->o_full, 1);
     tc::mbar_init(&bars->o_empty, 4);
@@ -164,15 +185,26 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tbase = bars->tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ scheduler + TMA producer
+    // Takes the next tile of the longest-first order from the global ticket, publishes it to
+    // the other roles, and streams its Q tile and K_j / V_j blocks.
     if (lane == 0) {
-      uint32_t g = 0, tcount = 0;
-      for (int64_t k = blockIdx.x; k < ntiles && !*abort; k += gridDim.x, ++tcount) {
-        const int tile = tile_order[k];
-        if (tile < 0 || tile >= ntiles) { fail(bars, 11); break; }
+      uint32_t g = 0;
+      for (uint32_t n = 0;; ++n) {
+        const int s = n & 1;
+        if (!tc::mbar_wait(&bars->sched_empty[s], ((n >> 1) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 1); break; }
+        const int k = atomicAdd(&control[2], 1);
+        int tile = -1;
+        if (k < ntiles) {
+          tile = tile_order[k];
+          if (tile < 0 || tile >= ntiles) { fail(bars, 11); tile = -1; }
+        }
+        bars->sched_tile[s] = tile;
+        tc::mbar_arrive(&bars->sched_full[s]);
+        if (tile < 0) break;
         const int64_t bh = tile / m.nt;
         const int t = (int)(tile - bh * m.nt);
-        if (!tc::mbar_wait(&bars->q_empty, (tcount & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 1); break; }
+        if (!tc::mbar_wait(&bars->q_empty, (n & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 2); break; }
         tc::mbar_expect_tx(&bars->q_full, L::kQBytes);
         for (int c = 0; c < D / 64; ++c)
           for (int h = 0; h < 2; ++h)
@@ -180,9 +212,10 @@ __global__ void __launch_bounds__(192, 1)
                             t * kTileRows + h * kBlock, (int)bh);
         PairMerge mg(row_ptr, col_idx, bh, t, m.nb);
         int j, mask;
+        bool ok = true;
         while (mg.next(j, mask)) {
           const int st = g % NS;
-          if (!tc::mbar_wait(&bars->kv_empty[st], ((g / NS) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 2); break; }
+          if (!tc::mbar_wait(&bars->kv_empty[st], ((g / NS) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 3); ok = false; break; }
           unsigned char* sK = sKV + st * L::kStage;
           unsigned char* sV = sK + L::kKBytes;
           tc::mbar_expect_tx(&bars->kv_full[st], L::kStage);
@@ -192,50 +225,50 @@ __global__ void __launch_bounds__(192, 1)
           }
           ++g;
         }
+        if (!ok) break;
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Issue order per tile: S_0, [S_1, PV_0], [S_2, PV_1], ..., PV_last. MMAs of one thread run
+    // in issue order, so S_{i+2} (same TMEM buffer as S_i / P_i) always follows PV_i.
     if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16_f32(kTileRows, kBlock, 0, 0);
       constexpr uint32_t idO = tc::idesc_bf16_f32(kTileRows, D, 0, 1);
-      const uint32_t qaddr = tc::smem_u32(sQ), kvaddr = tc::smem_u32(sKV), paddr = tc::smem_u32(sP);
-      uint32_t g = 0, tcount = 0;
+      const uint32_t qaddr = tc::smem_u32(sQ), kvaddr = tc::smem_u32(sKV);
+      uint32_t g = 0, n = 0;
       bool ok = true;
       // O += P_gs V_gs for step gs; `first` = first step of the tile (overwrites O).
       auto pv = [&](uint32_t gs, bool first) -> bool {
         const int pb = gs & 1;
         if (!tc::mbar_wait(&bars->p_full[pb], (gs >> 1) & 1, abort, kWaitLimit)) return false;
-        if (first && !tc::mbar_wait(&bars->o_empty, (tcount & 1) ^ 1, abort, kWaitLimit)) return false;
+        if (first && !tc::mbar_wait(&bars->o_empty, (n & 1) ^ 1, abort, kWaitLimit)) return false;
         tc::fence_after_sync();
         const uint32_t vaddr = kvaddr + (gs % NS) * L::kStage + L::kKBytes;
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk) {
-          const uint64_t a = tc::smem_desc_sw128(paddr + pb * L::kPBytes + kk * 32, 16, 1024);
           const uint64_t b = tc::smem_desc_sw128(vaddr + kk * 16 * 128, L::kKVChunk, 1024);
-          tc::mma_f16(tbase + L::kColO, a, b, idO, (first && kk == 0) ? 0u : 1u);
+          tc::mma_f16_tmem_a(tbase + L::kColO, tbase + pb * kBlock + kk * 8, b, idO, (first && kk == 0) ? 0u : 1u);
         }
         tc::mma_commit(&bars->pv_done[pb]);
         tc::mma_commit(&bars->kv_empty[gs % NS]);
         return true;
       };
-      for (int64_t k = blockIdx.x; k < ntiles && ok; k += gridDim.x, ++tcount) {
-        const int tile = tile_order[k];
-        if (tile < 0 || tile >= ntiles) { fail(bars, 11); break; }
+      for (;; ++n) {
+        const int s = n & 1;
+        if (!tc::mbar_wait(&bars->sched_full[s], (n >> 1) & 1, abort, kWaitLimit)) { fail(bars, 4); ok = false; break; }
+        const int tile = bars->sched_tile[s];
+        tc::mbar_arrive(&bars->sched_empty[s]);
+        if (tile < 0) break;
         const int64_t bh = tile / m.nt;
         const int t = (int)(tile - bh * m.nt);
-        if (!tc::mbar_wait(&bars->q_full, tcount & 1, abort, kWaitLimit)) { fail(bars, 3); ok = false; break; }
+        if (!tc::mbar_wait(&bars->q_full, n & 1, abort, kWaitLimit)) { fail(bars, 5); ok = false; break; }
         PairMerge mg(row_ptr, col_idx, bh, t, m.nb);
         int j, mask, i = 0;
         while (mg.next(j, mask)) {
           const uint32_t gi = g + i;
           const int st = gi % NS, sb = gi & 1;
-          if (!tc::mbar_wait(&bars->kv_full[st], (gi / NS) & 1, abort, kWaitLimit) ||
-              !tc::mbar_wait(&bars->s_empty[sb], ((gi >> 1) & 1) ^ 1, abort, kWaitLimit)) {
-            fail(bars, 4);
-            ok = false;
-            break;
-          }
+          if (!tc::mbar_wait(&bars->kv_full[st], (gi / NS) & 1, abort, kWaitLimit)) { fail(bars, 6); ok = false; break; }
           tc::fence_after_sync();
           const uint32_t kaddr = kvaddr + st * L::kStage;
 #pragma unroll
@@ -246,110 +279,114 @@ __global__ void __launch_bounds__(192, 1)
             tc::mma_f16(tbase + sb * kBlock, a, b, idS, kk > 0 ? 1u : 0u);
           }
           tc::mma_commit(&bars->s_full[sb]);
-          if (i > 0 && !pv(gi - 1, i == 1)) { fail(bars, 5); ok = false; break; }
+          if (i > 0 && !pv(gi - 1, i == 1)) { fail(bars, 7); ok = false; break; }
           ++i;
         }
         if (!ok) break;
         tc::mma_commit(&bars->q_empty);          // every S of this tile issued: Q may be replaced
-        if (i > 0 && !pv(g + i - 1, i == 1)) { fail(bars, 6); ok = false; break; }
+        if (i > 0 && !pv(g + i - 1, i == 1)) { fail(bars, 8); ok = false; break; }
         tc::mma_commit(&bars->o_full);
         g += i;
       }
       // Drain: every MMA issued so far has completed before TMEM can be released.
-      if (ok && tcount > 0) tc::mbar_wait(&bars->o_full, (tcount - 1) & 1, abort, kWaitLimit);
+      if (ok && n > 0) tc::mbar_wait(&bars->o_full, (n - 1) & 1, abort, kWaitLimit);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;             // tile row == TMEM lane
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const bool lo_half = r < kBlock;
-    uint32_t g = 0, tcount = 0;
-    for (int64_t k = blockIdx.x; k < ntiles; k += gridDim.x, ++tcount) {
-      const int tile = tile_order[k];
-      if (tile < 0 || tile >= ntiles) { fail(bars, 11); break; }
+    const int half_bit = (r < kBlock) ? 1 : 2;   // rows 0-63: query block 2t, 64-127: 2t+1
+    const uint64_t scale2 = f2(scale_log2, scale_log2);
+    uint32_t g = 0;
+    for (uint32_t n = 0;; ++n) {
+      const int s = n & 1;
+      if (!warp_wait(&bars->sched_full[s], (n >> 1) & 1, abort)) { fail(bars, 9); break; }
+      const int tile = bars->sched_tile[s];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bars->sched_empty[s]);
+      if (tile < 0) break;
       const int64_t bh = tile / m.nt;
       const int t = (int)(tile - bh * m.nt);
-      float mrow = -INFINITY, lrow = 0.f;
+      float mrow = -INFINITY;
+      uint64_t lsum = f2(0.f, 0.f);
       PairMerge mg(row_ptr, col_idx, bh, t, m.nb);
       int j, mask, i = 0;
       bool ok = true;
       while (mg.next(j, mask)) {
         const uint32_t gi = g + i;
         const int sb = gi & 1;
-        if (!warp_wait(&bars->s_full[sb], (gi >> 1) & 1, abort)) { fail(bars, 7); ok = false; break; }
+        const uint32_t sp = tbase + lane_off + sb * kBlock;     // S_i, then P_i, of this row
+        if (!warp_wait(&bars->s_full[sb], (gi >> 1) & 1, abort)) { fail(bars, 10); ok = false; break; }
         tc::fence_after_sync();
-        uint32_t sraw[64];
-        {
-          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]);
-          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]);
-          tc::tmem_ld32(tbase + lane_off + sb * kBlock, lo);
-          tc::tmem_ld32(tbase + lane_off + sb * kBlock + 32, hi);
-          tc::tmem_ld_wait();
-        }
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&bars->s_empty[sb]);
-
-        const bool sel = lo_half ? (mask & 1) : (mask & 2);
-        const int nk = (int)imin<int64_t>(kBlock, m.S - (int64_t)j * kBlock);
-        float x[64];
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          x[c] = (sel && c < nk) ? __uint_as_float(sraw[c]) * scale_log2 : -INFINITY;
-          mx = fmaxf(mx, x[c]);
-        }
-        // Raise the running max only when it grows by more than 2^8 (or on the row's first
-        // kept block); rows whose O already holds earlier blocks then scale O in TMEM.
-        const bool raise = sel && (mrow == -INFINITY || mx > mrow + kRescaleLog2);
-        const bool scale_o = raise && i > 0 && mrow != -INFINITY;
-        if (__any_sync(0xffffffffu, scale_o)) {
-          // tcgen05.ld/st are warp-collective: the whole warp takes part, each lane with its
-          // own factor (1 for rows that keep their max).
-          const uint32_t gp = gi - 1;
-          if (!warp_wait(&bars->pv_done[gp & 1], (gp >> 1) & 1, abort)) { fail(bars, 8); ok = false; break; }
-          tc::fence_after_sync();
-          const float alpha = scale_o ? ex2(mrow - mx) : 1.f;
-#pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            tc::tmem_ld32(tbase + lane_off + L::kColO + cc * 32, o);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tc::tmem_st32(tbase + lane_off + L::kColO + cc * 32, o);
-          }
-          tc::tmem_st_wait();
-          lrow *= alpha;
-        }
-        if (raise) mrow = mx;
         uint32_t packed[32];
+        const bool sel = (mask & half_bit) != 0;               // uniform across the warp
         if (sel) {
-#pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            const float p0 = ex2(x[c] - mrow);
-            const float p1 = ex2(x[c + 1] - mrow);
-            lrow += p0 + p1;
-            packed[c >> 1] = pack_bf16(p0, p1);
+          uint32_t sraw[64];
+          {
+            uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]);
+            uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]);
+            tc::tmem_ld32(sp, lo);
+            tc::tmem_ld32(sp + 32, hi);
+            tc::tmem_ld_wait();
           }
+          const int nk = (int)imin<int64_t>(kBlock, m.S - (int64_t)j * kBlock);
+          if (nk < kBlock) {                                   // ragged last block: keys >= S
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (c >= nk) sraw[c] = __float_as_uint(-INFINITY);
+          }
+          float mx8[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(sraw[c]);
+#pragma unroll
+          for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sraw[c]));
+          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
+          // Raise the running max only when it grows by more than 2^8 (or on the row's first
+          // kept block); rows whose O already holds earlier blocks then scale O in TMEM.
+          const bool raise = mrow == -INFINITY || mx > mrow + kRescaleLog2;
+          const bool scale_o = raise && i > 0 && mrow != -INFINITY;
+          if (__any_sync(0xffffffffu, scale_o)) {
+            // tcgen05.ld/st are warp-collective: the whole warp takes part, each lane with its
+            // own factor (1 for rows that keep their max).
+            const uint32_t gp = gi - 1;
+            if (!warp_wait(&bars->pv_done[gp & 1], (gp >> 1) & 1, abort)) { fail(bars, 12); ok = false; break; }
+            tc::fence_after_sync();
+            const float alpha = scale_o ? ex2(mrow - mx) : 1.f;
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t o[32];
+              tc::tmem_ld32(tbase + lane_off + L::kColO + cc * 32, o);
+              tc::tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tc::tmem_st32(tbase + lane_off + L::kColO + cc * 32, o);
+            }
+            tc::tmem_st_wait();
+            float l0, l1;
+            f2_split(lsum, l0, l1);
+            lsum = f2(l0 * alpha, l1 * alpha);
+          }
+          if (raise) mrow = mx;
+          const uint64_t negm = f2(-mrow, -mrow);
+          uint64_t acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            float x0, x1;
+            f2_split(ffma2(f2(__uint_as_float(sraw[2 * c]), __uint_as_float(sraw[2 * c + 1])), scale2, negm), x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            acc[c & 3] = fadd2(acc[c & 3], f2(p0, p1));
+            packed[c] = pack_bf16(p0, p1);
+          }
+          lsum = fadd2(lsum, fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])));
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) packed[c] = 0u;
         }
-        if (gi >= 2) {       // P buffer sb was last read by the P.V of step gi-2
-          const uint32_t gp = gi - 2;
-          if (!warp_wait(&bars->pv_done[sb], (gp >> 1) & 1, abort)) { fail(bars, 9); ok = false; break; }
-        }
-        // Row r of P in the 128-byte-swizzled K-major layout: 16-byte chunk c of the row goes
-        // to chunk position c ^ (r mod 8).
-        unsigned char* prow = sP + sb * L::kPBytes + r * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 v = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = v;
-        }
-        tc::fence_proxy_async_smem();
+        // P_i (bf16 pairs) over the first 32 columns of its S buffer; S_i is already in registers.
+        tc::tmem_st32(sp, packed);
+        tc::tmem_st_wait();
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&bars->p_full[sb]);
@@ -357,8 +394,11 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (__any_sync(0xffffffffu, !ok || *abort)) break;
       // ---------------------------------------------------------- epilogue
-      if (!warp_wait(&bars->o_full, tcount & 1, abort)) { fail(bars, 10); break; }
+      if (!warp_wait(&bars->o_full, n & 1, abort)) { fail(bars, 13); break; }
       tc::fence_after_sync();
+      float l0, l1;
+      f2_split(lsum, l0, l1);
+      const float lrow = l0 + l1;
       const int64_t trow = (int64_t)t * kTileRows + r;
       const bool valid = trow < m.S;
       const float inv = 1.f / lrow;
@@ -435,7 +475,7 @@ cudaError_t launch_tc_d(const void* Q, const void* K, const void* V, const Dims&
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t ntiles = m.BH * m.nt;
-  const int grid = (int)imin<int64_t>(ntiles, (int64_t)nsm);
+  const int grid = (int)imin<int64_t>(ntiles, (int64_t)nsm * 2);
   attn_tc_kernel<D><<<grid, 192, smem, st>>>(mq, mk, mv, m, scale * 1.4426950408889634f, row_ptr, col_idx,
                                              tile_order, control, static_cast<__nv_bfloat16*>(O), lse);
   return cudaGetLastError();
