@@ -37,6 +37,7 @@ int validate_cfg(const fvattn_shape* s, const fvattn_route_cfg* c) {
   if (c->force_diag != 0 && c->force_diag != 1) return FVATTN_ERR_INVALID;
   if (c->force_first_frame != 0 && c->force_first_frame != 1) return FVATTN_ERR_INVALID;
   if ((c->frame_window >= 0 || c->force_first_frame) && c->frame_len == 0) return FVATTN_ERR_INVALID;
+  if (c->mode == FVATTN_MODE_TOPP && (s->S + kBlock - 1) / kBlock > 1536) return FVATTN_ERR_UNSUPPORTED;
   if (c->mode == FVATTN_MODE_FRAME_TOPK) {
     if (c->frame_len < kBlock || c->topk_frames < 1) return FVATTN_ERR_INVALID;
     const int64_t F = (s->S + c->frame_len - 1) / c->frame_len;
@@ -58,7 +59,7 @@ size_t take(size_t& off, size_t bytes) {
 WsLayout ws_layout(const Dims& m, int mode) {
   WsLayout L{};
   size_t off = 0;
-  const size_t means = (size_t)m.BH * m.nb * m.d * sizeof(double);
+  const size_t means = (mode == FVATTN_MODE_TOPP ? means_t_elems(m) : (size_t)m.BH * m.nb * m.d) * sizeof(double);
   L.qlo = take(off, means);
   L.klo = take(off, means);
   if (mode == FVATTN_MODE_FRAME_TOPK) {
@@ -153,7 +154,7 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const 
   if (cudaMemsetAsync(out->status, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
   cudaError_t e;
   if (cfg->mode == FVATTN_MODE_TOPP) {
-    e = launch_pool(Q, K, 2, shape->dtype, m, 0, qlo, klo, nullptr, nullptr, nsm, s);
+    e = launch_pool(Q, K, 2, shape->dtype, m, 1, 0, qlo, klo, nullptr, nullptr, nsm, s);
     if (e == cudaSuccess)
       e = launch_topp(qlo, klo, m, cfg->p >= 1.f ? 1.0 : (double)cfg->p, scale, fc, bits, counts, out->tile_cost, s);
   } else {
@@ -161,7 +162,7 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const 
     double* khi = reinterpret_cast<double*>(ws + L.khi);
     double* qf = reinterpret_cast<double*>(ws + L.qf);
     double* kf = reinterpret_cast<double*>(ws + L.kf);
-    e = launch_pool(Q, K, 2, shape->dtype, m, cfg->frame_len, qlo, klo, qhi, khi, nsm, s);
+    e = launch_pool(Q, K, 2, shape->dtype, m, 2, cfg->frame_len, qlo, klo, qhi, khi, nsm, s);
     if (e == cudaSuccess)
       e = launch_frame(qlo, qhi, klo, khi, qf, kf, m, cfg->frame_len, cfg->topk_frames, scale, fc, bits, counts,
                        out->tile_cost, s);
@@ -204,7 +205,7 @@ int fvattn_block_means(const void* X, const fvattn_shape* shape, double* out, fv
   const Dims m = make_dims(*shape, 0);
   const int nsm = num_sms();
   if (nsm <= 0) return FVATTN_ERR_CUDA;
-  cudaError_t e = launch_pool(X, nullptr, 1, shape->dtype, m, 0, out, nullptr, nullptr, nullptr, nsm,
+  cudaError_t e = launch_pool(X, nullptr, 1, shape->dtype, m, 0, 0, out, nullptr, nullptr, nullptr, nsm,
                               reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
 }

@@ -40,12 +40,14 @@ __device__ __forceinline__ T warp_incl_scan(T v, int lane) {
 
 // ------------------------------------------------------------------ K1: block pooling
 //
-// One 64-token block of one tensor per loop iteration. Every thread streams 16-byte vectors
-// of PASSES rows (all loads issued before any use), sums them in AccT (fp32 for bf16 input:
-// a sum of four bf16 values is exact unless their exponents are 16+ apart; fp64 for fp32
-// input), and the row groups are combined in fp64 in a fixed order. Output: fp64 means over
-// the valid tokens, or (frame mode) fp64 sums of the tokens before / after the block's first
-// frame boundary.
+// One warp streams one 64-token block of one tensor. Lane l reads the 16-byte vector
+// c = l mod CPR of rows r0 + RPI*it (r0 = l / CPR); a batch of 16 loads is issued before any
+// is used, so every lane keeps 256 bytes in flight and no barrier is needed. Four rows are
+// summed in AccT (fp32 for bf16 input: exact unless the values' exponents are 16+ apart;
+// fp64 for fp32 input), the partial sums in fp64 in a fixed order, and the row groups of a
+// column are folded with shuffles. OUT selects what is written: means [row][d]; means
+// transposed per head, [bh][d][ld] with ld >= nb (the operand layout of the score GEMM); or
+// fp64 sums of the tokens before / after the block's first frame boundary, [row][d].
 
 template <typename T> struct Acc;
 template <> struct Acc<__nv_bfloat16> { using type = float; static constexpr int kVec = 8; };
@@ -67,78 +69,94 @@ __device__ __forceinline__ void unpack(const uint4& v, double (&o)[4], const flo
   o[3] = __uint_as_float(v.w);
 }
 
-template <typename T, int D, bool FRAME>
-__global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ Q, const T* __restrict__ K,
-                                                   int ntensors, Dims m, int frame_len,
-                                                   double* __restrict__ qlo, double* __restrict__ klo,
+enum PoolOut { kMeans = 0, kMeansT = 1, kFrameSums = 2 };
+
+template <typename T, int D, int OUT>
+__global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ Q, const T* __restrict__ K,
+                                                   int ntensors, Dims m, int frame_len, int ld,
+                                                   double* __restrict__ qo, double* __restrict__ ko,
                                                    double* __restrict__ qhi, double* __restrict__ khi) {
   using AccT = typename Acc<T>::type;
   constexpr int VEC = Acc<T>::kVec;
-  constexpr int CPR = D / VEC;         // 16-byte chunks per row
-  constexpr int RPP = 256 / CPR;       // rows per pass
-  constexpr int PASSES = kBlock / RPP;
-  __shared__ double red[FRAME ? 2 : 1][RPP][D];
-
-  const int tid = threadIdx.x;
-  const int c = tid % CPR, r0 = tid / CPR;
+  constexpr int CPR = D / VEC;         // 16-byte vectors per row
+  constexpr int RPI = 32 / CPR;        // rows per warp-wide load
+  constexpr int NIT = kBlock / RPI;    // loads per lane per block
+  constexpr int BATCH = NIT < 16 ? NIT : 16;
+  constexpr bool FRAME = OUT == kFrameSums;
+  const int lane = threadIdx.x & 31;
+  const int c = lane % CPR, r0 = lane / CPR;
   const int64_t per = m.BH * m.nb;
   const int64_t units = per * ntensors;
-  for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t u = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); u < units; u += nwarps) {
     const bool isK = u >= per;
     const int64_t row = isK ? u - per : u;       // bh * nb + blk
     const int64_t bh = row / m.nb;
     const int blk = (int)(row - bh * m.nb);
     const int64_t t0 = (int64_t)blk * kBlock;
     const int nvalid = (int)imin<int64_t>(kBlock, m.S - t0);
-    const T* X = (isK ? K : Q) + (bh * m.S + t0) * D;
+    const T* X = (isK ? K : Q) + (bh * m.S + t0) * D + c * VEC;
     int boundary = kBlock;
     if (FRAME) boundary = (int)imin<int64_t>(kBlock, (t0 / frame_len + 1) * frame_len - t0);
-
-    uint4 v[PASSES];
+    double lo[VEC], hi[VEC];
 #pragma unroll
-    for (int p = 0; p < PASSES; ++p) {
-      const int r = r0 + p * RPP;
-      if (r < nvalid)
-        v[p] = __ldg(reinterpret_cast<const uint4*>(X + (int64_t)r * D + c * VEC));
-      else
-        v[p] = make_uint4(0, 0, 0, 0);
+    for (int e = 0; e < VEC; ++e) lo[e] = hi[e] = 0.0;
+#pragma unroll
+    for (int b0 = 0; b0 < NIT; b0 += BATCH) {
+      uint4 v[BATCH];
+#pragma unroll
+      for (int it = 0; it < BATCH; ++it) {
+        const int r = r0 + (b0 + it) * RPI;
+        v[it] = r < nvalid ? __ldg(reinterpret_cast<const uint4*>(X + (int64_t)r * D)) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int g = 0; g < BATCH; g += 4) {
+        AccT sl[VEC], sh[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) sl[e] = sh[e] = 0;
+#pragma unroll
+        for (int it = g; it < g + 4; ++it) {
+          AccT x[VEC];
+          unpack(v[it], x, (const T*)nullptr);
+          const bool in_lo = !FRAME || (r0 + (b0 + it) * RPI) < boundary;
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) {
+            if (in_lo) sl[e] += x[e];
+            else sh[e] += x[e];
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          lo[e] += (double)sl[e];
+          if (FRAME) hi[e] += (double)sh[e];
+        }
+      }
     }
-    AccT lo[VEC], hi[VEC];
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) lo[e] = hi[e] = 0;
-#pragma unroll
-    for (int p = 0; p < PASSES; ++p) {
-      AccT x[VEC];
-      unpack(v[p], x, (const T*)nullptr);
-      const bool in_lo = !FRAME || (r0 + p * RPP) < boundary;
+    for (int off = CPR; off < 32; off <<= 1)
 #pragma unroll
       for (int e = 0; e < VEC; ++e) {
-        if (in_lo) lo[e] += x[e];
-        else hi[e] += x[e];
+        lo[e] += __shfl_xor_sync(0xffffffffu, lo[e], off);
+        if (FRAME) hi[e] += __shfl_xor_sync(0xffffffffu, hi[e], off);
       }
-    }
+    if (r0 == 0) {
+      double* o = isK ? ko : qo;
+      if (OUT == kMeans) {
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      red[0][r0][c * VEC + e] = (double)lo[e];
-      if (FRAME) red[FRAME ? 1 : 0][r0][c * VEC + e] = (double)hi[e];
-    }
-    __syncthreads();
-    if (tid < D) {
-      double s = 0.0;
+        for (int e = 0; e < VEC; ++e) o[row * D + c * VEC + e] = lo[e] / (double)nvalid;
+      } else if (OUT == kMeansT) {
+        double* ot = o + bh * (int64_t)D * ld + blk;
 #pragma unroll
-      for (int rr = 0; rr < RPP; ++rr) s += red[0][rr][tid];
-      double* out = (isK ? klo : qlo) + row * D + tid;
-      if (FRAME) {
-        double h = 0.0;
-#pragma unroll
-        for (int rr = 0; rr < RPP; ++rr) h += red[FRAME ? 1 : 0][rr][tid];
-        *out = s;
-        (isK ? khi : qhi)[row * D + tid] = h;
+        for (int e = 0; e < VEC; ++e) ot[(int64_t)(c * VEC + e) * ld] = lo[e] / (double)nvalid;
       } else {
-        *out = s / (double)nvalid;
+        double* oh = isK ? khi : qhi;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          o[row * D + c * VEC + e] = lo[e];
+          oh[row * D + c * VEC + e] = hi[e];
+        }
       }
     }
-    __syncthreads();
   }
 }
 
@@ -194,206 +212,222 @@ __device__ __forceinline__ int finalize_row(uint32_t* w, int i, const Dims& m, c
 
 constexpr int RT = 16;      // query blocks per CTA
 constexpr int KT = 256;     // key blocks per pass of the score tile
-constexpr int KC = 16;      // head-dim chunk staged in shared memory
+constexpr int KC = 8;       // head-dim rows of one pipelined operand chunk
 constexpr int NWARP = 8;
+constexpr int kExtract = 16;   // max-extraction steps before the bisection fallback
 
-// In-place softmax of a row of n logits (fp64): pi_j = exp(s_j - max) / sum.
-__device__ void softmax_row(double* L, int n, int lane) {
-  double mx = -INFINITY;
-  for (int j = lane; j < n; j += 32) mx = fmax(mx, L[j]);
-  mx = warp_max(mx);
-  double z = 0.0;
-  for (int j = lane; j < n; j += 32) {
-    const double e = exp(L[j] - mx);
-    L[j] = e;
-    z += e;
-  }
-  z = warp_sum(z);
-  for (int j = lane; j < n; j += 32) L[j] = L[j] / z;
-  __syncwarp();
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// Order key of a probability weight: the bits of its fp32 rounding (non-negative floats order
+// like their bit patterns).
+__device__ __forceinline__ uint32_t wkey(double e) { return __float_as_uint(__double2float_rn(e)); }
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
-// Probability mass as a 62-bit fixed-point integer, so that every sum below is exact and
-// independent of summation order (rounding: 2^-63 per block).
-__device__ __forceinline__ uint64_t fixmass(double x) {
-  return (uint64_t)__double2ull_rn(x * 4611686018427387904.0);
-}
-
-// Top-p cut of one row of probabilities (one warp). The kept set is the descending prefix
-// (ties: lower index first) of minimal length whose mass reaches p. Positive doubles order
-// like their bit patterns, so the cut is found as the largest key T with
-//   mass{ j : key_j >= T } >= P
-// by an MSB-first radix select over 8-bit digits of the keys (histograms of exact
-// fixed-point mass); then every key > T is kept and as many keys == T, in ascending index,
-// as are needed to reach P. Writes the bitmask words w[0..nw).
-__device__ void topp_select(const double* pi, int n, double p, uint64_t* hm, uint32_t* hc, uint32_t* w,
-                            int lane) {
+// Top-p cut of one row held in shared memory (one warp). On entry E[0..n) are fp64 logits;
+// they are replaced by the weights e_j = 2^((s_j - max) log2 e), computed with the SFU on the
+// fp64 difference (relative error < 3e-7), and the cut compares masses with p * sum(e), so no
+// division is needed. The kept set is the descending prefix (ties: lower index first) of
+// minimal length whose mass reaches p. It is found by extracting maxima (REDUX on the fp32
+// order key, lowest index on ties) until the mass reaches p, which ends within a few steps
+// for peaked rows; flat rows fall back to a bisection over the 32-bit key space for the
+// largest key T with mass{key >= T} >= p, keeping every key > T and, in ascending index, as
+// many keys == T as the mass needs. All sums are fp64 in a fixed order: the result is
+// deterministic. Writes the row's bitmask words w[0..nw).
+__device__ void topp_select(double* E, int n, double p, uint32_t* w, int lane) {
   const int nw = (n + 31) / 32;
-  bool all = p >= 1.0;
-  const uint64_t P = fixmass(p);
-  if (!all) {
-    uint64_t tot = 0;
-    for (int j = lane; j < n; j += 32) tot += fixmass(pi[j]);
-    tot = warp_sum(tot);
-    all = tot < P;      // the whole row falls short of p by rounding: keep everything
-  }
-  if (all) {
+  if (p >= 1.0) {
     for (int q = lane; q < nw; q += 32) w[q] = range_bits(0, n - 1, q);
     __syncwarp();
     return;
   }
-  uint64_t prefix = 0, pmask = 0, above = 0;
-  for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int b = lane; b < 256; b += 32) { hm[b] = 0; hc[b] = 0; }
-    __syncwarp();
-    for (int j = lane; j < n; j += 32) {
-      const uint64_t key = (uint64_t)__double_as_longlong(pi[j]);
-      if ((key & pmask) == prefix) {
-        const int dg = (int)((key >> shift) & 255);
-        atomicAdd(reinterpret_cast<unsigned long long*>(&hm[dg]), (unsigned long long)fixmass(pi[j]));
-        atomicAdd(&hc[dg], 1u);
-      }
-    }
-    __syncwarp();
-    // Lane l holds bins 255-8l .. 248-8l, so scanning lanes upward walks the digits downward.
-    uint64_t lsum = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) lsum += hm[255 - 8 * lane - q];
-    const uint64_t incl = warp_incl_scan(lsum, lane);
-    uint64_t cum = above + (incl - lsum);
-    int found = -1;
-    uint64_t before = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int dg = 255 - 8 * lane - q;
-      const uint64_t nc = cum + hm[dg];
-      if (found < 0 && nc >= P) { found = dg; before = cum; }
-      cum = nc;
-    }
-    const uint32_t bal = __ballot_sync(0xffffffffu, found >= 0);
-    const int src = __ffs(bal) - 1;     // invariant: above < P <= above + candidates' mass
-    const int dg = __shfl_sync(0xffffffffu, found, src);
-    above = __shfl_sync(0xffffffffu, before, src);
-    prefix |= (uint64_t)dg << shift;
-    pmask |= (uint64_t)0xff << shift;
-    const uint32_t cnt = hc[dg];
-    __syncwarp();
-    if (cnt == 1) {      // a single candidate left: it is T
-      uint64_t T = 0;
-      for (int j = lane; j < n; j += 32) {
-        const uint64_t key = (uint64_t)__double_as_longlong(pi[j]);
-        if ((key & pmask) == prefix) T = key;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const uint64_t u = __shfl_xor_sync(0xffffffffu, T, o);
-        T = u > T ? u : T;
-      }
-      prefix = T;
-      pmask = ~0ull;
-      break;
-    }
+  double mx = -INFINITY;
+  for (int j = lane; j < n; j += 32) mx = fmax(mx, E[j]);
+  mx = warp_max(mx);
+  double z = 0.0;
+  for (int j = lane; j < n; j += 32) {
+    float ef;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(ef) : "f"((float)((E[j] - mx) * 1.4426950408889634)));
+    E[j] = (double)ef;
+    z += (double)ef;
   }
-  const uint64_t T = prefix;
-  const uint64_t mT = fixmass(__longlong_as_double((long long)T));
-  const uint64_t need = mT ? (P - above + mT - 1) / mT : 0;
-  uint32_t taken = 0;
-  for (int q = 0; q < nw; ++q) {
-    const int j = q * 32 + lane;
-    const uint64_t key = j < n ? (uint64_t)__double_as_longlong(pi[j]) : 0;
-    const bool gt = j < n && key > T;
-    const bool eq = j < n && key == T;
-    const uint32_t be = __ballot_sync(0xffffffffu, eq);
-    const uint32_t rank = taken + __popc(be & lanemask_lt());
-    const bool sel = gt || (eq && rank < need);
-    const uint32_t word = __ballot_sync(0xffffffffu, sel);
-    if (lane == 0) w[q] = word;
-    taken += __popc(be);
+  z = warp_sum_d(z);
+  const double P = p * z;
+  __syncwarp();
+
+  // Max extraction. Each lane keeps the best (key, slot) of its unselected elements.
+  uint64_t taken = 0;                       // bit e: element lane + 32 e is selected
+  uint32_t bkey = 0;
+  int bslot = -1;
+  auto rescan = [&]() {
+    bkey = 0;
+    bslot = -1;
+    for (int e = 0; e < nw; ++e) {
+      const int j = lane + 32 * e;
+      if (j < n && !((taken >> e) & 1ull)) {
+        const uint32_t k = wkey(E[j]);
+        if (bslot < 0 || k > bkey) { bkey = k; bslot = e; }
+      }
+    }
+  };
+  rescan();
+  double acc = 0.0;
+  bool done = false;
+  for (int it = 0; it < kExtract && !done; ++it) {
+    const uint32_t gk = __reduce_max_sync(0xffffffffu, bslot >= 0 ? bkey : 0u);
+    const uint32_t cand = (bslot >= 0 && bkey == gk) ? (uint32_t)(lane + 32 * bslot) : 0xffffffffu;
+    const uint32_t gj = __reduce_min_sync(0xffffffffu, cand);
+    if (gj == 0xffffffffu) break;
+    acc += E[gj];
+    if ((int)(gj & 31) == lane) {
+      taken |= 1ull << (gj >> 5);
+      rescan();
+    }
+    done = acc >= P;
+  }
+  if (done) {
+    for (int e = 0; e < nw; ++e) {
+      const uint32_t word = __ballot_sync(0xffffffffu, (taken >> e) & 1ull);
+      if (lane == 0) w[e] = word;
+    }
+    __syncwarp();
+    return;
+  }
+  // Bisection: largest T with mass{key >= T} >= P. M(0) = z >= P; keys are below 2^31.
+  uint32_t lo = 0, hi = 0x7f800001u;
+  while (hi - lo > 1) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    double s = 0.0;
+    for (int j = lane; j < n; j += 32)
+      if (wkey(E[j]) >= mid) s += E[j];
+    s = warp_sum_d(s);
+    if (s >= P) lo = mid;
+    else hi = mid;
+  }
+  const uint32_t T = lo;
+  double above = 0.0;
+  for (int j = lane; j < n; j += 32)
+    if (wkey(E[j]) > T) above += E[j];
+  above = warp_sum_d(above);
+  for (int e = 0; e < nw; ++e) {
+    const int j = lane + 32 * e;
+    const uint32_t k = j < n ? wkey(E[j]) : 0u;
+    uint32_t word = __ballot_sync(0xffffffffu, j < n && k > T);
+    uint32_t ties = __ballot_sync(0xffffffffu, j < n && k == T);
+    while (ties != 0u && above < P) {           // ties at the cut, lowest index first
+      const int b = __ffs(ties) - 1;
+      ties &= ties - 1;
+      above += E[32 * e + b];
+      word |= 1u << b;
+    }
+    if (lane == 0) w[e] = word;
   }
   __syncwarp();
 }
 
+// Transposed block means are stored with a row stride of nb rounded up to 32.
+__host__ __device__ __forceinline__ int means_ld(int nb) { return (nb + 31) & ~31; }
+
 size_t topp_smem_bytes(const Dims& m) {
   const size_t nbp = (size_t)m.nw * 32;
-  const size_t u = (size_t)KC * KT * 8 > (size_t)NWARP * 256 * 12 ? (size_t)KC * KT * 8 : (size_t)NWARP * 256 * 12;
-  return (size_t)KC * RT * 8 + (size_t)RT * nbp * 8 + u + (size_t)NWARP * 2 * m.nw * 4;
+  return 2 * ((size_t)KC * RT + (size_t)KC * KT) * 8 + (size_t)RT * nbp * 8 + (size_t)NWARP * 2 * m.nw * 4;
 }
 
+// One CTA per (head, 16 query blocks): the fp64 score tile Sc[i][j] = <qbar_i, kbar_j> * scale
+// over all key blocks (operand chunks double-buffered with cp.async; 4 x 4 fp64 register
+// tile per thread), then one warp per pair of rows: softmax weights, Top-p cut, forced blocks,
+// bitmask row, count, and the cost of the 128-row tile the pair forms.
 template <int D>
-__global__ void __launch_bounds__(256) topp_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
+__global__ void __launch_bounds__(256) topp_kernel(const double* __restrict__ qT, const double* __restrict__ kT,
                                                    Dims m, double p, double scale, ForceCfg fc,
                                                    uint32_t* __restrict__ bits, int32_t* __restrict__ counts,
                                                    int32_t* __restrict__ tile_cost) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int nbp = m.nw * 32;
-  double* sA = reinterpret_cast<double*>(smem_raw);      // [KC][RT]
-  double* sL = sA + KC * RT;                               // [RT][nbp] logits, then probabilities
-  double* sU = sL + (size_t)RT * nbp;                      // [KC][KT] key-mean chunk | histograms
-  uint32_t* sW = reinterpret_cast<uint32_t*>(sU + KC * KT); // [NWARP][2][nw] row bitmasks
+  const int ld = means_ld(m.nb);
+  double* sA = reinterpret_cast<double*>(smem_raw);          // [2][KC][RT]
+  double* sB = sA + 2 * KC * RT;                             // [2][KC][KT]
+  double* sL = sB + 2 * KC * KT;                             // [RT][nbp] logits, then weights
+  uint32_t* sW = reinterpret_cast<uint32_t*>(sL + (size_t)RT * nbp);   // [NWARP][2][nw]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t bh = blockIdx.y;
   const int row0 = blockIdx.x * RT;
-  const double* qb = qbar + bh * m.nb * D;
-  const double* kb = kbar + bh * m.nb * D;
+  const double* qh = qT + bh * (int64_t)D * ld;
+  const double* kh = kT + bh * (int64_t)D * ld;
   const int lm = lane >> 3, ln = lane & 7;   // 4 x 8 lanes: 4 rows x 4 keys per lane
+  constexpr int CPP = D / KC;                // chunks per pass
+  const int npass = (m.nb + KT - 1) / KT;
+  const int nch = npass * CPP;
 
-  // Scores Sc[i][j] = <qbar_i, kbar_j> * scale, fp64 FMA in ascending head-dim order.
-  for (int kp = 0; kp < m.nb; kp += KT) {
-    double acc[4][4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[r][c] = 0.0;
-    for (int k0 = 0; k0 < D; k0 += KC) {
-      __syncthreads();
-      {
-        const int r = tid / KC, kk = tid % KC;
-        const int i = row0 + r;
-        sA[kk * RT + r] = (i < m.nb) ? qb[(int64_t)i * D + k0 + kk] : 0.0;
-      }
-      {
-        const int j = kp + tid;
-        if (j < m.nb) {
-          const double2* src = reinterpret_cast<const double2*>(kb + (int64_t)j * D + k0);
-#pragma unroll
-          for (int q = 0; q < KC / 2; ++q) {
-            const double2 v = src[q];
-            sU[(2 * q) * KT + tid] = v.x;
-            sU[(2 * q + 1) * KT + tid] = v.y;
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < KC; ++q) sU[q * KT + tid] = 0.0;
-        }
-      }
-      __syncthreads();
-#pragma unroll
-      for (int kk = 0; kk < KC; ++kk) {
-        const double2 a01 = *reinterpret_cast<const double2*>(sA + kk * RT + lm * 4);
-        const double2 a23 = *reinterpret_cast<const double2*>(sA + kk * RT + lm * 4 + 2);
-        const double a[4] = {a01.x, a01.y, a23.x, a23.y};
-        double bq[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) bq[c] = sU[kk * KT + warp * 32 + ln + 8 * c];
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) acc[r][c] = fma(a[r], bq[c], acc[r][c]);
-      }
+  auto issue = [&](int ch) {
+    const int st = ch & 1;
+    const int kp = (ch / CPP) * KT, k0 = (ch % CPP) * KC;
+    double* a = sA + st * KC * RT;
+    double* b = sB + st * KC * KT;
+    for (int x = tid; x < KC * KT / 2; x += 256) {
+      const int kk = x / (KT / 2), j = kp + (x % (KT / 2)) * 2;
+      const int valid = imax(0, imin(2, m.nb - j));
+      cp_async16(b + kk * KT + (j - kp), kh + (int64_t)(k0 + kk) * ld + (valid ? j : 0), valid * 8);
     }
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int j = kp + warp * 32 + ln + 8 * c;
-        if (j < m.nb) sL[(lm * 4 + r) * nbp + j] = acc[r][c] * scale;
-      }
-  }
-  __syncthreads();
+    if (tid < KC * RT / 2) {
+      const int kk = tid / (RT / 2), i = row0 + (tid % (RT / 2)) * 2;
+      const int valid = imax(0, imin(2, m.nb - i));
+      cp_async16(a + kk * RT + (i - row0), qh + (int64_t)(k0 + kk) * ld + (valid ? i : 0), valid * 8);
+    }
+    cp_async_commit();
+  };
 
-  uint64_t* hm = reinterpret_cast<uint64_t*>(sU) + warp * 256;
-  uint32_t* hc = reinterpret_cast<uint32_t*>(reinterpret_cast<uint64_t*>(sU) + NWARP * 256) + warp * 256;
+  double acc[4][4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = 0.0;
+  issue(0);
+  for (int ch = 0; ch < nch; ++ch) {
+    if (ch + 1 < nch) issue(ch + 1);
+    else cp_async_commit();
+    cp_async_wait1();
+    __syncthreads();
+    const double* a = sA + (ch & 1) * KC * RT;
+    const double* b = sB + (ch & 1) * KC * KT;
+#pragma unroll
+    for (int kk = 0; kk < KC; ++kk) {
+      const double2 a01 = *reinterpret_cast<const double2*>(a + kk * RT + lm * 4);
+      const double2 a23 = *reinterpret_cast<const double2*>(a + kk * RT + lm * 4 + 2);
+      const double av[4] = {a01.x, a01.y, a23.x, a23.y};
+      double bq[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) bq[c] = b[kk * KT + warp * 32 + ln + 8 * c];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[r][c] = fma(av[r], bq[c], acc[r][c]);
+    }
+    if (ch % CPP == CPP - 1) {
+      const int kp = (ch / CPP) * KT;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int j = kp + warp * 32 + ln + 8 * c;
+          if (j < m.nb) sL[(lm * 4 + r) * nbp + j] = acc[r][c] * scale;
+          acc[r][c] = 0.0;
+        }
+    }
+    __syncthreads();
+  }
+
   uint32_t* w0 = sW + warp * 2 * m.nw;
 #pragma unroll 1
   for (int rr = 0; rr < 2; ++rr) {
@@ -404,9 +438,7 @@ __global__ void __launch_bounds__(256) topp_kernel(const double* __restrict__ qb
       __syncwarp();
       continue;
     }
-    double* L = sL + (size_t)r * nbp;
-    softmax_row(L, m.nb, lane);
-    topp_select(L, m.nb, p, hm, hc, w, lane);
+    topp_select(sL + (size_t)r * nbp, m.nb, p, w, lane);
     const int64_t grow = bh * m.nb + i;
     finalize_row(w, i, m, fc, lane, bits + grow * m.nw, counts + grow);
   }
@@ -694,32 +726,37 @@ __global__ void __launch_bounds__(256) csr_kernel(const uint32_t* __restrict__ b
 
 // ------------------------------------------------------------------ launchers
 
-template <typename T>
-static cudaError_t launch_pool_t(const void* Q, const void* K, int ntensors, const Dims& m, int frame_len,
-                                 double* qlo, double* klo, double* qhi, double* khi, int nsm,
-                                 cudaStream_t st) {
+template <typename T, int D>
+static cudaError_t launch_pool_td(const void* Q, const void* K, int ntensors, const Dims& m, int out, int frame_len,
+                                  double* qo, double* ko, double* qhi, double* khi, int nsm, cudaStream_t st) {
   const int64_t units = m.BH * m.nb * ntensors;
-  const int grid = (int)imin<int64_t>(units, (int64_t)nsm * 8);
+  const int grid = (int)imin<int64_t>((units + 3) / 4, (int64_t)nsm * 16);
   const T* q = static_cast<const T*>(Q);
   const T* k = static_cast<const T*>(K);
-  if (m.d == 128) {
-    if (frame_len > 0) pool_kernel<T, 128, true><<<grid, 256, 0, st>>>(q, k, ntensors, m, frame_len, qlo, klo, qhi, khi);
-    else pool_kernel<T, 128, false><<<grid, 256, 0, st>>>(q, k, ntensors, m, 0, qlo, klo, qhi, khi);
-  } else {
-    if (frame_len > 0) pool_kernel<T, 64, true><<<grid, 256, 0, st>>>(q, k, ntensors, m, frame_len, qlo, klo, qhi, khi);
-    else pool_kernel<T, 64, false><<<grid, 256, 0, st>>>(q, k, ntensors, m, 0, qlo, klo, qhi, khi);
-  }
+  const int ld = means_ld(m.nb);
+  if (out == kMeansT)
+    pool_kernel<T, D, kMeansT><<<grid, 128, 0, st>>>(q, k, ntensors, m, 0, ld, qo, ko, nullptr, nullptr);
+  else if (out == kFrameSums)
+    pool_kernel<T, D, kFrameSums><<<grid, 128, 0, st>>>(q, k, ntensors, m, frame_len, ld, qo, ko, qhi, khi);
+  else
+    pool_kernel<T, D, kMeans><<<grid, 128, 0, st>>>(q, k, ntensors, m, 0, ld, qo, ko, nullptr, nullptr);
   return cudaGetLastError();
 }
 
-cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int frame_len,
-                        double* qlo, double* klo, double* qhi, double* khi, int nsm, cudaStream_t st) {
-  if (dtype == FVATTN_BF16)
-    return launch_pool_t<__nv_bfloat16>(Q, K, ntensors, m, frame_len, qlo, klo, qhi, khi, nsm, st);
-  return launch_pool_t<float>(Q, K, ntensors, m, frame_len, qlo, klo, qhi, khi, nsm, st);
+// out: 0 = means [row][d], 1 = transposed means [bh][d][ld], 2 = frame segment sums.
+cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int out, int frame_len,
+                        double* qo, double* ko, double* qhi, double* khi, int nsm, cudaStream_t st) {
+  if (dtype == FVATTN_BF16) {
+    if (m.d == 128) return launch_pool_td<__nv_bfloat16, 128>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, nsm, st);
+    return launch_pool_td<__nv_bfloat16, 64>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, nsm, st);
+  }
+  if (m.d == 128) return launch_pool_td<float, 128>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, nsm, st);
+  return launch_pool_td<float, 64>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, nsm, st);
 }
 
-cudaError_t launch_topp(const double* qbar, const double* kbar, const Dims& m, double p, double scale,
+size_t means_t_elems(const Dims& m) { return (size_t)m.BH * m.d * means_ld(m.nb); }
+
+cudaError_t launch_topp(const double* qT, const double* kT, const Dims& m, double p, double scale,
                         const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
                         cudaStream_t st) {
   const size_t smem = topp_smem_bytes(m);
@@ -728,11 +765,11 @@ cudaError_t launch_topp(const double* qbar, const double* kbar, const Dims& m, d
   if (m.d == 128) {
     e = cudaFuncSetAttribute(topp_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    topp_kernel<128><<<grid, 256, smem, st>>>(qbar, kbar, m, p, scale, fc, bits, counts, tile_cost);
+    topp_kernel<128><<<grid, 256, smem, st>>>(qT, kT, m, p, scale, fc, bits, counts, tile_cost);
   } else {
     e = cudaFuncSetAttribute(topp_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    topp_kernel<64><<<grid, 256, smem, st>>>(qbar, kbar, m, p, scale, fc, bits, counts, tile_cost);
+    topp_kernel<64><<<grid, 256, smem, st>>>(qT, kT, m, p, scale, fc, bits, counts, tile_cost);
   }
   return cudaGetLastError();
 }

@@ -11,12 +11,14 @@ struct ForceCfg {
 };
 
 size_t topp_smem_bytes(const Dims& m);
+size_t means_t_elems(const Dims& m);     // doubles of one transposed block-mean array
 size_t frame_smem_bytes(const Dims& m);
 size_t schedule_smem_bytes(const Dims& m, int* groups);
 
-cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int frame_len,
-                        double* qlo, double* klo, double* qhi, double* khi, int nsm, cudaStream_t st);
-cudaError_t launch_topp(const double* qbar, const double* kbar, const Dims& m, double p, double scale,
+// out: 0 = means [row][d], 1 = means transposed per head [bh][d][ld], 2 = frame segment sums.
+cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int out, int frame_len,
+                        double* qo, double* ko, double* qhi, double* khi, int nsm, cudaStream_t st);
+cudaError_t launch_topp(const double* qT, const double* kT, const Dims& m, double p, double scale,
                         const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
                         cudaStream_t st);
 cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,
