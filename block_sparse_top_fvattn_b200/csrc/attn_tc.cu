@@ -15,7 +15,8 @@
 //                        raised (with a rescale of O in TMEM) when it grows by more than
 //                        2^8, and writes P as bf16 into shared memory in the MMA's layout
 //   O += P V_j           tcgen05.mma M=128 N=d K=64, V MN-major, O accumulated in TMEM
-// Warp roles: warp 0 issues TMA loads (Q once per tile, K_j and V_j into a 4-stage ring),
+// Warp roles: warp 0 issues TMA loads (lane 0: Q once per tile and K_j, lane 1: V_j, each into
+// its own 2-stage ring, so a K stage is reloaded as soon as its S MMA is done),
 // warp 1 allocates TMEM and issues the MMAs, warps 2-5 do softmax and the epilogue.
 // Every mbarrier wait is bounded; a wait that runs out sets an abort flag, every role
 // unwinds, TMEM is freed and FVATTN_ERR_TIMEOUT is written to the device status word.
@@ -39,11 +40,11 @@ struct TcLayout {
   static constexpr int kQChunk = kTileRows * 128;     // [128 rows x 64 dims] bf16 = 16 KB
   static constexpr int kQBytes = (D / 64) * kQChunk;
   static constexpr int kKVChunk = kBlock * 128;       // [64 rows x 64 dims] bf16 = 8 KB
-  static constexpr int kKBytes = (D / 64) * kKVChunk;
-  static constexpr int kStage = 2 * kKBytes;          // K_j and V_j
+  static constexpr int kKBytes = (D / 64) * kKVChunk; // one K_j (or V_j) block
   static constexpr int kOffQ = 0;
-  static constexpr int kOffKV = kQBytes;
-  static constexpr int kOffBar = kOffKV + NS * kStage;
+  static constexpr int kOffK = kQBytes;               // NS stages of K
+  static constexpr int kOffV = kOffK + NS * kKBytes;  // NS stages of V
+  static constexpr int kOffBar = kOffV + NS * kKBytes;
   static constexpr int kBytes = kOffBar + 512;
   // TMEM: S double buffer at columns 0 and 64 (P, bf16, overwrites the first 32 columns of its
   // S buffer), O at column 128.
@@ -51,13 +52,17 @@ struct TcLayout {
   static constexpr uint32_t kColO = 128;
 };
 
+constexpr int NI = 8;        // step records in flight
+
 struct TcBars {
   uint64_t q_full, q_empty;
-  uint64_t kv_full[NS], kv_empty[NS];
+  uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t o_full, o_empty;
   uint64_t sched_full[2], sched_empty[2];
+  uint64_t info_full[NI];
   int sched_tile[2];
+  int step_info[NI];          // key block j | membership mask << 28 | last step of tile << 30
   uint32_t tmem_base;
   int abort;
 };
@@ -79,6 +84,7 @@ struct PairMerge {
       b = be = 0;
     }
   }
+  __device__ __forceinline__ bool more() const { return a < ae || b < be; }
   __device__ __forceinline__ bool next(int& j, int& mask) {
     if (a >= ae && b >= be) return false;
     const int ja = a < ae ? ci[a] : 0x7fffffff;
@@ -146,7 +152,8 @@ __global__ void __launch_bounds__(192, 2)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   TcBars* bars = reinterpret_cast<TcBars*>(smem + L::kOffBar);
   unsigned char* sQ = smem + L::kOffQ;
-  unsigned char* sKV = smem + L::kOffKV;
+  unsigned char* sK = smem + L::kOffK;
+  unsigned char* sV = smem + L::kOffV;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ntiles = m.BH * m.nt;
   volatile int* abort = &bars->abort;
@@ -155,16 +162,19 @@ __global__ void __launch_bounds__(192, 2)
     tc::mbar_init(&bars->q_full, 1);
     tc::mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < NS; ++s) {
-      tc::mbar_init(&bars->kv_full[s], 1);
-      tc::mbar_init(&bars->kv_empty[s], 1);
+      tc::mbar_init(&bars->k_full[s], 1);
+      tc::mbar_init(&bars->k_empty[s], 1);
+      tc::mbar_init(&bars->v_full[s], 1);
+      tc::mbar_init(&bars->v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->s_full[s], 1);
       tc::mbar_init(&bars->p_full[s], 4);
       tc::mbar_init(&bars->pv_done[s], 1);
       tc::mbar_init(&bars->sched_full[s], 1);
-      tc::mbar_init(&bars->sched_empty[s], 5);    // the MMA thread and the four softmax warps
+      tc::mbar_init(&bars->sched_empty[s], 6);    // V loader, MMA thread, four softmax warps
     }
+    for (int s = 0; s < NI; ++s) tc::mbar_init(&bars->info_full[s], 1);
     tc::mbar_init(&bars->o_full, 1);
     tc::mbar_init(&bars->o_empty, 4);
     bars->abort = 0;
@@ -185,10 +195,14 @@ __global__ void __launch_bounds__(192, 2)
   const uint32_t tbase = bars->tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ scheduler + TMA producer
-    // Takes the next tile of the longest-first order from the global ticket, publishes it to
-    // the other roles, and streams its Q tile and K_j / V_j blocks.
     if (lane == 0) {
+      // ---------------------------------------------------------- scheduler, Q and K loader
+      // Takes the next tile of the longest-first order from the global ticket, publishes it,
+      // loads its Q tile, and for every key block of the tile's list publishes a step record
+      // and loads K_j. A K stage is refilled as soon as the S MMA that read it is done.
+      // The record ring is deep enough that a record is never overwritten before every
+      // reader has taken it: record g+NI is written only after S_{g+NI-3} was issued, which
+      // follows P_{g+NI-5} of the softmax warps.
       uint32_t g = 0;
       for (uint32_t n = 0;; ++n) {
         const int s = n & 1;
@@ -214,15 +228,38 @@ __global__ void __launch_bounds__(192, 2)
         int j, mask;
         bool ok = true;
         while (mg.next(j, mask)) {
+          bars->step_info[g % NI] = j | (mask << 28) | (mg.more() ? 0 : (1 << 30));
+          tc::mbar_arrive(&bars->info_full[g % NI]);
           const int st = g % NS;
-          if (!tc::mbar_wait(&bars->kv_empty[st], ((g / NS) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 3); ok = false; break; }
-          unsigned char* sK = sKV + st * L::kStage;
-          unsigned char* sV = sK + L::kKBytes;
-          tc::mbar_expect_tx(&bars->kv_full[st], L::kStage);
-          for (int c = 0; c < D / 64; ++c) {
-            tc::tma_load_3d(sK + c * L::kKVChunk, &tmK, &bars->kv_full[st], c * 64, j * kBlock, (int)bh);
-            tc::tma_load_3d(sV + c * L::kKVChunk, &tmV, &bars->kv_full[st], c * 64, j * kBlock, (int)bh);
-          }
+          if (!tc::mbar_wait(&bars->k_empty[st], ((g / NS) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 3); ok = false; break; }
+          tc::mbar_expect_tx(&bars->k_full[st], L::kKBytes);
+          for (int c = 0; c < D / 64; ++c)
+            tc::tma_load_3d(sK + st * L::kKBytes + c * L::kKVChunk, &tmK, &bars->k_full[st], c * 64, j * kBlock, (int)bh);
+          ++g;
+        }
+        if (!ok) break;
+      }
+    } else if (lane == 1) {
+      // ---------------------------------------------------------- V loader
+      // Loads V_j for the same steps; a V stage is refilled once the P.V that read it is done.
+      uint32_t g = 0;
+      for (uint32_t n = 0;; ++n) {
+        const int s = n & 1;
+        if (!tc::mbar_wait(&bars->sched_full[s], (n >> 1) & 1, abort, kWaitLimit)) { fail(bars, 15); break; }
+        const int tile = bars->sched_tile[s];
+        tc::mbar_arrive(&bars->sched_empty[s]);
+        if (tile < 0) break;
+        const int64_t bh = tile / m.nt;
+        const int t = (int)(tile - bh * m.nt);
+        PairMerge mg(row_ptr, col_idx, bh, t, m.nb);
+        int j, mask;
+        bool ok = true;
+        while (mg.next(j, mask)) {
+          const int st = g % NS;
+          if (!tc::mbar_wait(&bars->v_empty[st], ((g / NS) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 16); ok = false; break; }
+          tc::mbar_expect_tx(&bars->v_full[st], L::kKBytes);
+          for (int c = 0; c < D / 64; ++c)
+            tc::tma_load_3d(sV + st * L::kKBytes + c * L::kKVChunk, &tmV, &bars->v_full[st], c * 64, j * kBlock, (int)bh);
           ++g;
         }
         if (!ok) break;
@@ -235,23 +272,24 @@ __global__ void __launch_bounds__(192, 2)
     if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16_f32(kTileRows, kBlock, 0, 0);
       constexpr uint32_t idO = tc::idesc_bf16_f32(kTileRows, D, 0, 1);
-      const uint32_t qaddr = tc::smem_u32(sQ), kvaddr = tc::smem_u32(sKV);
+      const uint32_t qaddr = tc::smem_u32(sQ), kaddr0 = tc::smem_u32(sK), vaddr0 = tc::smem_u32(sV);
       uint32_t g = 0, n = 0;
       bool ok = true;
       // O += P_gs V_gs for step gs; `first` = first step of the tile (overwrites O).
       auto pv = [&](uint32_t gs, bool first) -> bool {
-        const int pb = gs & 1;
+        const int pb = gs & 1, st = gs % NS;
         if (!tc::mbar_wait(&bars->p_full[pb], (gs >> 1) & 1, abort, kWaitLimit)) return false;
         if (first && !tc::mbar_wait(&bars->o_empty, (n & 1) ^ 1, abort, kWaitLimit)) return false;
+        if (!tc::mbar_wait(&bars->v_full[st], (gs / NS) & 1, abort, kWaitLimit)) return false;
         tc::fence_after_sync();
-        const uint32_t vaddr = kvaddr + (gs % NS) * L::kStage + L::kKBytes;
+        const uint32_t vaddr = vaddr0 + st * L::kKBytes;
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk) {
           const uint64_t b = tc::smem_desc_sw128(vaddr + kk * 16 * 128, L::kKVChunk, 1024);
           tc::mma_f16_tmem_a(tbase + L::kColO, tbase + pb * kBlock + kk * 8, b, idO, (first && kk == 0) ? 0u : 1u);
         }
         tc::mma_commit(&bars->pv_done[pb]);
-        tc::mma_commit(&bars->kv_empty[gs % NS]);
+        tc::mma_commit(&bars->v_empty[st]);
         return true;
       };
       for (;; ++n) {
@@ -260,17 +298,20 @@ __global__ void __launch_bounds__(192, 2)
         const int tile = bars->sched_tile[s];
         tc::mbar_arrive(&bars->sched_empty[s]);
         if (tile < 0) break;
-        const int64_t bh = tile / m.nt;
-        const int t = (int)(tile - bh * m.nt);
         if (!tc::mbar_wait(&bars->q_full, n & 1, abort, kWaitLimit)) { fail(bars, 5); ok = false; break; }
-        PairMerge mg(row_ptr, col_idx, bh, t, m.nb);
-        int j, mask, i = 0;
-        while (mg.next(j, mask)) {
+        int i = 0;
+        for (bool last = false; !last;) {
           const uint32_t gi = g + i;
           const int st = gi % NS, sb = gi & 1;
-          if (!tc::mbar_wait(&bars->kv_full[st], (gi / NS) & 1, abort, kWaitLimit)) { fail(bars, 6); ok = false; break; }
+          if (!tc::mbar_wait(&bars->info_full[gi % NI], (gi / NI) & 1, abort, kWaitLimit) ||
+              !tc::mbar_wait(&bars->k_full[st], (gi / NS) & 1, abort, kWaitLimit)) {
+            fail(bars, 6);
+            ok = false;
+            break;
+          }
+          last = (bars->step_info[gi % NI] >> 30) & 1;
           tc::fence_after_sync();
-          const uint32_t kaddr = kvaddr + st * L::kStage;
+          const uint32_t kaddr = kaddr0 + st * L::kKBytes;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const int c = kk >> 2, off = (kk & 3) * 32;
@@ -279,6 +320,7 @@ __global__ void __launch_bounds__(192, 2)
             tc::mma_f16(tbase + sb * kBlock, a, b, idS, kk > 0 ? 1u : 0u);
           }
           tc::mma_commit(&bars->s_full[sb]);
+          tc::mma_commit(&bars->k_empty[st]);       // K_j may be replaced once S_i is done
           if (i > 0 && !pv(gi - 1, i == 1)) { fail(bars, 7); ok = false; break; }
           ++i;
         }
@@ -310,13 +352,17 @@ __global__ void __launch_bounds__(192, 2)
       const int t = (int)(tile - bh * m.nt);
       float mrow = -INFINITY;
       uint64_t lsum = f2(0.f, 0.f);
-      PairMerge mg(row_ptr, col_idx, bh, t, m.nb);
-      int j, mask, i = 0;
+      int i = 0;
       bool ok = true;
-      while (mg.next(j, mask)) {
+      for (bool last = false; !last;) {
         const uint32_t gi = g + i;
         const int sb = gi & 1;
         const uint32_t sp = tbase + lane_off + sb * kBlock;     // S_i, then P_i, of this row
+        // The step record published by the loader names the key block and its row halves.
+        if (!warp_wait(&bars->info_full[gi % NI], (gi / NI) & 1, abort)) { fail(bars, 14); ok = false; break; }
+        const int info = bars->step_info[gi % NI];
+        const int j = info & 0x0fffffff, mask = (info >> 28) & 3;
+        last = (info >> 30) & 1;
         if (!warp_wait(&bars->s_full[sb], (gi >> 1) & 1, abort)) { fail(bars, 10); ok = false; break; }
         tc::fence_after_sync();
         uint32_t packed[32];
