@@ -134,6 +134,12 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -382,13 +388,15 @@ __global__ void __launch_bounds__(192, 2)
             for (int c = 0; c < 64; ++c)
               if (c >= nk) sraw[c] = __float_as_uint(-INFINITY);
           }
-          float mx8[8];
+          float m21[21];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(sraw[c]);
+          for (int c = 0; c < 21; ++c)
+            m21[c] = max3(__uint_as_float(sraw[3 * c]), __uint_as_float(sraw[3 * c + 1]), __uint_as_float(sraw[3 * c + 2]));
+          float m7[7];
 #pragma unroll
-          for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sraw[c]));
-          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
+          for (int c = 0; c < 7; ++c) m7[c] = max3(m21[3 * c], m21[3 * c + 1], m21[3 * c + 2]);
+          const float mx = max3(max3(m7[0], m7[1], m7[2]), max3(m7[3], m7[4], m7[5]),
+                                max3(m7[6], __uint_as_float(sraw[63]), m7[6])) * scale_log2;
           // Raise the running max only when it grows by more than 2^8 (or on the row's first
           // kept block); rows whose O already holds earlier blocks then scale O in TMEM.
           const bool raise = mrow == -INFINITY || mx > mrow + kRescaleLog2;
@@ -419,9 +427,12 @@ __global__ void __launch_bounds__(192, 2)
           uint64_t acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
+            const uint64_t x2 = ffma2(f2(__uint_as_float(sraw[2 * c]), __uint_as_float(sraw[2 * c + 1])), scale2, negm);
+            float p0, p1;
             float x0, x1;
-            f2_split(ffma2(f2(__uint_as_float(sraw[2 * c]), __uint_as_float(sraw[2 * c + 1])), scale2, negm), x0, x1);
-            const float p0 = ex2(x0), p1 = ex2(x1);
+            f2_split(x2, x0, x1);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
             acc[c & 3] = fadd2(acc[c & 3], f2(p0, p1));
             packed[c] = pack_bf16(p0, p1);
           }
