@@ -46,9 +46,11 @@ def env_rank():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
 
 
-def workload_desc(w) -> str:
+def workload_desc(w, mode: str = "topp", topk_frames: int = 4) -> str:
+    sel = (f"p={w.p},diag forced" if mode == "topp" else
+           f"frame top-k={topk_frames} + frames +-1 + frame 0 + diag")
     return (f"{w.name}: B={w.B},H={w.H},S={w.S} ({w.frames} frames x {w.frame_len} tokens),d={w.d},{w.dtype},"
-            f"block=64,p={w.p},diag forced")
+            f"block=64,{sel}")
 
 
 # ------------------------------------------------------------------ clocks
@@ -140,9 +142,23 @@ def traffic_from_profile(kernel_src: str):
     return d.get("dram_bytes_per_launch")
 
 
+def reduce_over_ranks(ms: float, flops: float, device):
+    """Max of the device-timed milliseconds and sum of the work over all ranks (the job's
+    time is its slowest rank's; its work is every rank's). Identity on one process."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(ms), float(flops)
+    t = torch.tensor([float(ms)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    f = torch.tensor([float(flops)], device=device, dtype=torch.float64)
+    dist.all_reduce(f, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(f.item())
+
+
 # ------------------------------------------------------------------ CPU oracle baseline
 
-def cpu_oracle_run(w, q_cpu, k_cpu, v_cpu, n_items: int, seed: int = 0):
+def cpu_oracle_run(w, q_cpu, k_cpu, v_cpu, n_items: int, seed: int = 0, heads_sample=None):
     """Time the oracle (as it stands) on a bounded sample of the layer: the full router on
     `heads` heads and exact attention for `n_items` query blocks of those heads. Returns
     (estimated seconds for the whole layer, sample description, threads used, sample FLOPs)."""
@@ -154,7 +170,7 @@ def cpu_oracle_run(w, q_cpu, k_cpu, v_cpu, n_items: int, seed: int = 0):
     except Exception:
         threads = os.cpu_count() or 1
     BH = w.B * w.H
-    heads = min(BH, 4)
+    heads = BH if heads_sample is None else min(BH, heads_sample)
     Q = q_cpu.reshape(BH, w.S, w.d)[:heads]
     K = k_cpu.reshape(BH, w.S, w.d)[:heads]
     V = v_cpu.reshape(BH, w.S, w.d)[:heads]
@@ -190,7 +206,7 @@ def run_reference(args, w):
     flops = None
     desc = threads = None
     for s in range(args.warmup + args.steps):
-        t_layer, desc, threads, flops = cpu_oracle_run(w.replace(H=4), x["q"], x["k"], x["v"], n_items=8, seed=s)
+        t_layer, desc, threads, flops = cpu_oracle_run(w.replace(H=4), x["q"], x["k"], x["v"], n_items=24, seed=s)
         t_layer *= w.H / 4
         if s >= args.warmup:
             times.append(t_layer)
@@ -230,7 +246,11 @@ def run_ours(args, w):
     q, k, v = x["q"], x["k"], x["v"]
     B, H, S, d = q.shape
     BH = B * H
-    cfg = fv.RouteConfig(p=w.p, force_diag=True)
+    if args.mode == "frame_topk":
+        cfg = fv.RouteConfig(mode="frame_topk", topk_frames=args.topk_frames, frame_len=w.frame_len, frame_window=1,
+                             force_first_frame=True, force_diag=True)
+    else:
+        cfg = fv.RouteConfig(p=w.p, force_diag=True)
     csr = fv.alloc_csr(B, H, S, dev)
     ws = torch.empty(fv.workspace_bytes(q, cfg), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
@@ -273,15 +293,7 @@ def run_ours(args, w):
     total_ms = t_start.elapsed_time(t_end)
     route_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.steps)]
     attn_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(args.steps)]
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-        ft = torch.tensor([float(flops)], device=dev, dtype=torch.float64)
-        dist.all_reduce(ft, op=dist.ReduceOp.SUM)
-        flops_all = float(ft.item())
-    else:
-        flops_all = float(flops)
+    total_ms, flops_all = reduce_over_ranks(total_ms, flops, dev)
     ms_step = total_ms / args.steps
     value = flops_all * args.steps / (total_ms * 1e-3) / 1e12
     attn_avg = statistics.mean(attn_ms)
@@ -327,7 +339,7 @@ def run_ours(args, w):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t_layer, desc, threads, _ = cpu_oracle_run(w, q.cpu(), k.cpu(), v.cpu(), n_items=12)
+        t_layer, desc, threads, _ = cpu_oracle_run(w, q.cpu(), k.cpu(), v.cpu(), n_items=160)
         cpu = {"value": flops / t_layer / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
 
     if world > 1:
@@ -340,7 +352,8 @@ def run_ours(args, w):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": workload_desc(w), "l2": "inputs larger than L2 (Q,K,V = 1.0 GB per layer)",
+        "config": {"workload": workload_desc(w, args.mode, args.topk_frames),
+                   "l2": f"inputs larger than L2 (Q,K,V = {3 * q.numel() * q.element_size() / 1e9:.2f} GB per layer)",
                    "parallelism": f"independent layer per GPU x{world}"},
         "route_ms": route_avg, "attn_ms": attn_avg, "attn_tflops": attn_tflops,
         "pct_bf16_peak": 100.0 * value / pk["bf16_tflops"],
@@ -373,11 +386,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling case)")
+    ap.add_argument("--p", type=float, default=0.0, help="override the Top-p threshold")
+    ap.add_argument("--mode", default="topp", choices=["topp", "frame_topk"])
+    ap.add_argument("--topk-frames", type=int, default=4)
     args = ap.parse_args()
     from workloads import get_workload
     w = get_workload(args.workload)
     if args.heads:
         w = w.replace(H=args.heads)
+    if args.p:
+        w = w.replace(p=args.p)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -37,7 +37,6 @@ int validate_cfg(const fvattn_shape* s, const fvattn_route_cfg* c) {
   if (c->force_diag != 0 && c->force_diag != 1) return FVATTN_ERR_INVALID;
   if (c->force_first_frame != 0 && c->force_first_frame != 1) return FVATTN_ERR_INVALID;
   if ((c->frame_window >= 0 || c->force_first_frame) && c->frame_len == 0) return FVATTN_ERR_INVALID;
-  if (c->mode == FVATTN_MODE_TOPP && (s->S + kBlock - 1) / kBlock > 1536) return FVATTN_ERR_UNSUPPORTED;
   if (c->mode == FVATTN_MODE_FRAME_TOPK) {
     if (c->frame_len < kBlock || c->topk_frames < 1) return FVATTN_ERR_INVALID;
     const int64_t F = (s->S + c->frame_len - 1) / c->frame_len;
@@ -47,7 +46,7 @@ int validate_cfg(const fvattn_shape* s, const fvattn_route_cfg* c) {
 }
 
 struct WsLayout {
-  size_t qlo, klo, qhi, khi, qf, kf, bits, counts, total;
+  size_t qlo, klo, qhi, khi, qf, kf, logits, bits, counts, total;
 };
 
 size_t take(size_t& off, size_t bytes) {
@@ -69,6 +68,7 @@ WsLayout ws_layout(const Dims& m, int mode) {
     L.qf = take(off, fm);
     L.kf = take(off, fm);
   }
+  if (mode == FVATTN_MODE_TOPP) L.logits = take(off, logits_elems(m) * sizeof(double));
   L.bits = take(off, (size_t)m.BH * m.nb * m.nw * sizeof(uint32_t));
   L.counts = take(off, (size_t)m.BH * m.nb * sizeof(int32_t));
   L.total = off;
@@ -156,7 +156,8 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const 
   if (cfg->mode == FVATTN_MODE_TOPP) {
     e = launch_pool(Q, K, 2, shape->dtype, m, 1, 0, qlo, klo, nullptr, nullptr, nsm, s);
     if (e == cudaSuccess)
-      e = launch_topp(qlo, klo, m, cfg->p >= 1.f ? 1.0 : (double)cfg->p, scale, fc, bits, counts, out->tile_cost, s);
+      e = launch_topp(qlo, klo, reinterpret_cast<double*>(ws + L.logits), m, cfg->p >= 1.f ? 1.0 : (double)cfg->p, scale, fc,
+                      bits, counts, out->tile_cost, s);
   } else {
     double* qhi = reinterpret_cast<double*>(ws + L.qhi);
     double* khi = reinterpret_cast<double*>(ws + L.khi);

@@ -210,9 +210,6 @@ __device__ __forceinline__ int finalize_row(uint32_t* w, int i, const Dims& m, c
 
 // ------------------------------------------------------------------ K2: Top-p
 
-constexpr int RT = 16;      // query blocks per CTA
-constexpr int KT = 256;     // key blocks per pass of the score tile
-constexpr int KC = 8;       // head-dim rows of one pipelined operand chunk
 constexpr int NWARP = 8;
 constexpr int kExtract = 16;   // max-extraction steps before the bisection fallback
 
@@ -338,52 +335,43 @@ __device__ void topp_select(double* E, int n, double p, uint32_t* w, int lane) {
 // Transposed block means are stored with a row stride of nb rounded up to 32.
 __host__ __device__ __forceinline__ int means_ld(int nb) { return (nb + 31) & ~31; }
 
-size_t topp_smem_bytes(const Dims& m) {
-  const size_t nbp = (size_t)m.nw * 32;
-  return 2 * ((size_t)KC * RT + (size_t)KC * KT) * 8 + (size_t)RT * nbp * 8 + (size_t)NWARP * 2 * m.nw * 4;
-}
+size_t logits_elems(const Dims& m) { return (size_t)m.BH * m.nb * means_ld(m.nb); }
 
-// One CTA per (head, 16 query blocks): the fp64 score tile Sc[i][j] = <qbar_i, kbar_j> * scale
-// over all key blocks (operand chunks double-buffered with cp.async; 4 x 4 fp64 register
-// tile per thread), then one warp per pair of rows: softmax weights, Top-p cut, forced blocks,
-// bitmask row, count, and the cost of the 128-row tile the pair forms.
+constexpr int ST = 64;      // score GEMM output tile: 64 query blocks x 64 key blocks
+constexpr int SKC = 16;     // head-dim depth of one pipelined operand chunk
+constexpr int SNS = 3;      // pipeline stages
+
+__device__ __forceinline__ void cp_async_wait2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
+
+// Sc[bh][i][j] = <qbar_i, kbar_j> * scale in fp64 for all i, j < nb, written row-major with row
+// stride ld. One 64 x 64 tile per CTA; warps in a 4 x 2 grid of 16 rows x 32 keys; each lane
+// 4 rows (lm * 4 ..) by 4 keys (2 ln, 2 ln + 1, 16 + 2 ln, 17 + 2 ln), so that every shared
+// load of an operand is a single wavefront. Operands stream from the transposed block means
+// [bh][d][ld] through a 3-stage cp.async ring of 16-deep head-dim chunks. FMAs accumulate in
+// ascending head-dim order.
 template <int D>
-__global__ void __launch_bounds__(256) topp_kernel(const double* __restrict__ qT, const double* __restrict__ kT,
-                                                   Dims m, double p, double scale, ForceCfg fc,
-                                                   uint32_t* __restrict__ bits, int32_t* __restrict__ counts,
-                                                   int32_t* __restrict__ tile_cost) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int nbp = m.nw * 32;
-  const int ld = means_ld(m.nb);
-  double* sA = reinterpret_cast<double*>(smem_raw);          // [2][KC][RT]
-  double* sB = sA + 2 * KC * RT;                             // [2][KC][KT]
-  double* sL = sB + 2 * KC * KT;                             // [RT][nbp] logits, then weights
-  uint32_t* sW = reinterpret_cast<uint32_t*>(sL + (size_t)RT * nbp);   // [NWARP][2][nw]
-
+__global__ void __launch_bounds__(256) score_kernel(const double* __restrict__ qT, const double* __restrict__ kT,
+                                                    Dims m, double scale, double* __restrict__ logits) {
+  __shared__ __align__(16) double sA[SNS][SKC][ST];
+  __shared__ __align__(16) double sB[SNS][SKC][ST];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t bh = blockIdx.y;
-  const int row0 = blockIdx.x * RT;
+  const int wr = warp >> 1, wc = warp & 1;
+  const int lm = lane >> 3, ln = lane & 7;
+  const int64_t bh = blockIdx.z;
+  const int i0 = blockIdx.y * ST, j0 = blockIdx.x * ST;
+  const int ld = means_ld(m.nb);
   const double* qh = qT + bh * (int64_t)D * ld;
   const double* kh = kT + bh * (int64_t)D * ld;
-  const int lm = lane >> 3, ln = lane & 7;   // 4 x 8 lanes: 4 rows x 4 keys per lane
-  constexpr int CPP = D / KC;                // chunks per pass
-  const int npass = (m.nb + KT - 1) / KT;
-  const int nch = npass * CPP;
+  constexpr int NCH = D / SKC;
 
   auto issue = [&](int ch) {
-    const int st = ch & 1;
-    const int kp = (ch / CPP) * KT, k0 = (ch % CPP) * KC;
-    double* a = sA + st * KC * RT;
-    double* b = sB + st * KC * KT;
-    for (int x = tid; x < KC * KT / 2; x += 256) {
-      const int kk = x / (KT / 2), j = kp + (x % (KT / 2)) * 2;
-      const int valid = imax(0, imin(2, m.nb - j));
-      cp_async16(b + kk * KT + (j - kp), kh + (int64_t)(k0 + kk) * ld + (valid ? j : 0), valid * 8);
-    }
-    if (tid < KC * RT / 2) {
-      const int kk = tid / (RT / 2), i = row0 + (tid % (RT / 2)) * 2;
-      const int valid = imax(0, imin(2, m.nb - i));
-      cp_async16(a + kk * RT + (i - row0), qh + (int64_t)(k0 + kk) * ld + (valid ? i : 0), valid * 8);
+    const int st = ch % SNS, k0 = ch * SKC;
+    for (int x = tid; x < SKC * ST / 2; x += 256) {
+      const int kk = x / (ST / 2), c = (x % (ST / 2)) * 2;
+      const int i = i0 + c, j = j0 + c;
+      const int vi = imax(0, imin(2, m.nb - i)), vj = imax(0, imin(2, m.nb - j));
+      cp_async16(&sA[st][kk][c], qh + (int64_t)(k0 + kk) * ld + (vi ? i : 0), vi * 8);
+      cp_async16(&sB[st][kk][c], kh + (int64_t)(k0 + kk) * ld + (vj ? j : 0), vj * 8);
     }
     cp_async_commit();
   };
@@ -394,60 +382,88 @@ __global__ void __launch_bounds__(256) topp_kernel(const double* __restrict__ qT
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[r][c] = 0.0;
   issue(0);
-  for (int ch = 0; ch < nch; ++ch) {
-    if (ch + 1 < nch) issue(ch + 1);
+  issue(1);
+  for (int ch = 0; ch < NCH; ++ch) {
+    if (ch + 2 < NCH) issue(ch + 2);
     else cp_async_commit();
-    cp_async_wait1();
+    cp_async_wait2();
     __syncthreads();
-    const double* a = sA + (ch & 1) * KC * RT;
-    const double* b = sB + (ch & 1) * KC * KT;
+    const int st = ch % SNS;
 #pragma unroll
-    for (int kk = 0; kk < KC; ++kk) {
-      const double2 a01 = *reinterpret_cast<const double2*>(a + kk * RT + lm * 4);
-      const double2 a23 = *reinterpret_cast<const double2*>(a + kk * RT + lm * 4 + 2);
+    for (int kk = 0; kk < SKC; ++kk) {
+      const double2 a01 = *reinterpret_cast<const double2*>(&sA[st][kk][wr * 16 + lm * 4]);
+      const double2 a23 = *reinterpret_cast<const double2*>(&sA[st][kk][wr * 16 + lm * 4 + 2]);
+      const double2 b01 = *reinterpret_cast<const double2*>(&sB[st][kk][wc * 32 + ln * 2]);
+      const double2 b23 = *reinterpret_cast<const double2*>(&sB[st][kk][wc * 32 + 16 + ln * 2]);
       const double av[4] = {a01.x, a01.y, a23.x, a23.y};
-      double bq[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) bq[c] = b[kk * KT + warp * 32 + ln + 8 * c];
+      const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
 #pragma unroll
       for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] = fma(av[r], bq[c], acc[r][c]);
-    }
-    if (ch % CPP == CPP - 1) {
-      const int kp = (ch / CPP) * KT;
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int j = kp + warp * 32 + ln + 8 * c;
-          if (j < m.nb) sL[(lm * 4 + r) * nbp + j] = acc[r][c] * scale;
-          acc[r][c] = 0.0;
-        }
+        for (int c = 0; c < 4; ++c) acc[r][c] = fma(av[r], bv[c], acc[r][c]);
     }
     __syncthreads();
   }
-
-  uint32_t* w0 = sW + warp * 2 * m.nw;
-#pragma unroll 1
-  for (int rr = 0; rr < 2; ++rr) {
-    const int r = 2 * warp + rr, i = row0 + r;
-    uint32_t* w = w0 + rr * m.nw;
-    if (i >= m.nb) {
-      for (int q = lane; q < m.nw; q += 32) w[q] = 0;
-      __syncwarp();
-      continue;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int i = i0 + wr * 16 + lm * 4 + r;
+    if (i >= m.nb) continue;
+    double* row = logits + (bh * m.nb + i) * (int64_t)ld;
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2) {
+      const int j = j0 + wc * 32 + c2 * 16 + ln * 2;
+      if (j + 1 < m.nb) {
+        *reinterpret_cast<double2*>(row + j) = make_double2(acc[r][2 * c2] * scale, acc[r][2 * c2 + 1] * scale);
+      } else if (j < m.nb) {
+        row[j] = acc[r][2 * c2] * scale;
+      }
     }
-    topp_select(sL + (size_t)r * nbp, m.nb, p, w, lane);
+  }
+}
+
+constexpr int SEL_WARPS = 8;
+
+size_t select_smem_bytes(const Dims& m) {
+  return (size_t)SEL_WARPS * m.nw * 32 * 8 + (size_t)SEL_WARPS * m.nw * 4;
+}
+
+// One warp per query block: its fp64 logit row to shared memory, the Top-p cut, forced blocks,
+// bitmask row and count; warps 2w and 2w+1 hold the two rows of a 128-row tile and write its
+// cost (distinct key blocks of the pair).
+__global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ logits, Dims m, double p,
+                                                     ForceCfg fc, uint32_t* __restrict__ bits,
+                                                     int32_t* __restrict__ counts, int32_t* __restrict__ tile_cost) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int nbp = m.nw * 32;
+  double* sE = reinterpret_cast<double*>(smem_raw);                               // [warp][nbp]
+  uint32_t* sW = reinterpret_cast<uint32_t*>(sE + (size_t)SEL_WARPS * nbp);      // [warp][nw]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t bh = blockIdx.y;
+  const int i = blockIdx.x * SEL_WARPS + warp;
+  const int ld = means_ld(m.nb);
+  double* E = sE + (size_t)warp * nbp;
+  uint32_t* w = sW + warp * m.nw;
+  if (i < m.nb) {
+    const double* src = logits + (bh * m.nb + i) * (int64_t)ld;
+    for (int j = lane; j < m.nb; j += 32) E[j] = src[j];
+    __syncwarp();
+    topp_select(E, m.nb, p, w, lane);
     const int64_t grow = bh * m.nb + i;
     finalize_row(w, i, m, fc, lane, bits + grow * m.nw, counts + grow);
+  } else {
+    for (int q = lane; q < m.nw; q += 32) w[q] = 0;
   }
-  const int t = (row0 >> 1) + warp;
-  if (2 * t < m.nb) {
-    int c = 0;
-    for (int q = lane; q < m.nw; q += 32) c += __popc(w0[q] | w0[m.nw + q]);
-    c = warp_sum(c);
-    if (lane == 0) tile_cost[bh * m.nt + t] = c;
+  __syncthreads();
+  if (warp < SEL_WARPS / 2) {
+    const int t = blockIdx.x * (SEL_WARPS / 2) + warp;
+    if (2 * t < m.nb) {
+      const uint32_t* wa = sW + (2 * warp) * m.nw;
+      const uint32_t* wb = wa + m.nw;
+      int c = 0;
+      for (int q = lane; q < m.nw; q += 32) c += __popc(wa[q] | wb[q]);
+      c = warp_sum(c);
+      if (lane == 0) tile_cost[bh * m.nt + t] = c;
+    }
   }
 }
 
@@ -756,21 +772,19 @@ cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, c
 
 size_t means_t_elems(const Dims& m) { return (size_t)m.BH * m.d * means_ld(m.nb); }
 
-cudaError_t launch_topp(const double* qT, const double* kT, const Dims& m, double p, double scale,
+cudaError_t launch_topp(const double* qT, const double* kT, double* logits, const Dims& m, double p, double scale,
                         const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
                         cudaStream_t st) {
-  const size_t smem = topp_smem_bytes(m);
-  dim3 grid((m.nb + RT - 1) / RT, (unsigned)m.BH);
-  cudaError_t e;
-  if (m.d == 128) {
-    e = cudaFuncSetAttribute(topp_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    topp_kernel<128><<<grid, 256, smem, st>>>(qT, kT, m, p, scale, fc, bits, counts, tile_cost);
-  } else {
-    e = cudaFuncSetAttribute(topp_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    topp_kernel<64><<<grid, 256, smem, st>>>(qT, kT, m, p, scale, fc, bits, counts, tile_cost);
-  }
+  dim3 g1((m.nb + ST - 1) / ST, (m.nb + ST - 1) / ST, (unsigned)m.BH);
+  if (m.d == 128) score_kernel<128><<<g1, 256, 0, st>>>(qT, kT, m, scale, logits);
+  else score_kernel<64><<<g1, 256, 0, st>>>(qT, kT, m, scale, logits);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = select_smem_bytes(m);
+  e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 g2((m.nb + SEL_WARPS - 1) / SEL_WARPS, (unsigned)m.BH);
+  select_kernel<<<g2, 256, smem, st>>>(logits, m, p, fc, bits, counts, tile_cost);
   return cudaGetLastError();
 }
 

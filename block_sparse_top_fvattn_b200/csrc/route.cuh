@@ -10,15 +10,15 @@ struct ForceCfg {
   int force_diag, local_window, frame_len, frame_window, force_first;
 };
 
-size_t topp_smem_bytes(const Dims& m);
 size_t means_t_elems(const Dims& m);     // doubles of one transposed block-mean array
+size_t logits_elems(const Dims& m);      // doubles of the fp64 block-score matrix
 size_t frame_smem_bytes(const Dims& m);
 size_t schedule_smem_bytes(const Dims& m, int* groups);
 
 // out: 0 = means [row][d], 1 = means transposed per head [bh][d][ld], 2 = frame segment sums.
 cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int out, int frame_len,
                         double* qo, double* ko, double* qhi, double* khi, int nsm, cudaStream_t st);
-cudaError_t launch_topp(const double* qT, const double* kT, const Dims& m, double p, double scale,
+cudaError_t launch_topp(const double* qT, const double* kT, double* logits, const Dims& m, double p, double scale,
                         const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
                         cudaStream_t st);
 cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,

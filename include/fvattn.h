@@ -125,7 +125,8 @@ int64_t fvattn_csr_max_nnz(const fvattn_shape* shape);
 int64_t fvattn_num_tiles(const fvattn_shape* shape);
 
 /* Workspace bytes fvattn_route needs for this shape and configuration (block means in
- * fp64, per-row selection bitmasks and counts). 0 on invalid arguments. Host only. */
+ * fp64, the fp64 block-score matrix in Top-p mode, per-row selection bitmasks and counts).
+ * 0 on invalid arguments. Host only. */
 size_t fvattn_route_workspace_bytes(const fvattn_shape* shape, const fvattn_route_cfg* cfg);
 
 /*
