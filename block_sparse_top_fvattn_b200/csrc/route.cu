@@ -423,31 +423,152 @@ __global__ void __launch_bounds__(256) score_kernel(const double* __restrict__ q
 
 constexpr int SEL_WARPS = 8;
 
-size_t select_smem_bytes(const Dims& m) {
-  return (size_t)SEL_WARPS * m.nw * 32 * 8 + (size_t)SEL_WARPS * m.nw * 4;
+// Pairwise (fixed-order) sum of the lane's masked weights, as fp64: at most log2(NE) + 1
+// roundings of fp32 relative error each.
+template <int NE>
+__device__ __forceinline__ double lane_sum(const float (&e)[NE], const uint32_t (&k)[NE], uint32_t lo_key,
+                                           bool strict) {
+  float t[NE];
+#pragma unroll
+  for (int i = 0; i < NE; ++i) t[i] = (strict ? k[i] > lo_key : k[i] >= lo_key) ? e[i] : 0.f;
+#pragma unroll
+  for (int w = 1; w < NE; w <<= 1)
+#pragma unroll
+    for (int i = 0; i + w < NE; i += 2 * w) t[i] += t[i + w];
+  return (double)t[0];
 }
 
-// One warp per query block: its fp64 logit row to shared memory, the Top-p cut, forced blocks,
-// bitmask row and count; warps 2w and 2w+1 hold the two rows of a 128-row tile and write its
-// cost (distinct key blocks of the pair).
+// The Top-p cut of one row with its weights in registers (NE per lane, element j = lane + 32 i),
+// the same rule as topp_select: weights e_j = 2^((s_j - max) log2 e) from the SFU on fp64
+// logit differences, masses compared with p * sum(e). Peaked rows are cut by max extraction
+// (REDUX on the fp32 key = the weight's bits, lowest index on ties); rows with more than
+// kExtract weights above 1/64 go straight to a bisection over the 32-bit key space. Lane sums
+// are pairwise in fp32 and folded across the warp in fp64 in a fixed order (deterministic).
+template <int NE>
+__device__ void topp_select_reg(const double* __restrict__ src, int n, double p, uint32_t* w, int lane) {
+  const int nw = (n + 31) / 32;
+  if (p >= 1.0) {
+    for (int q = lane; q < nw; q += 32) w[q] = range_bits(0, n - 1, q);
+    __syncwarp();
+    return;
+  }
+  double mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const int j = lane + 32 * i;
+    if (j < n) mx = fmax(mx, src[j]);
+  }
+  mx = warp_max(mx);
+  float e[NE];
+  uint32_t k[NE];
+  int big = 0;
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const int j = lane + 32 * i;
+    float v = 0.f;
+    if (j < n) asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(v) : "f"((float)((src[j] - mx) * 1.4426950408889634)));
+    e[i] = v;
+    k[i] = __float_as_uint(v);
+    big += v > 0.015625f;
+  }
+  const double z = warp_sum_d(lane_sum(e, k, 0u, false));
+  const double P = p * z;
+  big = warp_sum(big);
+
+  uint64_t taken = 0;
+  bool done = false;
+  if (big <= kExtract) {
+    uint32_t bkey = 0;
+    int bslot = -1;
+    auto rescan = [&]() {
+      bkey = 0;
+      bslot = -1;
+#pragma unroll
+      for (int i = 0; i < NE; ++i)
+        if (lane + 32 * i < n && !((taken >> i) & 1ull) && (bslot < 0 || k[i] > bkey)) { bkey = k[i]; bslot = i; }
+    };
+    rescan();
+    double acc = 0.0;
+    for (int it = 0; it < kExtract && !done; ++it) {
+      const uint32_t gk = __reduce_max_sync(0xffffffffu, bslot >= 0 ? bkey : 0u);
+      const uint32_t cand = (bslot >= 0 && bkey == gk) ? (uint32_t)(lane + 32 * bslot) : 0xffffffffu;
+      const uint32_t gj = __reduce_min_sync(0xffffffffu, cand);
+      if (gj == 0xffffffffu) break;
+      acc += (double)__uint_as_float(gk);
+      if ((int)(gj & 31) == lane) {
+        taken |= 1ull << (gj >> 5);
+        rescan();
+      }
+      done = acc >= P;
+    }
+  }
+  if (done) {
+#pragma unroll
+    for (int i = 0; i < NE; ++i) {
+      const uint32_t word = __ballot_sync(0xffffffffu, (taken >> i) & 1ull);
+      if (lane == 0 && i < nw) w[i] = word;
+    }
+    __syncwarp();
+    return;
+  }
+  // Bisection: largest T with mass{key >= T} >= P. Weights are at most 1, so keys <= 0x3f800000.
+  uint32_t lo = 0, hi = 0x3f800001u;
+  while (hi - lo > 1) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    const double sm = warp_sum_d(lane_sum(e, k, mid, false));
+    if (sm >= P) lo = mid;
+    else hi = mid;
+  }
+  const uint32_t T = lo;
+  double above = warp_sum_d(lane_sum(e, k, T, true));
+  const double tval = (double)__uint_as_float(T);
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const bool valid = lane + 32 * i < n;
+    uint32_t word = __ballot_sync(0xffffffffu, valid && k[i] > T);
+    uint32_t ties = __ballot_sync(0xffffffffu, valid && k[i] == T);
+    while (ties != 0u && above < P) {           // ties at the cut, lowest index first
+      const int b = __ffs(ties) - 1;
+      ties &= ties - 1;
+      above += tval;
+      word |= 1u << b;
+    }
+    if (lane == 0 && i < nw) w[i] = word;
+  }
+  __syncwarp();
+}
+
+template <int NE>
+size_t select_smem_bytes_t(const Dims& m) {
+  return NE > 0 ? (size_t)SEL_WARPS * m.nw * 4 : (size_t)SEL_WARPS * m.nw * 32 * 8 + (size_t)SEL_WARPS * m.nw * 4;
+}
+
+// One warp per query block: the Top-p cut of its fp64 logit row (in registers when the row
+// has at most 32 NE blocks, else through shared memory), forced blocks, bitmask row and count;
+// warps 2w and 2w+1 hold the two rows of a 128-row tile and write its cost.
+template <int NE>
 __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ logits, Dims m, double p,
                                                      ForceCfg fc, uint32_t* __restrict__ bits,
                                                      int32_t* __restrict__ counts, int32_t* __restrict__ tile_cost) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int nbp = m.nw * 32;
-  double* sE = reinterpret_cast<double*>(smem_raw);                               // [warp][nbp]
-  uint32_t* sW = reinterpret_cast<uint32_t*>(sE + (size_t)SEL_WARPS * nbp);      // [warp][nw]
+  uint32_t* sW = reinterpret_cast<uint32_t*>(smem_raw);                          // [warp][nw]
+  double* sE = reinterpret_cast<double*>(smem_raw + (((size_t)SEL_WARPS * m.nw * 4 + 15) & ~(size_t)15));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t bh = blockIdx.y;
   const int i = blockIdx.x * SEL_WARPS + warp;
   const int ld = means_ld(m.nb);
-  double* E = sE + (size_t)warp * nbp;
   uint32_t* w = sW + warp * m.nw;
   if (i < m.nb) {
     const double* src = logits + (bh * m.nb + i) * (int64_t)ld;
-    for (int j = lane; j < m.nb; j += 32) E[j] = src[j];
-    __syncwarp();
-    topp_select(E, m.nb, p, w, lane);
+    if (NE > 0) {
+      topp_select_reg<(NE > 0 ? NE : 1)>(src, m.nb, p, w, lane);
+    } else {
+      double* E = sE + (size_t)warp * nbp;
+      for (int j = lane; j < m.nb; j += 32) E[j] = src[j];
+      __syncwarp();
+      topp_select(E, m.nb, p, w, lane);
+    }
     const int64_t grow = bh * m.nb + i;
     finalize_row(w, i, m, fc, lane, bits + grow * m.nw, counts + grow);
   } else {
@@ -465,6 +586,17 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
       if (lane == 0) tile_cost[bh * m.nt + t] = c;
     }
   }
+}
+
+template <int NE>
+static cudaError_t launch_select_t(const double* logits, const Dims& m, double p, const ForceCfg& fc, uint32_t* bits,
+                                   int32_t* counts, int32_t* tile_cost, cudaStream_t st) {
+  const size_t smem = select_smem_bytes_t<NE>(m) + 16;
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<NE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 g((m.nb + SEL_WARPS - 1) / SEL_WARPS, (unsigned)m.BH);
+  select_kernel<NE><<<g, 256, smem, st>>>(logits, m, p, fc, bits, counts, tile_cost);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ frame mode
@@ -780,12 +912,9 @@ cudaError_t launch_topp(const double* qT, const double* kT, double* logits, cons
   else score_kernel<64><<<g1, 256, 0, st>>>(qT, kT, m, scale, logits);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem = select_smem_bytes(m);
-  e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  dim3 g2((m.nb + SEL_WARPS - 1) / SEL_WARPS, (unsigned)m.BH);
-  select_kernel<<<g2, 256, smem, st>>>(logits, m, p, fc, bits, counts, tile_cost);
-  return cudaGetLastError();
+  if (m.nb <= 32 * 16) return launch_select_t<16>(logits, m, p, fc, bits, counts, tile_cost, st);
+  if (m.nb <= 32 * 40) return launch_select_t<40>(logits, m, p, fc, bits, counts, tile_cost, st);
+  return launch_select_t<0>(logits, m, p, fc, bits, counts, tile_cost, st);
 }
 
 cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,
