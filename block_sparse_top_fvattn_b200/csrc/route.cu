@@ -452,12 +452,15 @@ __device__ void topp_select_reg(const double* __restrict__ src, int n, double p,
     __syncwarp();
     return;
   }
-  double mx = -INFINITY;
+  double s[NE];                              // the row's logits, loaded once
 #pragma unroll
   for (int i = 0; i < NE; ++i) {
     const int j = lane + 32 * i;
-    if (j < n) mx = fmax(mx, src[j]);
+    s[i] = j < n ? __ldg(src + j) : -INFINITY;
   }
+  double mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < NE; ++i) mx = fmax(mx, s[i]);
   mx = warp_max(mx);
   float e[NE];
   uint32_t k[NE];
@@ -466,7 +469,7 @@ __device__ void topp_select_reg(const double* __restrict__ src, int n, double p,
   for (int i = 0; i < NE; ++i) {
     const int j = lane + 32 * i;
     float v = 0.f;
-    if (j < n) asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(v) : "f"((float)((src[j] - mx) * 1.4426950408889634)));
+    if (j < n) asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(v) : "f"((float)((s[i] - mx) * 1.4426950408889634)));
     e[i] = v;
     k[i] = __float_as_uint(v);
     big += v > 0.015625f;
@@ -746,30 +749,38 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int32_t* __restric
   __shared__ int32_t wtot[32];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // ---- row offsets
+  // ---- row offsets: an exclusive scan of the counts in coalesced 4096-row slices, each
+  // thread taking 4 consecutive rows, carried from slice to slice.
   const int64_t N = m.BH * m.nb;
-  const int64_t per = (N + 1023) / 1024;
-  const int64_t r0 = min(N, (int64_t)tid * per), r1 = min(N, r0 + per);
-  int64_t s = 0;
-  for (int64_t r = r0; r < r1; ++r) s += counts[r];
-  const int64_t incl = warp_incl_scan(s, lane);
-  if (lane == 31) wsum[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int64_t v = wsum[lane];
-    const int64_t vi = warp_incl_scan(v, lane);
-    wsum[lane] = vi - v;
+  int64_t carry = 0;
+  for (int64_t b0 = 0; b0 < N; b0 += 4096) {
+    const int64_t r = b0 + 4 * (int64_t)tid;
+    int c[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c[e] = (r + e < N) ? counts[r + e] : 0;
+    const int64_t s = (int64_t)c[0] + c[1] + c[2] + c[3];
+    const int64_t incl = warp_incl_scan(s, lane);
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int64_t v = wsum[lane];
+      const int64_t vi = warp_incl_scan(v, lane);
+      wsum[lane] = vi;                                  // inclusive over warps
+    }
+    __syncthreads();
+    int64_t base = carry + (warp ? wsum[warp - 1] : 0) + incl - s;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (r + e < N) row_ptr[r + e] = (int32_t)base;
+      base += c[e];
+    }
+    carry += wsum[31];
+    __syncthreads();
   }
-  __syncthreads();
-  int64_t base = wsum[warp] + incl - s;
-  for (int64_t r = r0; r < r1; ++r) {
-    row_ptr[r] = (int32_t)base;
-    base += counts[r];
-  }
-  if (tid == 1023) {
-    row_ptr[N] = (int32_t)base;
-    *nnz_out = base;
-    if (base > capacity) report_error(status, FVATTN_ERR_CAPACITY, 1);
+  if (tid == 0) {
+    row_ptr[N] = (int32_t)carry;
+    *nnz_out = carry;
+    if (carry > capacity) report_error(status, FVATTN_ERR_CAPACITY, 1);
   }
   __syncthreads();
   for (int64_t bh = tid; bh < m.BH; bh += 1024)
