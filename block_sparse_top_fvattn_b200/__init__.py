@@ -32,7 +32,7 @@ BLOCK = 64
 @dataclasses.dataclass
 class RouteConfig:
     """Mirror of fvattn_route_cfg (see include/fvattn.h for the meaning of each field)."""
-    mode: str = "topp"            # "topp" | "frame_topk"
+    mode: str = "topp"            # "topp" | "frame_topk" | "topk"
     p: float = 0.9
     force_diag: bool = True
     local_window: int = 0
@@ -40,11 +40,14 @@ class RouteConfig:
     topk_frames: int = 0
     frame_window: int = -1
     force_first_frame: bool = False
+    topk_blocks: int = 0
 
     def to_c(self) -> _lib.RouteCfg:
-        mode = {"topp": FVATTN_MODE_TOPP, "frame_topk": FVATTN_MODE_FRAME_TOPK}[self.mode]
+        mode = {"topp": FVATTN_MODE_TOPP, "frame_topk": FVATTN_MODE_FRAME_TOPK,
+                "topk": _lib.FVATTN_MODE_TOPK_BLOCKS}[self.mode]
         return _lib.RouteCfg(mode, float(self.p), int(self.force_diag), int(self.local_window), int(self.frame_len),
-                             int(self.topk_frames), int(self.frame_window), int(self.force_first_frame))
+                             int(self.topk_frames), int(self.frame_window), int(self.force_first_frame),
+                             int(self.topk_blocks))
 
 
 @dataclasses.dataclass

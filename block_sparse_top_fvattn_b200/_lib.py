@@ -18,6 +18,7 @@ FVATTN_BF16 = 0
 FVATTN_F32 = 1
 FVATTN_MODE_TOPP = 0
 FVATTN_MODE_FRAME_TOPK = 1
+FVATTN_MODE_TOPK_BLOCKS = 2
 
 
 class Shape(ctypes.Structure):
@@ -28,7 +29,8 @@ class Shape(ctypes.Structure):
 class RouteCfg(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("p", ctypes.c_float), ("force_diag", ctypes.c_int32),
                 ("local_window", ctypes.c_int32), ("frame_len", ctypes.c_int32), ("topk_frames", ctypes.c_int32),
-                ("frame_window", ctypes.c_int32), ("force_first_frame", ctypes.c_int32)]
+                ("frame_window", ctypes.c_int32), ("force_first_frame", ctypes.c_int32),
+                ("topk_blocks", ctypes.c_int32)]
 
 
 class Csr(ctypes.Structure):

@@ -31,7 +31,12 @@ int validate_shape(const fvattn_shape* s) {
 
 int validate_cfg(const fvattn_shape* s, const fvattn_route_cfg* c) {
   if (c == nullptr) return FVATTN_ERR_INVALID;
-  if (c->mode != FVATTN_MODE_TOPP && c->mode != FVATTN_MODE_FRAME_TOPK) return FVATTN_ERR_INVALID;
+  if (c->mode != FVATTN_MODE_TOPP && c->mode != FVATTN_MODE_FRAME_TOPK && c->mode != FVATTN_MODE_TOPK_BLOCKS)
+    return FVATTN_ERR_INVALID;
+  if (c->mode == FVATTN_MODE_TOPK_BLOCKS) {
+    if (c->topk_blocks < 1) return FVATTN_ERR_INVALID;
+    if ((s->S + kBlock - 1) / kBlock > 1280) return FVATTN_ERR_UNSUPPORTED;
+  }
   if (!(c->p > 0.f) || isinf(c->p)) return FVATTN_ERR_INVALID;        // rejects p <= 0 and NaN
   if (c->local_window < 0 || c->frame_len < 0 || c->frame_window < -1) return FVATTN_ERR_INVALID;
   if (c->force_diag != 0 && c->force_diag != 1) return FVATTN_ERR_INVALID;
@@ -58,7 +63,8 @@ size_t take(size_t& off, size_t bytes) {
 WsLayout ws_layout(const Dims& m, int mode) {
   WsLayout L{};
   size_t off = 0;
-  const size_t means = (mode == FVATTN_MODE_TOPP ? means_t_elems(m) : (size_t)m.BH * m.nb * m.d) * sizeof(double);
+  const bool scored = mode == FVATTN_MODE_TOPP || mode == FVATTN_MODE_TOPK_BLOCKS;
+  const size_t means = (scored ? means_t_elems(m) : (size_t)m.BH * m.nb * m.d) * sizeof(double);
   L.qlo = take(off, means);
   L.klo = take(off, means);
   if (mode == FVATTN_MODE_FRAME_TOPK) {
@@ -68,7 +74,7 @@ WsLayout ws_layout(const Dims& m, int mode) {
     L.qf = take(off, fm);
     L.kf = take(off, fm);
   }
-  if (mode == FVATTN_MODE_TOPP) L.logits = take(off, logits_elems(m) * sizeof(double));
+  if (scored) L.logits = take(off, logits_elems(m) * sizeof(double));
   L.bits = take(off, (size_t)m.BH * m.nb * m.nw * sizeof(uint32_t));
   L.counts = take(off, (size_t)m.BH * m.nb * sizeof(int32_t));
   L.total = off;
@@ -153,11 +159,12 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const 
 
   if (cudaMemsetAsync(out->status, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
   cudaError_t e;
-  if (cfg->mode == FVATTN_MODE_TOPP) {
+  if (cfg->mode == FVATTN_MODE_TOPP || cfg->mode == FVATTN_MODE_TOPK_BLOCKS) {
+    const int kblocks = cfg->mode == FVATTN_MODE_TOPK_BLOCKS ? cfg->topk_blocks : 0;
     e = launch_pool(Q, K, 2, shape->dtype, m, 1, 0, qlo, klo, nullptr, nullptr, nsm, s);
     if (e == cudaSuccess)
-      e = launch_topp(qlo, klo, reinterpret_cast<double*>(ws + L.logits), m, cfg->p >= 1.f ? 1.0 : (double)cfg->p, scale, fc,
-                      bits, counts, out->tile_cost, s);
+      e = launch_topp(qlo, klo, reinterpret_cast<double*>(ws + L.logits), m, cfg->p >= 1.f ? 1.0 : (double)cfg->p,
+                      kblocks, scale, fc, bits, counts, out->tile_cost, s);
   } else {
     double* qhi = reinterpret_cast<double*>(ws + L.qhi);
     double* khi = reinterpret_cast<double*>(ws + L.khi);

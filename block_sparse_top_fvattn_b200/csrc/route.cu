@@ -541,6 +541,65 @@ __device__ void topp_select_reg(const double* __restrict__ src, int n, double p,
   __syncwarp();
 }
 
+// The kk highest scores of one row (the notes' teaching variant, §5.2: scores.topk), ties to
+// the lower block index. The order key of a block is its fp32 score relative to the row
+// maximum (s_j - max <= 0) mapped to an unsigned integer that orders like the float; the cut
+// is the largest key T with count{key >= T} >= kk, found by bisection, then every key > T and,
+// in ascending index, as many keys == T as are needed for kk.
+template <int NE>
+__device__ void topk_select_reg(const double* __restrict__ src, int n, int kk, uint32_t* w, int lane) {
+  const int nw = (n + 31) / 32;
+  if (kk >= n) {
+    for (int q = lane; q < nw; q += 32) w[q] = range_bits(0, n - 1, q);
+    __syncwarp();
+    return;
+  }
+  double s[NE];
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const int j = lane + 32 * i;
+    s[i] = j < n ? __ldg(src + j) : -INFINITY;
+  }
+  double mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < NE; ++i) mx = fmax(mx, s[i]);
+  mx = warp_max(mx);
+  uint32_t k[NE];
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const uint32_t b = __float_as_uint((float)(s[i] - mx));
+    k[i] = (lane + 32 * i < n) ? ((b & 0x80000000u) ? ~b : (b | 0x80000000u)) : 0u;
+  }
+  auto count_ge = [&](uint32_t t, bool strict) {
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < NE; ++i) c += (lane + 32 * i < n) && (strict ? k[i] > t : k[i] >= t);
+    return warp_sum(c);
+  };
+  uint32_t lo = 0, hi = 0x80000001u;       // scores relative to the maximum are <= 0
+  while (hi - lo > 1) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    if (count_ge(mid, false) >= kk) lo = mid;
+    else hi = mid;
+  }
+  const uint32_t T = lo;
+  int have = count_ge(T, true);
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const bool valid = lane + 32 * i < n;
+    uint32_t word = __ballot_sync(0xffffffffu, valid && k[i] > T);
+    uint32_t ties = __ballot_sync(0xffffffffu, valid && k[i] == T);
+    while (ties != 0u && have < kk) {
+      const int b = __ffs(ties) - 1;
+      ties &= ties - 1;
+      ++have;
+      word |= 1u << b;
+    }
+    if (lane == 0 && i < nw) w[i] = word;
+  }
+  __syncwarp();
+}
+
 template <int NE>
 size_t select_smem_bytes_t(const Dims& m) {
   return NE > 0 ? (size_t)SEL_WARPS * m.nw * 4 : (size_t)SEL_WARPS * m.nw * 32 * 8 + (size_t)SEL_WARPS * m.nw * 4;
@@ -551,7 +610,7 @@ size_t select_smem_bytes_t(const Dims& m) {
 // warps 2w and 2w+1 hold the two rows of a 128-row tile and write its cost.
 template <int NE>
 __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ logits, Dims m, double p,
-                                                     ForceCfg fc, uint32_t* __restrict__ bits,
+                                                     int kblocks, ForceCfg fc, uint32_t* __restrict__ bits,
                                                      int32_t* __restrict__ counts, int32_t* __restrict__ tile_cost) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int nbp = m.nw * 32;
@@ -565,7 +624,8 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   if (i < m.nb) {
     const double* src = logits + (bh * m.nb + i) * (int64_t)ld;
     if (NE > 0) {
-      topp_select_reg<(NE > 0 ? NE : 1)>(src, m.nb, p, w, lane);
+      if (kblocks > 0) topk_select_reg<(NE > 0 ? NE : 1)>(src, m.nb, kblocks, w, lane);
+      else topp_select_reg<(NE > 0 ? NE : 1)>(src, m.nb, p, w, lane);
     } else {
       double* E = sE + (size_t)warp * nbp;
       for (int j = lane; j < m.nb; j += 32) E[j] = src[j];
@@ -592,13 +652,13 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
 }
 
 template <int NE>
-static cudaError_t launch_select_t(const double* logits, const Dims& m, double p, const ForceCfg& fc, uint32_t* bits,
-                                   int32_t* counts, int32_t* tile_cost, cudaStream_t st) {
+static cudaError_t launch_select_t(const double* logits, const Dims& m, double p, int kblocks, const ForceCfg& fc,
+                                   uint32_t* bits, int32_t* counts, int32_t* tile_cost, cudaStream_t st) {
   const size_t smem = select_smem_bytes_t<NE>(m) + 16;
   cudaError_t e = cudaFuncSetAttribute(select_kernel<NE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 g((m.nb + SEL_WARPS - 1) / SEL_WARPS, (unsigned)m.BH);
-  select_kernel<NE><<<g, 256, smem, st>>>(logits, m, p, fc, bits, counts, tile_cost);
+  select_kernel<NE><<<g, 256, smem, st>>>(logits, m, p, kblocks, fc, bits, counts, tile_cost);
   return cudaGetLastError();
 }
 
@@ -915,7 +975,8 @@ cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, c
 
 size_t means_t_elems(const Dims& m) { return (size_t)m.BH * m.d * means_ld(m.nb); }
 
-cudaError_t launch_topp(const double* qT, const double* kT, double* logits, const Dims& m, double p, double scale,
+cudaError_t launch_topp(const double* qT, const double* kT, double* logits, const Dims& m, double p, int kblocks,
+                        double scale,
                         const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
                         cudaStream_t st) {
   dim3 g1((m.nb + ST - 1) / ST, (m.nb + ST - 1) / ST, (unsigned)m.BH);
@@ -923,9 +984,9 @@ cudaError_t launch_topp(const double* qT, const double* kT, double* logits, cons
   else score_kernel<64><<<g1, 256, 0, st>>>(qT, kT, m, scale, logits);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (m.nb <= 32 * 16) return launch_select_t<16>(logits, m, p, fc, bits, counts, tile_cost, st);
-  if (m.nb <= 32 * 40) return launch_select_t<40>(logits, m, p, fc, bits, counts, tile_cost, st);
-  return launch_select_t<0>(logits, m, p, fc, bits, counts, tile_cost, st);
+  if (m.nb <= 32 * 16) return launch_select_t<16>(logits, m, p, kblocks, fc, bits, counts, tile_cost, st);
+  if (m.nb <= 32 * 40) return launch_select_t<40>(logits, m, p, kblocks, fc, bits, counts, tile_cost, st);
+  return launch_select_t<0>(logits, m, p, 0, fc, bits, counts, tile_cost, st);
 }
 
 cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,

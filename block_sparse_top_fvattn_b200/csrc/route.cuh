@@ -18,7 +18,9 @@ size_t schedule_smem_bytes(const Dims& m, int* groups);
 // out: 0 = means [row][d], 1 = means transposed per head [bh][d][ld], 2 = frame segment sums.
 cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int out, int frame_len,
                         double* qo, double* ko, double* qhi, double* khi, int nsm, cudaStream_t st);
-cudaError_t launch_topp(const double* qT, const double* kT, double* logits, const Dims& m, double p, double scale,
+// kblocks > 0: keep the kblocks highest scores per row instead of the Top-p cut.
+cudaError_t launch_topp(const double* qT, const double* kT, double* logits, const Dims& m, double p, int kblocks,
+                        double scale,
                         const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
                         cudaStream_t st);
 cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,

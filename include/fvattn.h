@@ -48,7 +48,9 @@ typedef enum { FVATTN_BF16 = 0, FVATTN_F32 = 1 } fvattn_dtype;
 
 typedef enum {
   FVATTN_MODE_TOPP = 0,        /* FVAttn Top-p over key blocks                             */
-  FVATTN_MODE_FRAME_TOPK = 1   /* Sol-Attn frame-level top-k (vLLM-Omni article §2.1-§2.2) */
+  FVATTN_MODE_FRAME_TOPK = 1,  /* Sol-Attn frame-level top-k (vLLM-Omni article §2.1-§2.2) */
+  FVATTN_MODE_TOPK_BLOCKS = 2  /* a fixed number of key blocks per query block (the notes'
+                                  teaching variant, §5.2: scores.topk(topk_blocks))        */
 } fvattn_mode;
 
 /* Problem shape. block must be 64; d must be 64 or 128; scale <= 0 means 1/sqrt(d). */
@@ -70,7 +72,9 @@ typedef struct {
  *  frame_window      fw >= 0 keeps the frames within +-fw of the query block's frames
  *                    (Sol-Attn §2.2, neighbouring frames); -1 disables.
  *  force_first_frame 1: the blocks of frame 0 are always kept (Sol-Attn §5.2).
- * Forced blocks are added after the Top-p cut (a union); they do not count toward p.
+ *  topk_blocks       FVATTN_MODE_TOPK_BLOCKS: key blocks kept per query block by score
+ *                    (>= 1; ties go to the lower block index); at most 1280 blocks per row.
+ * Forced blocks are added after the cut (a union); they do not count toward p or k.
  */
 typedef struct {
   int32_t mode;
@@ -81,6 +85,7 @@ typedef struct {
   int32_t topk_frames;
   int32_t frame_window;
   int32_t force_first_frame;
+  int32_t topk_blocks;
 } fvattn_route_cfg;
 
 /*
@@ -135,6 +140,7 @@ size_t fvattn_route_workspace_bytes(const fvattn_shape* shape, const fvattn_rout
  *      accumulated exactly enough to be held in fp64;
  *   2. Top-p: scores Sc[i][j] = <Qbar_i, Kbar_j> * scale in fp64, softmax over j, and the
  *      smallest descending-probability prefix whose mass is >= p (ties: lower j first);
+ *      fixed top-k: the same scores, the k highest per row (ties: lower j first);
  *      frame mode: frame means, frame scores, top-k frames per query frame, expanded to the
  *      key blocks that hold tokens of a kept frame;
  *   3. union with the forced blocks of cfg; CSR rows (ascending), per-head loads, tile

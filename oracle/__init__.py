@@ -25,13 +25,13 @@ forms, brute force on tiny inputs, hand-computed golden cases (tests/golden/) an
 routines (torch scaled_dot_product_attention). No function is unpinned.
 """
 from .route import (RouteCfg, pool_blocks, pool_frames, block_scores, row_softmax,
-                    topp_row, forced_blocks, frame_topk_select, route, near_tie_rows,
+                    topp_row, topk_row, forced_blocks, frame_topk_select, route, near_tie_rows,
                     valid_near_tie_set)
 from .attention import attention_sets, attention_token_mask, attention_rows, selected_flops
 from .schedule import csr_from_mask, head_loads, tile_costs, lpt_order
 
 __all__ = [
-    "RouteCfg", "pool_blocks", "pool_frames", "block_scores", "row_softmax", "topp_row",
+    "RouteCfg", "pool_blocks", "pool_frames", "block_scores", "row_softmax", "topp_row", "topk_row",
     "forced_blocks", "frame_topk_select", "route", "near_tie_rows", "valid_near_tie_set",
     "attention_sets", "attention_token_mask", "attention_rows", "selected_flops",
     "csr_from_mask", "head_loads", "tile_costs", "lpt_order",

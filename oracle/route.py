@@ -19,13 +19,15 @@ EPS_MASS = 1e-5   # distance of a cumulative mass from p under which the cut cou
 class RouteCfg:
     """Routing configuration.
 
-    mode         "topp" (FVAttn Top-p) or "frame_topk" (Sol-Attn frame-level top-k).
+    mode         "topp" (FVAttn Top-p), "frame_topk" (Sol-Attn frame-level top-k) or "topk"
+                 (a fixed number of key blocks per query block, the notes' teaching variant).
     p            Top-p mass threshold; p >= 1 selects every key block.
     block        tokens per block (the pages use 32 or 64; the library supports 64).
     force_diag   always keep key block i for query block i.
     local_window w > 0 forces the band |i - j| <= w (wzjinhao notes §5.2 "邻近块保底").
     frame_len    tokens per frame (0: no frame structure).
     topk_frames  k for frame mode.
+    topk_blocks  k for "topk" mode.
     frame_window fw >= 0 forces the frames within +-fw of the query's frames; < 0 disables.
     force_first_frame  always keep the blocks of frame 0.
     scale        softmax scale; None means 1/sqrt(d).
@@ -37,6 +39,7 @@ class RouteCfg:
     local_window: int = 0
     frame_len: int = 0
     topk_frames: int = 0
+    topk_blocks: int = 0
     frame_window: int = -1
     force_first_frame: bool = False
     scale: Optional[float] = None
@@ -109,6 +112,13 @@ def topp_row(pi: np.ndarray, p: float):
     reach = np.nonzero(csum >= p)[0]
     k_star = int(reach[0]) + 1 if reach.size else nb
     return order, k_star, csum
+
+
+def topk_row(sc: np.ndarray, k: int) -> np.ndarray:
+    """The k highest block scores of one row (wzjinhao notes §5.2: scores.topk(topk_blocks));
+    ties go to the lower block index. Returns the kept indices in descending score order."""
+    order = np.argsort(-sc, kind="stable")
+    return order[:min(k, sc.shape[0])]
 
 
 def _frames_of_block(j: int, S: int, block: int, frame_len: int):
@@ -213,6 +223,14 @@ def route(Q, K, cfg: RouteCfg):
                 routed[bh, i, order[:ks]] = True
                 kstar[bh, i] = ks
         out.update(pi=pi, kstar=kstar, qbar=qbar, kbar=kbar)
+    elif cfg.mode == "topk":
+        qbar, kbar = pool_blocks(Q, bs), pool_blocks(K, bs)
+        sc = block_scores(qbar, kbar, scale)
+        routed = np.zeros((BH, nb, nb), dtype=bool)
+        for bh in range(BH):
+            for i in range(nb):
+                routed[bh, i, topk_row(sc[bh, i], cfg.topk_blocks)] = True
+        out.update(scores=sc, qbar=qbar, kbar=kbar)
     elif cfg.mode == "frame_topk":
         qf, kf = pool_frames(Q, cfg.frame_len), pool_frames(K, cfg.frame_len)
         routed, fs, chosen = frame_topk_select(qf, kf, S, cfg, scale)
@@ -233,6 +251,15 @@ def near_tie_rows(r: dict, S: int, cfg: RouteCfg) -> np.ndarray:
     mask = r["mask"]
     BH, nb, _ = mask.shape
     near = np.zeros((BH, nb), dtype=bool)
+    if cfg.mode == "topk":
+        k = min(cfg.topk_blocks, nb)
+        if k >= nb:
+            return near
+        for bh in range(BH):
+            for i in range(nb):
+                srt = np.sort(r["scores"][bh, i])[::-1]
+                near[bh, i] = (srt[k - 1] - srt[k]) < EPS_GAP * max(1.0, abs(srt[k - 1]))
+        return near
     if cfg.mode == "topp":
         if cfg.p >= 1.0:
             return near
@@ -272,6 +299,15 @@ def valid_near_tie_set(r: dict, bh: int, i: int, gpu_row: np.ndarray, S: int, cf
     gpu_row = np.asarray(gpu_row, dtype=bool)
     if np.any(forced & ~gpu_row):
         return False
+    if cfg.mode == "topk":
+        sc = r["scores"][bh, i]
+        k = min(cfg.topk_blocks, sc.shape[0])
+        srt = np.sort(sc)[::-1]
+        eps = EPS_GAP * max(1.0, abs(srt[k - 1]))
+        lo_cut = srt[k] if k < sc.shape[0] else -np.inf
+        must = (sc > srt[k - 1] + eps) | forced
+        may = (sc >= lo_cut - eps) | forced
+        return bool(np.all(gpu_row[must]) and not np.any(gpu_row & ~may))
     if cfg.mode == "topp":
         pi = r["pi"][bh, i]
         order, ks, csum = topp_row(pi, cfg.p)

@@ -41,7 +41,7 @@ def gpu_mask(csr) -> np.ndarray:
 def to_oracle_cfg(cfg: fv.RouteConfig) -> oracle.RouteCfg:
     return oracle.RouteCfg(mode=cfg.mode, p=cfg.p, force_diag=cfg.force_diag, local_window=cfg.local_window,
                            frame_len=cfg.frame_len, topk_frames=cfg.topk_frames, frame_window=cfg.frame_window,
-                           force_first_frame=cfg.force_first_frame)
+                           force_first_frame=cfg.force_first_frame, topk_blocks=cfg.topk_blocks)
 
 
 def check_route(q, k, cfg: fv.RouteConfig, csr=None, r=None):
@@ -146,6 +146,24 @@ def test_frame_mode_parity(fl, topk, fw, first):
     cfg = fv.RouteConfig(mode="frame_topk", topk_frames=topk, frame_len=fl, frame_window=fw,
                          force_first_frame=first, force_diag=True)
     check_route(q, k, cfg)
+
+
+TOPK_CASES = [
+    ("single", {"H": 3, "S": 3000}, fv.RouteConfig(mode="topk", topk_blocks=8, local_window=2, force_diag=False)),
+    ("single", {"H": 2, "S": 8192, "alpha": ("const", 0.3)}, fv.RouteConfig(mode="topk", topk_blocks=5)),
+    ("tiny", {}, fv.RouteConfig(mode="topk", topk_blocks=16, force_diag=False)),        # k = nb: dense
+    ("single", {"H": 2, "S": 700}, fv.RouteConfig(mode="topk", topk_blocks=1, force_diag=False)),
+]
+
+
+@pytest.mark.parametrize("name,kw,cfg", TOPK_CASES)
+def test_topk_blocks_parity(name, kw, cfg):
+    w, q, k, v = small_inputs(name, **kw)
+    csr, gm, r = check_route(q, k, cfg)
+    if cfg.topk_blocks >= w.nb:
+        assert gm.all()
+    if w.dtype == "bf16":
+        check_attention(q, k, v, csr, gm, 1.0 / np.sqrt(w.d))
 
 
 def test_route_deterministic():

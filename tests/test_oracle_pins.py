@@ -287,3 +287,37 @@ def test_selected_flops_hand():
     m = np.zeros((1, 2, 2), bool)
     m[0, 0, 1] = True; m[0, 1, 1] = True     # S = 100: block 0 = 64 tokens, block 1 = 36
     assert oracle.selected_flops(m, 100, 64, 16) == 4 * 16 * (64 * 36 + 36 * 36)
+
+
+# ---------------------------------------------------------------- fixed top-k (notes §5.2)
+
+def test_topk_row_hand_and_ties():
+    sc = np.array([0.5, 2.0, -1.0, 2.0, 1.5])
+    assert oracle.topk_row(sc, 1).tolist() == [1]                  # tie 2.0 / 2.0: lower index first
+    assert oracle.topk_row(sc, 3).tolist() == [1, 3, 4]
+    assert sorted(oracle.topk_row(sc, 9).tolist()) == [0, 1, 2, 3, 4]
+
+
+def test_topk_mode_full_coverage_is_dense_like_the_notes_test():
+    # The notes' own correctness check: topk_blocks = nb and local_window = nb -> dense.
+    w, Q, K, V = _small(H=2, S=512, d=64, frame_len=256, region_len=64, dtype="f32", seed=0)
+    r = oracle.route(Q, K, oracle.RouteCfg(mode="topk", topk_blocks=8, local_window=8, force_diag=False))
+    assert r["mask"].all()
+    o = oracle.attention_sets(Q, K, V, r["mask"], 1 / 8.0)
+    dense = torch.nn.functional.scaled_dot_product_attention(Q.double(), K.double(), V.double()).numpy()
+    assert np.abs(o - dense).max() < 1e-12
+
+
+def test_topk_mode_matches_brute_force_ranking():
+    w, Q, K, _ = _small(H=2, S=1000, frame_len=500, region_len=128, seed=21)
+    cfg = oracle.RouteCfg(mode="topk", topk_blocks=3, force_diag=False)
+    r = oracle.route(Q, K, cfg)
+    Qd, Kd = Q.double().numpy(), K.double().numpy()
+    nb = 16
+    for bh in range(2):
+        qm = [Qd[bh, i * 64:min(1000, i * 64 + 64)].mean(axis=0) for i in range(nb)]
+        km = [Kd[bh, j * 64:min(1000, j * 64 + 64)].mean(axis=0) for j in range(nb)]
+        for i in range(nb):
+            s = [float(np.dot(qm[i], km[j])) for j in range(nb)]
+            top = sorted(range(nb), key=lambda j: (-s[j], j))[:3]
+            assert sorted(np.nonzero(r["mask"][bh, i])[0].tolist()) == sorted(top)
