@@ -13,7 +13,8 @@ Sources (page title, section):
   * FVAttn blog summary "腾讯+中山大学新作：视频生成提速2.11×，靠的是RLB和SASA",
     section "AI视频生成的阿喀琉斯之踵…": Top-p routing keeps, per query, the smallest
     descending-importance set of key blocks whose cumulative importance reaches p;
-    section "RLB…": per-head load = number of blocks each head must compute, heaviest first.
+    section "RLB…": per-head load = number of blocks each head must compute, heaviest first;
+    section "SASA…": fill a unit's slack with the best blocks routing left out, within a budget.
   * Video-generation acceleration notes (wzjinhao.cn) §5.2 "块稀疏注意力的教学实现":
     block representatives are token means, block score = mean(Q_blk)·mean(K_blk)/sqrt(d),
     a forced local band, then masked softmax attention; §5.3: full coverage equals dense.
@@ -26,13 +27,14 @@ routines (torch scaled_dot_product_attention). No function is unpinned.
 """
 from .route import (RouteCfg, pool_blocks, pool_frames, block_scores, row_softmax,
                     topp_row, topk_row, forced_blocks, frame_topk_select, route, near_tie_rows,
-                    valid_near_tie_set)
+                    valid_near_tie_set, sasa_tile_augment, sasa_near_tie_rows, valid_sasa_row)
 from .attention import attention_sets, attention_token_mask, attention_rows, selected_flops
 from .schedule import csr_from_mask, head_loads, tile_costs, lpt_order
 
 __all__ = [
     "RouteCfg", "pool_blocks", "pool_frames", "block_scores", "row_softmax", "topp_row", "topk_row",
     "forced_blocks", "frame_topk_select", "route", "near_tie_rows", "valid_near_tie_set",
+    "sasa_tile_augment", "sasa_near_tie_rows", "valid_sasa_row",
     "attention_sets", "attention_token_mask", "attention_rows", "selected_flops",
     "csr_from_mask", "head_loads", "tile_costs", "lpt_order",
 ]

@@ -31,6 +31,9 @@ class RouteCfg:
     frame_window fw >= 0 forces the frames within +-fw of the query's frames; < 0 disables.
     force_first_frame  always keep the blocks of frame 0.
     scale        softmax scale; None means 1/sqrt(d).
+    sasa_coef    augmentation coefficient in [0, 1] of slack-aware sparse augmentation
+                 (sasa_tile_augment); 0 disables it. Top-p and "topk" modes only.
+    sasa_trigger smallest slack, in key blocks, at which a row is augmented.
     """
     mode: str = "topp"
     p: float = 0.9
@@ -43,6 +46,8 @@ class RouteCfg:
     frame_window: int = -1
     force_first_frame: bool = False
     scale: Optional[float] = None
+    sasa_coef: float = 0.0
+    sasa_trigger: int = 1
 
 
 def _f64(x) -> np.ndarray:
@@ -240,7 +245,118 @@ def route(Q, K, cfg: RouteCfg):
     out["routed"] = routed
     out["mask"] = routed | forced[None]
     out["near_tie"] = near_tie_rows(out, S, cfg)
+    if cfg.sasa_coef > 0.0:
+        if cfg.mode == "frame_topk":
+            raise ValueError("slack-aware augmentation needs a per-block order (topp or topk mode)")
+        key = out["pi"] if cfg.mode == "topp" else out["scores"]
+        base = out["mask"]
+        out["base_mask"] = base
+        out["mask"] = sasa_tile_augment(base, key, cfg.sasa_coef, cfg.sasa_trigger)
+        tie = out["near_tie"] | sasa_near_tie_rows(base, key, cfg.sasa_coef, cfg.sasa_trigger, cfg.mode)
+        # a tile's augmentation reads both rows' sets, so a tie in either row reaches both
+        partner = tie.copy()
+        partner[:, 0:nb - nb % 2:2] |= tie[:, 1:nb - nb % 2 + 1:2]
+        partner[:, 1::2] |= tie[:, 0:nb - nb % 2:2]
+        out["base_near_tie"] = out["near_tie"]
+        out["near_tie"] = partner
     return out
+
+
+def _sasa_budget(coef: float, slack: int, trigger: int) -> int:
+    """Blocks added to a row with `slack` free key-block steps: floor(coef * slack) once the
+    slack reaches the trigger. coef is taken at float32 precision (the configuration's type)
+    and the product formed in float64, where it is exact."""
+    if slack <= 0 or slack < trigger:
+        return 0
+    return int(math.floor(float(np.float32(coef)) * slack))
+
+
+def _sasa_candidates(mask_bh: np.ndarray, r: int):
+    """Candidates of row r of one head: key blocks of its tile's union that r did not select
+    (the tile's rows are query blocks 2t and 2t+1). None for a row without a partner."""
+    nb = mask_bh.shape[0]
+    partner = r ^ 1
+    if partner >= nb:
+        return None
+    union = mask_bh[r] | mask_bh[partner]
+    return np.nonzero(union & ~mask_bh[r])[0]
+
+
+def sasa_tile_augment(mask: np.ndarray, key: np.ndarray, coef: float, trigger: int) -> np.ndarray:
+    """Slack-aware sparse augmentation (FVAttn summary, section "SASA") on one GPU.
+
+    The pages' slack is the idle time a rank would spend at a synchronisation point; SASA fills
+    it, up to a budget set by an augmentation coefficient and a trigger threshold, with the
+    highest-importance blocks that routing left out, reusing routing's importance order and
+    never lengthening the critical path. On one GPU the synchronous unit is the 128-row
+    attention tile: query blocks 2t and 2t+1 step through the union of their key blocks
+    together, so a row's slack is the number of union blocks it did not select, and filling it
+    costs no extra tile step. Row r with slack s >= trigger gains the floor(coef * s)
+    candidates ranked highest by `key` (pi in Top-p mode, the block score in top-k mode; ties
+    to the lower block index). Both rows are augmented from the sets before augmentation; the
+    union, hence the tile's cost, is unchanged.
+
+    mask [BH, nb, nb] bool (routed set union forced set), key [BH, nb, nb]. Returns a new mask.
+    """
+    out = mask.copy()
+    BH, nb, _ = mask.shape
+    for bh in range(BH):
+        for r in range(nb):
+            cand = _sasa_candidates(mask[bh], r)
+            if cand is None:
+                continue
+            n = _sasa_budget(coef, cand.size, trigger)
+            if n == 0:
+                continue
+            ranked = cand[np.argsort(-key[bh, r, cand], kind="stable")]
+            out[bh, r, ranked[:n]] = True
+    return out
+
+
+def _gap_eps(v: float, mode: str) -> float:
+    return EPS_GAP if mode == "topp" else EPS_GAP * max(1.0, abs(v))
+
+
+def sasa_near_tie_rows(mask: np.ndarray, key: np.ndarray, coef: float, trigger: int, mode: str) -> np.ndarray:
+    """Rows whose augmentation is decided by a key gap below the stated resolution: the last
+    candidate added and the first one left out differ by less than EPS_GAP (in pi; in top-k
+    mode relative to the score)."""
+    BH, nb, _ = mask.shape
+    near = np.zeros((BH, nb), dtype=bool)
+    for bh in range(BH):
+        for r in range(nb):
+            cand = _sasa_candidates(mask[bh], r)
+            if cand is None:
+                continue
+            n = _sasa_budget(coef, cand.size, trigger)
+            if n == 0 or n >= cand.size:
+                continue
+            srt = np.sort(key[bh, r, cand])[::-1]
+            near[bh, r] = (srt[n - 1] - srt[n]) < _gap_eps(srt[n - 1], mode)
+    return near
+
+
+def valid_sasa_row(key_row: np.ndarray, base_row: np.ndarray, partner_row: np.ndarray, final_row: np.ndarray,
+                   coef: float, trigger: int, mode: str) -> bool:
+    """Is `final_row` an acceptable augmentation of `base_row` (its tile partner's set
+    `partner_row`) when the choice is a near-tie? It must keep the base set, add exactly the
+    budget from the candidates only, and add no candidate ranked clearly below one it left out."""
+    base_row, partner_row, final_row = (np.asarray(x, dtype=bool) for x in (base_row, partner_row, final_row))
+    if np.any(base_row & ~final_row):
+        return False
+    cand_mask = (base_row | partner_row) & ~base_row
+    added = final_row & ~base_row
+    if np.any(added & ~cand_mask):
+        return False
+    n = _sasa_budget(coef, int(cand_mask.sum()), trigger)
+    if int(added.sum()) != n:
+        return False
+    left = cand_mask & ~added
+    if n == 0 or not left.any():
+        return True
+    lo_added = key_row[added].min()
+    hi_left = key_row[left].max()
+    return bool(lo_added >= hi_left - _gap_eps(lo_added, mode))
 
 
 def near_tie_rows(r: dict, S: int, cfg: RouteCfg) -> np.ndarray:

@@ -321,3 +321,103 @@ def test_topk_mode_matches_brute_force_ranking():
             s = [float(np.dot(qm[i], km[j])) for j in range(nb)]
             top = sorted(range(nb), key=lambda j: (-s[j], j))[:3]
             assert sorted(np.nonzero(r["mask"][bh, i])[0].tolist()) == sorted(top)
+
+
+# ---------------------------------------------------------------- slack-aware augmentation (SASA)
+
+def _sets_to_mask(sets, nb):
+    m = np.zeros((1, nb, nb), dtype=bool)
+    for i, s in enumerate(sets):
+        m[0, i, s] = True
+    return m
+
+
+def test_sasa_golden_hand_cases():
+    cases = json.load(open(os.path.join(GOLDEN, "sasa_hand_cases.json")))["cases"]
+    for c in cases:
+        nb = c["nb"]
+        key = np.array(c["key"], dtype=np.float64)[None]
+        out = oracle.sasa_tile_augment(_sets_to_mask(c["mask"], nb), key, c["coef"], c["trigger"])
+        got = [np.nonzero(out[0, i])[0].tolist() for i in range(nb)]
+        assert got == c["expect"], c["why"]
+
+
+def _random_tile_masks(rng, BH, nb, density):
+    mask = rng.random((BH, nb, nb)) < density
+    mask[:, np.arange(nb), np.arange(nb)] = True        # every row non-empty, as routing guarantees
+    return mask
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_sasa_budget_and_brute_force_best_mass(seed):
+    # Closed-form count (floor(coef * slack) when slack >= trigger) and, by brute force over every
+    # subset of the candidates of that size, the added set has the largest importance mass.
+    rng = np.random.default_rng(seed)
+    nb = int(rng.integers(2, 9))
+    mask = _random_tile_masks(rng, 2, nb, 0.35)
+    key = rng.random((2, nb, nb))
+    coef = float(rng.choice([0.25, 0.5, 0.75, 1.0, 0.3]))
+    trigger = int(rng.integers(0, 3))
+    out = oracle.sasa_tile_augment(mask, key, coef, trigger)
+    for bh in range(2):
+        for r in range(nb):
+            if r ^ 1 >= nb:
+                assert np.array_equal(out[bh, r], mask[bh, r])
+                continue
+            union = mask[bh, r] | mask[bh, r ^ 1]
+            cand = np.nonzero(union & ~mask[bh, r])[0]
+            slack = cand.size
+            n = math.floor(float(np.float32(coef)) * slack) if slack >= trigger and slack > 0 else 0
+            added = np.nonzero(out[bh, r] & ~mask[bh, r])[0]
+            assert added.size == n
+            assert np.all(mask[bh, r] <= out[bh, r])
+            if n:
+                best = max(key[bh, r, list(s)].sum() for s in itertools.combinations(cand, n))
+                assert key[bh, r, added].sum() == pytest.approx(best, rel=0, abs=1e-15)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_sasa_tile_union_unchanged_and_coef_one_fills_union(seed):
+    rng = np.random.default_rng(100 + seed)
+    nb = 9
+    mask = _random_tile_masks(rng, 3, nb, 0.3)
+    key = rng.random((3, nb, nb))
+    for coef in (0.5, 1.0):
+        out = oracle.sasa_tile_augment(mask, key, coef, 1)
+        for t in range(nb // 2):
+            a, b = 2 * t, 2 * t + 1
+            assert np.array_equal(out[:, a] | out[:, b], mask[:, a] | mask[:, b])   # tile cost unchanged
+            if coef == 1.0:
+                assert np.array_equal(out[:, a], mask[:, a] | mask[:, b])
+                assert np.array_equal(out[:, b], mask[:, a] | mask[:, b])
+        assert np.array_equal(out[:, nb - 1], mask[:, nb - 1])                      # odd tail, no partner
+    assert np.array_equal(oracle.sasa_tile_augment(mask, key, 0.0, 1), mask)
+    assert np.array_equal(oracle.sasa_tile_augment(mask, key, 1.0, nb + 1), mask)  # trigger never reached
+
+
+def test_sasa_ties_go_to_lower_block_and_route_integration():
+    # All candidates tied: the lowest indices are added. Through route(): the augmented mask keeps
+    # the base mask, and the near-tie flags cover the tied rows.
+    mask = _sets_to_mask([[0], [1, 2, 3, 4, 5]], 6)
+    key = np.full((1, 6, 6), 0.1)
+    out = oracle.sasa_tile_augment(mask, key, 0.5, 1)
+    assert np.nonzero(out[0, 0])[0].tolist() == [0, 1, 2]
+    assert oracle.sasa_near_tie_rows(mask, key, 0.5, 1, "topp")[0, 0]
+    # a valid near-tie alternative: another 2 of the tied candidates
+    alt = mask[0, 0].copy()
+    alt[[4, 5]] = True
+    assert oracle.valid_sasa_row(key[0, 0], mask[0, 0], mask[0, 1], alt, 0.5, 1, "topp")
+    bad = mask[0, 0].copy()
+    bad[[4]] = True                                        # wrong count
+    assert not oracle.valid_sasa_row(key[0, 0], mask[0, 0], mask[0, 1], bad, 0.5, 1, "topp")
+
+    x = make_inputs(get_workload("tiny"), device="cpu")
+    BH = x["q"].shape[0] * x["q"].shape[1]
+    Q = x["q"].reshape(BH, -1, x["q"].shape[-1])
+    K = x["k"].reshape(BH, -1, x["k"].shape[-1])
+    base = oracle.route(Q, K, oracle.RouteCfg(p=0.6))
+    aug = oracle.route(Q, K, oracle.RouteCfg(p=0.6, sasa_coef=1.0, sasa_trigger=1))
+    assert np.array_equal(aug["base_mask"], base["mask"])
+    assert np.all(base["mask"] <= aug["mask"])
+    assert aug["mask"].sum() > base["mask"].sum()
+    assert np.array_equal(oracle.tile_costs(aug["mask"]), oracle.tile_costs(base["mask"]))
