@@ -46,9 +46,11 @@ def env_rank():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
 
 
-def workload_desc(w, mode: str = "topp", topk_frames: int = 4) -> str:
+def workload_desc(w, mode: str = "topp", topk_frames: int = 4, sasa_coef: float = 0.0, sasa_trigger: int = 1) -> str:
     sel = (f"p={w.p},diag forced" if mode == "topp" else
            f"frame top-k={topk_frames} + frames +-1 + frame 0 + diag")
+    if sasa_coef > 0:
+        sel += f",tile slack augmentation coef={sasa_coef} trigger={sasa_trigger}"
     return (f"{w.name}: B={w.B},H={w.H},S={w.S} ({w.frames} frames x {w.frame_len} tokens),d={w.d},{w.dtype},"
             f"block=64,{sel}")
 
@@ -122,6 +124,12 @@ def selected_flops_from_csr(csr, S: int, d: int):
     padded = int(counts.sum().item()) * 64 * 64
     kv_tokens = int(n[kj].sum().item())
     return 4 * d * pairs, nnz, 4 * d * padded, kv_tokens
+
+
+def tile_mma_flops(csr, d: int) -> int:
+    """FLOPs the attention kernel's MMAs issue: every key block of a 128-row tile's union is one
+    128 x 64 step of S = Q K^T and O += P V, whichever of the tile's two rows selected it."""
+    return 4 * d * 128 * 64 * int(csr.tile_cost.long().sum().item())
 
 
 def router_bytes(BH: int, S: int, d: int, esize: int, nb: int, nnz: int) -> int:
@@ -250,7 +258,7 @@ def run_ours(args, w):
         cfg = fv.RouteConfig(mode="frame_topk", topk_frames=args.topk_frames, frame_len=w.frame_len, frame_window=1,
                              force_first_frame=True, force_diag=True)
     else:
-        cfg = fv.RouteConfig(p=w.p, force_diag=True)
+        cfg = fv.RouteConfig(p=w.p, force_diag=True, sasa_coef=args.sasa_coef, sasa_trigger=args.sasa_trigger)
     csr = fv.alloc_csr(B, H, S, dev)
     ws = torch.empty(fv.workspace_bytes(q, cfg), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
@@ -267,6 +275,7 @@ def run_ours(args, w):
         raise RuntimeError(f"device status {fv.read_status(csr)}")
     flops, nnz, flops_padded, kv_tokens = selected_flops_from_csr(csr, S, d)
     density = nnz / (BH * csr.nb * csr.nb)
+    mma_flops = tile_mma_flops(csr, d)
 
     # timed region: K steps; per-kernel events on the launching stream
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
@@ -352,13 +361,14 @@ def run_ours(args, w):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": workload_desc(w, args.mode, args.topk_frames),
+        "config": {"workload": workload_desc(w, args.mode, args.topk_frames, args.sasa_coef, args.sasa_trigger),
                    "l2": f"inputs larger than L2 (Q,K,V = {3 * q.numel() * q.element_size() / 1e9:.2f} GB per layer)",
                    "parallelism": f"independent layer per GPU x{world}"},
         "route_ms": route_avg, "attn_ms": attn_avg, "attn_tflops": attn_tflops,
         "pct_bf16_peak": 100.0 * value / pk["bf16_tflops"],
         "pct_bf16_peak_attn": 100.0 * attn_tflops / pk["bf16_tflops"],
         "density": density, "selected_flops_per_layer": flops, "padded_tile_flops_per_layer": flops_padded,
+        "tile_mma_flops_per_layer": mma_flops, "tile_utilisation": flops / mma_flops if mma_flops else None,
         "selected_kv_tokens_per_s": kv_tokens / (attn_avg * 1e-3),
         "query_tokens_per_s": BH * S / (ms_step * 1e-3),
         "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": attn_tflops, "peak": bf16_peak,
@@ -389,6 +399,8 @@ def main():
     ap.add_argument("--p", type=float, default=0.0, help="override the Top-p threshold")
     ap.add_argument("--mode", default="topp", choices=["topp", "frame_topk"])
     ap.add_argument("--topk-frames", type=int, default=4)
+    ap.add_argument("--sasa-coef", type=float, default=0.0, help="tile slack augmentation coefficient (0: off)")
+    ap.add_argument("--sasa-trigger", type=int, default=1)
     args = ap.parse_args()
     from workloads import get_workload
     w = get_workload(args.workload)

@@ -41,13 +41,15 @@ class RouteConfig:
     frame_window: int = -1
     force_first_frame: bool = False
     topk_blocks: int = 0
+    sasa_coef: float = 0.0
+    sasa_trigger: int = 1
 
     def to_c(self) -> _lib.RouteCfg:
         mode = {"topp": FVATTN_MODE_TOPP, "frame_topk": FVATTN_MODE_FRAME_TOPK,
                 "topk": _lib.FVATTN_MODE_TOPK_BLOCKS}[self.mode]
         return _lib.RouteCfg(mode, float(self.p), int(self.force_diag), int(self.local_window), int(self.frame_len),
                              int(self.topk_frames), int(self.frame_window), int(self.force_first_frame),
-                             int(self.topk_blocks))
+                             int(self.topk_blocks), float(self.sasa_coef), int(self.sasa_trigger))
 
 
 @dataclasses.dataclass

@@ -30,7 +30,7 @@ class RouteCfg(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("p", ctypes.c_float), ("force_diag", ctypes.c_int32),
                 ("local_window", ctypes.c_int32), ("frame_len", ctypes.c_int32), ("topk_frames", ctypes.c_int32),
                 ("frame_window", ctypes.c_int32), ("force_first_frame", ctypes.c_int32),
-                ("topk_blocks", ctypes.c_int32)]
+                ("topk_blocks", ctypes.c_int32), ("sasa_coef", ctypes.c_float), ("sasa_trigger", ctypes.c_int32)]
 
 
 class Csr(ctypes.Structure):

@@ -10,7 +10,7 @@ using namespace fv;
 
 namespace {
 
-constexpr int kVersion = (1 << 16) | 0;
+constexpr int kVersion = (1 << 16) | 1;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -42,6 +42,11 @@ int validate_cfg(const fvattn_shape* s, const fvattn_route_cfg* c) {
   if (c->force_diag != 0 && c->force_diag != 1) return FVATTN_ERR_INVALID;
   if (c->force_first_frame != 0 && c->force_first_frame != 1) return FVATTN_ERR_INVALID;
   if ((c->frame_window >= 0 || c->force_first_frame) && c->frame_len == 0) return FVATTN_ERR_INVALID;
+  if (!(c->sasa_coef >= 0.f && c->sasa_coef <= 1.f) || c->sasa_trigger < 0) return FVATTN_ERR_INVALID;
+  if (c->sasa_coef > 0.f) {
+    if (c->mode == FVATTN_MODE_FRAME_TOPK) return FVATTN_ERR_UNSUPPORTED;
+    if ((s->S + kBlock - 1) / kBlock > 1280) return FVATTN_ERR_UNSUPPORTED;
+  }
   if (c->mode == FVATTN_MODE_FRAME_TOPK) {
     if (c->frame_len < kBlock || c->topk_frames < 1) return FVATTN_ERR_INVALID;
     const int64_t F = (s->S + c->frame_len - 1) / c->frame_len;
@@ -164,7 +169,8 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const 
     e = launch_pool(Q, K, 2, shape->dtype, m, 1, 0, qlo, klo, nullptr, nullptr, nsm, s);
     if (e == cudaSuccess)
       e = launch_topp(qlo, klo, reinterpret_cast<double*>(ws + L.logits), m, cfg->p >= 1.f ? 1.0 : (double)cfg->p,
-                      kblocks, scale, fc, bits, counts, out->tile_cost, s);
+                      kblocks, scale, fc, SasaCfg{cfg->sasa_coef, cfg->sasa_trigger}, bits, counts, out->tile_cost,
+                      s);
   } else {
     double* qhi = reinterpret_cast<double*>(ws + L.qhi);
     double* khi = reinterpret_cast<double*>(ws + L.khi);

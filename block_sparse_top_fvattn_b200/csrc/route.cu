@@ -546,19 +546,30 @@ __device__ void topp_select_reg(const double* __restrict__ src, int n, double p,
 // maximum (s_j - max <= 0) mapped to an unsigned integer that orders like the float; the cut
 // is the largest key T with count{key >= T} >= kk, found by bisection, then every key > T and,
 // in ascending index, as many keys == T as are needed for kk.
+// With `cand` (ceil(n/32) words, shared memory) only the blocks whose bit is set take part, and
+// w receives the chosen candidates only; kk must not exceed their number.
 template <int NE>
-__device__ void topk_select_reg(const double* __restrict__ src, int n, int kk, uint32_t* w, int lane) {
+__device__ void topk_select_reg(const double* __restrict__ src, int n, int kk, uint32_t* w, int lane,
+                                const uint32_t* cand = nullptr) {
   const int nw = (n + 31) / 32;
-  if (kk >= n) {
-    for (int q = lane; q < nw; q += 32) w[q] = range_bits(0, n - 1, q);
+  int ncand = n;
+  if (cand != nullptr) {
+    ncand = 0;
+    for (int q = lane; q < nw; q += 32) ncand += __popc(cand[q]);
+    ncand = warp_sum(ncand);
+  }
+  if (kk >= ncand) {
+    for (int q = lane; q < nw; q += 32) w[q] = cand != nullptr ? cand[q] : range_bits(0, n - 1, q);
     __syncwarp();
     return;
   }
   double s[NE];
+  bool in[NE];
 #pragma unroll
   for (int i = 0; i < NE; ++i) {
     const int j = lane + 32 * i;
     s[i] = j < n ? __ldg(src + j) : -INFINITY;
+    in[i] = j < n && (cand == nullptr || ((cand[i] >> lane) & 1u));
   }
   double mx = -INFINITY;
 #pragma unroll
@@ -568,12 +579,12 @@ __device__ void topk_select_reg(const double* __restrict__ src, int n, int kk, u
 #pragma unroll
   for (int i = 0; i < NE; ++i) {
     const uint32_t b = __float_as_uint((float)(s[i] - mx));
-    k[i] = (lane + 32 * i < n) ? ((b & 0x80000000u) ? ~b : (b | 0x80000000u)) : 0u;
+    k[i] = in[i] ? ((b & 0x80000000u) ? ~b : (b | 0x80000000u)) : 0u;
   }
   auto count_ge = [&](uint32_t t, bool strict) {
     int c = 0;
 #pragma unroll
-    for (int i = 0; i < NE; ++i) c += (lane + 32 * i < n) && (strict ? k[i] > t : k[i] >= t);
+    for (int i = 0; i < NE; ++i) c += in[i] && (strict ? k[i] > t : k[i] >= t);
     return warp_sum(c);
   };
   uint32_t lo = 0, hi = 0x80000001u;       // scores relative to the maximum are <= 0
@@ -586,9 +597,8 @@ __device__ void topk_select_reg(const double* __restrict__ src, int n, int kk, u
   int have = count_ge(T, true);
 #pragma unroll
   for (int i = 0; i < NE; ++i) {
-    const bool valid = lane + 32 * i < n;
-    uint32_t word = __ballot_sync(0xffffffffu, valid && k[i] > T);
-    uint32_t ties = __ballot_sync(0xffffffffu, valid && k[i] == T);
+    uint32_t word = __ballot_sync(0xffffffffu, in[i] && k[i] > T);
+    uint32_t ties = __ballot_sync(0xffffffffu, in[i] && k[i] == T);
     while (ties != 0u && have < kk) {
       const int b = __ffs(ties) - 1;
       ties &= ties - 1;
@@ -602,16 +612,47 @@ __device__ void topk_select_reg(const double* __restrict__ src, int n, int kk, u
 
 template <int NE>
 size_t select_smem_bytes_t(const Dims& m) {
-  return NE > 0 ? (size_t)SEL_WARPS * m.nw * 4 : (size_t)SEL_WARPS * m.nw * 32 * 8 + (size_t)SEL_WARPS * m.nw * 4;
+  return NE > 0 ? (size_t)3 * SEL_WARPS * m.nw * 4
+                : (size_t)SEL_WARPS * m.nw * 32 * 8 + (size_t)SEL_WARPS * m.nw * 4;
+}
+
+// Slack-aware augmentation of one row (FVAttn summary, section "SASA", applied to the 128-row
+// tile): the row and its partner i^1 (same tile, the neighbouring warp) step through the union
+// of their key blocks together; the row's slack is the union blocks it did not select, and
+// when the slack reaches the trigger it gains the floor(coef * slack) best of them in its own
+// routing order (the same fp32 order key as the top-k cut, ties to the lower block). Reads the
+// pre-augmentation rows in shared memory, writes the row's bitmask and count to global memory.
+template <int NE>
+__device__ void sasa_row(const double* __restrict__ src, const Dims& m, const SasaCfg& sasa, const uint32_t* ws,
+                         const uint32_t* wp, uint32_t* wc, uint32_t* wo, int lane, uint32_t* __restrict__ gbits,
+                         int32_t* __restrict__ gcount) {
+  int slack = 0, own = 0;
+  for (int q = lane; q < m.nw; q += 32) {
+    const uint32_t c = wp[q] & ~ws[q];
+    wc[q] = c;
+    slack += __popc(c);
+    own += __popc(ws[q]);
+  }
+  slack = warp_sum(slack);
+  own = warp_sum(own);
+  __syncwarp();
+  if (slack <= 0 || slack < sasa.trigger) return;
+  const int kk = (int)floor((double)sasa.coef * (double)slack);
+  if (kk <= 0) return;
+  topk_select_reg<NE>(src, m.nb, kk, wo, lane, wc);
+  for (int q = lane; q < m.nw; q += 32) gbits[q] = ws[q] | wo[q];
+  if (lane == 0) *gcount = own + kk;
 }
 
 // One warp per query block: the Top-p cut of its fp64 logit row (in registers when the row
 // has at most 32 NE blocks, else through shared memory), forced blocks, bitmask row and count;
-// warps 2w and 2w+1 hold the two rows of a 128-row tile and write its cost.
+// warps 2w and 2w+1 hold the two rows of a 128-row tile and write its cost, then (register
+// path, sasa.coef > 0) augment each other's slack.
 template <int NE>
 __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ logits, Dims m, double p,
-                                                     int kblocks, ForceCfg fc, uint32_t* __restrict__ bits,
-                                                     int32_t* __restrict__ counts, int32_t* __restrict__ tile_cost) {
+                                                     int kblocks, ForceCfg fc, SasaCfg sasa,
+                                                     uint32_t* __restrict__ bits, int32_t* __restrict__ counts,
+                                                     int32_t* __restrict__ tile_cost) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int nbp = m.nw * 32;
   uint32_t* sW = reinterpret_cast<uint32_t*>(smem_raw);                          // [warp][nw]
@@ -649,16 +690,27 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
       if (lane == 0) tile_cost[bh * m.nt + t] = c;
     }
   }
+  if constexpr (NE > 0) {
+    if (sasa.coef > 0.f && i < m.nb && (i ^ 1) < m.nb) {
+      // the rows of this CTA's tiles are final in sW; augmentation writes only wc/wo and global
+      uint32_t* wc = sW + (size_t)SEL_WARPS * m.nw + (size_t)warp * m.nw;
+      uint32_t* wo = sW + (size_t)2 * SEL_WARPS * m.nw + (size_t)warp * m.nw;
+      const int64_t grow = bh * m.nb + i;
+      sasa_row<NE>(logits + grow * (int64_t)ld, m, sasa, w, sW + (warp ^ 1) * m.nw, wc, wo, lane,
+                   bits + grow * m.nw, counts + grow);
+    }
+  }
 }
 
 template <int NE>
 static cudaError_t launch_select_t(const double* logits, const Dims& m, double p, int kblocks, const ForceCfg& fc,
-                                   uint32_t* bits, int32_t* counts, int32_t* tile_cost, cudaStream_t st) {
+                                   const SasaCfg& sasa, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
+                                   cudaStream_t st) {
   const size_t smem = select_smem_bytes_t<NE>(m) + 16;
   cudaError_t e = cudaFuncSetAttribute(select_kernel<NE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 g((m.nb + SEL_WARPS - 1) / SEL_WARPS, (unsigned)m.BH);
-  select_kernel<NE><<<g, 256, smem, st>>>(logits, m, p, kblocks, fc, bits, counts, tile_cost);
+  select_kernel<NE><<<g, 256, smem, st>>>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost);
   return cudaGetLastError();
 }
 
@@ -976,17 +1028,16 @@ cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, c
 size_t means_t_elems(const Dims& m) { return (size_t)m.BH * m.d * means_ld(m.nb); }
 
 cudaError_t launch_topp(const double* qT, const double* kT, double* logits, const Dims& m, double p, int kblocks,
-                        double scale,
-                        const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
-                        cudaStream_t st) {
+                        double scale, const ForceCfg& fc, const SasaCfg& sasa, uint32_t* bits, int32_t* counts,
+                        int32_t* tile_cost, cudaStream_t st) {
   dim3 g1((m.nb + ST - 1) / ST, (m.nb + ST - 1) / ST, (unsigned)m.BH);
   if (m.d == 128) score_kernel<128><<<g1, 256, 0, st>>>(qT, kT, m, scale, logits);
   else score_kernel<64><<<g1, 256, 0, st>>>(qT, kT, m, scale, logits);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (m.nb <= 32 * 16) return launch_select_t<16>(logits, m, p, kblocks, fc, bits, counts, tile_cost, st);
-  if (m.nb <= 32 * 40) return launch_select_t<40>(logits, m, p, kblocks, fc, bits, counts, tile_cost, st);
-  return launch_select_t<0>(logits, m, p, 0, fc, bits, counts, tile_cost, st);
+  if (m.nb <= 32 * 16) return launch_select_t<16>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost, st);
+  if (m.nb <= 32 * 40) return launch_select_t<40>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost, st);
+  return launch_select_t<0>(logits, m, p, 0, fc, SasaCfg{0.f, 0}, bits, counts, tile_cost, st);
 }
 
 cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,

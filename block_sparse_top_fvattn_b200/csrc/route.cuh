@@ -18,11 +18,16 @@ size_t schedule_smem_bytes(const Dims& m, int* groups);
 // out: 0 = means [row][d], 1 = means transposed per head [bh][d][ld], 2 = frame segment sums.
 cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int out, int frame_len,
                         double* qo, double* ko, double* qhi, double* khi, int nsm, cudaStream_t st);
+// Slack-aware augmentation of 128-row tiles (fvattn_route_cfg.sasa_coef / sasa_trigger).
+struct SasaCfg {
+  float coef;
+  int trigger;
+};
+
 // kblocks > 0: keep the kblocks highest scores per row instead of the Top-p cut.
 cudaError_t launch_topp(const double* qT, const double* kT, double* logits, const Dims& m, double p, int kblocks,
-                        double scale,
-                        const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
-                        cudaStream_t st);
+                        double scale, const ForceCfg& fc, const SasaCfg& sasa, uint32_t* bits, int32_t* counts,
+                        int32_t* tile_cost, cudaStream_t st);
 cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,
                          double* qf, double* kf, const Dims& m, int frame_len, int topk, double scale,
                          const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,

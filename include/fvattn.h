@@ -74,6 +74,16 @@ typedef struct {
  *  force_first_frame 1: the blocks of frame 0 are always kept (Sol-Attn §5.2).
  *  topk_blocks       FVATTN_MODE_TOPK_BLOCKS: key blocks kept per query block by score
  *                    (>= 1; ties go to the lower block index); at most 1280 blocks per row.
+ *  sasa_coef         slack-aware sparse augmentation (FVAttn summary, section "SASA"), in
+ *                    [0, 1]; 0 disables it. Top-p and top-k modes, at most 1280 blocks per
+ *                    row. The two query blocks 2t, 2t+1 of a 128-row attention tile step
+ *                    through the union of their key blocks together; a row's slack s is the
+ *                    number of union blocks it did not select. A row with s >= sasa_trigger
+ *                    also keeps the floor(sasa_coef * s) of those blocks that rank highest in
+ *                    its routing order (ties to the lower block index); the product is formed
+ *                    exactly from the float value. Both rows are augmented from their sets
+ *                    before augmentation, so the union (the tile's cost) does not change.
+ *  sasa_trigger      smallest slack, in key blocks, at which a row is augmented (>= 0).
  * Forced blocks are added after the cut (a union); they do not count toward p or k.
  */
 typedef struct {
@@ -86,6 +96,8 @@ typedef struct {
   int32_t frame_window;
   int32_t force_first_frame;
   int32_t topk_blocks;
+  float sasa_coef;
+  int32_t sasa_trigger;
 } fvattn_route_cfg;
 
 /*
@@ -143,8 +155,9 @@ size_t fvattn_route_workspace_bytes(const fvattn_shape* shape, const fvattn_rout
  *      fixed top-k: the same scores, the k highest per row (ties: lower j first);
  *      frame mode: frame means, frame scores, top-k frames per query frame, expanded to the
  *      key blocks that hold tokens of a kept frame;
- *   3. union with the forced blocks of cfg; CSR rows (ascending), per-head loads, tile
- *      costs and the longest-first tile order.
+ *   3. union with the forced blocks of cfg; with sasa_coef > 0, slack-aware augmentation of
+ *      each 128-row tile; CSR rows (ascending), per-head loads, tile costs and the
+ *      longest-first tile order.
  * Q, K: device [B,H,S,d]; out: caller buffers as above; workspace: device, at least
  * fvattn_route_workspace_bytes(shape, cfg) bytes, 256-byte aligned, contents need not be
  * initialised. Returns FVATTN_OK once everything is enqueued on `stream`.

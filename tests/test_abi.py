@@ -82,9 +82,22 @@ def test_invalid_shapes(lib, bad, code):
     dict(frame_window=0),                                   # neighbour frames without a frame length
     dict(mode=1, frame_len=32, topk_frames=2),              # frames shorter than a block
     dict(mode=1, frame_len=256, topk_frames=0),
+    dict(sasa_coef=-0.1), dict(sasa_coef=1.5), dict(sasa_coef=float("nan")), dict(sasa_trigger=-1),
+    dict(mode=1, frame_len=256, topk_frames=2, sasa_coef=0.5),   # frame mode has no per-block order
 ])
 def test_invalid_configs(lib, bad):
     assert lib.fvattn_route_workspace_bytes(ctypes.byref(shape()), ctypes.byref(cfg(**bad))) == 0
+
+
+def test_sasa_limits(lib):
+    # accepted in Top-p and top-k modes up to 1280 blocks per row, rejected (unsupported) above
+    ok = cfg(sasa_coef=1.0, sasa_trigger=0)
+    assert lib.fvattn_route_workspace_bytes(ctypes.byref(shape()), ctypes.byref(ok)) > 0
+    assert lib.fvattn_route_workspace_bytes(ctypes.byref(shape()), ctypes.byref(cfg(mode=2, topk_blocks=3,
+                                                                                   sasa_coef=0.5))) > 0
+    assert lib.fvattn_route_workspace_bytes(ctypes.byref(shape(S=1280 * 64)), ctypes.byref(ok)) > 0
+    assert lib.fvattn_route_workspace_bytes(ctypes.byref(shape(S=1280 * 64 + 1)), ctypes.byref(ok)) == 0
+    assert lib.fvattn_route_workspace_bytes(ctypes.byref(shape(S=1280 * 64 + 1)), ctypes.byref(cfg())) > 0
 
 
 def _fake_csr(cap):

@@ -5,6 +5,8 @@ Block selections must match bit for bit except on near-tie rows (a cumulative ma
 must be a valid selection and is then fed to the attention oracle. Attention outputs must
 be within max-abs 2e-2 and mean-abs 2e-3 of the oracle for bf16 inputs (fp32 inputs: the
 notes' own full-coverage bound, max-abs 1e-4)."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -41,7 +43,8 @@ def gpu_mask(csr) -> np.ndarray:
 def to_oracle_cfg(cfg: fv.RouteConfig) -> oracle.RouteCfg:
     return oracle.RouteCfg(mode=cfg.mode, p=cfg.p, force_diag=cfg.force_diag, local_window=cfg.local_window,
                            frame_len=cfg.frame_len, topk_frames=cfg.topk_frames, frame_window=cfg.frame_window,
-                           force_first_frame=cfg.force_first_frame, topk_blocks=cfg.topk_blocks)
+                           force_first_frame=cfg.force_first_frame, topk_blocks=cfg.topk_blocks,
+                           sasa_coef=cfg.sasa_coef, sasa_trigger=cfg.sasa_trigger)
 
 
 def check_route(q, k, cfg: fv.RouteConfig, csr=None, r=None):
@@ -164,6 +167,56 @@ def test_topk_blocks_parity(name, kw, cfg):
         assert gm.all()
     if w.dtype == "bf16":
         check_attention(q, k, v, csr, gm, 1.0 / np.sqrt(w.d))
+
+
+# Slack-aware augmentation of 128-row tiles: the GPU's base routing is checked as above; the
+# augmented sets must equal the oracle's (augmentation of the oracle's base) on every row whose
+# tile has no near-tie, and on every row be a valid augmentation of the GPU's own base sets.
+SASA_CASES = [
+    ("single", {"H": 3, "S": 3000}, fv.RouteConfig(p=0.8, sasa_coef=0.5, sasa_trigger=1)),
+    ("single", {"H": 2, "S": 8192}, fv.RouteConfig(p=0.9, sasa_coef=1.0, sasa_trigger=1)),
+    ("dit", {"H": 3, "S": 1560 * 2}, fv.RouteConfig(p=0.9, sasa_coef=0.75, sasa_trigger=2)),
+    ("single", {"H": 3, "S": 64 * 7 + 5, "d": 64}, fv.RouteConfig(p=0.7, sasa_coef=0.3, sasa_trigger=1)),
+    ("single", {"H": 3, "S": 3000}, fv.RouteConfig(mode="topk", topk_blocks=6, sasa_coef=0.5, sasa_trigger=0)),
+    ("single", {"H": 2, "S": 2048}, fv.RouteConfig(p=0.9, sasa_coef=0.5, sasa_trigger=1000)),
+    ("single", {"H": 2, "S": 64 * 40, "alpha": ("const", 0.3)}, fv.RouteConfig(p=0.6, sasa_coef=0.7)),
+]
+
+
+@pytest.mark.parametrize("name,kw,cfg", SASA_CASES)
+def test_sasa_parity(name, kw, cfg):
+    w, q, k, v = small_inputs(name, **kw)
+    B, H, S, d = q.shape
+    _, gb, _ = check_route(q, k, dataclasses.replace(cfg, sasa_coef=0.0))
+    csr = fv.route(q, k, cfg)
+    assert fv.read_status(csr) == 0
+    gm = gpu_mask(csr)
+    oc = to_oracle_cfg(cfg)
+    r = oracle.route(q.reshape(B * H, S, d), k.reshape(B * H, S, d), oc)
+    key = r["pi"] if cfg.mode == "topp" else r["scores"]
+    nb = w.nb
+    for bh in range(B * H):
+        for i in range(nb):
+            if i ^ 1 >= nb:
+                assert np.array_equal(gm[bh, i], gb[bh, i])
+            else:
+                assert oracle.valid_sasa_row(key[bh, i], gb[bh, i], gb[bh, i ^ 1], gm[bh, i], cfg.sasa_coef,
+                                             cfg.sasa_trigger, cfg.mode), (bh, i)
+    diff = np.any(gm != r["mask"], axis=2)
+    bad = diff & ~r["near_tie"]
+    assert not bad.any(), f"{int(bad.sum())} non-tie rows differ, e.g. {np.argwhere(bad)[:5].tolist()}"
+    if cfg.sasa_trigger > nb:
+        assert np.array_equal(gm, gb)
+    # the tile costs (unions) do not change; the bookkeeping follows the augmented sets
+    costs = oracle.tile_costs(gm)
+    np.testing.assert_array_equal(costs, oracle.tile_costs(gb))
+    np.testing.assert_array_equal(csr.tile_cost.cpu().numpy(), costs.reshape(-1))
+    np.testing.assert_array_equal(csr.tile_order.cpu().numpy(), oracle.lpt_order(costs))
+    np.testing.assert_array_equal(csr.head_load.cpu().numpy(), oracle.head_loads(gm))
+    rp, ci = oracle.csr_from_mask(gm)
+    np.testing.assert_array_equal(csr.row_ptr.cpu().numpy(), rp)
+    np.testing.assert_array_equal(csr.col_idx[: len(ci)].cpu().numpy(), ci)
+    check_attention(q, k, v, csr, gm, 1.0 / np.sqrt(d))
 
 
 def test_route_deterministic():
