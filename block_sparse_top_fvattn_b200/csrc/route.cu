@@ -587,11 +587,24 @@ __device__ void topk_select_reg(const double* __restrict__ src, int n, int kk, u
     for (int i = 0; i < NE; ++i) c += in[i] && (strict ? k[i] > t : k[i] >= t);
     return warp_sum(c);
   };
-  uint32_t lo = 0, hi = 0x80000001u;       // scores relative to the maximum are <= 0
+  // Bracket: count{key >= min} = every candidate >= kk, count{key >= max + 1} = 0 < kk. The search
+  // stops early once exactly kk keys are >= mid: that set is the answer (every key above the
+  // final cut plus all its ties).
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int i = 0; i < NE; ++i)
+    if (in[i]) {
+      kmin = min(kmin, k[i]);
+      kmax = max(kmax, k[i]);
+    }
+  uint32_t lo = __reduce_min_sync(0xffffffffu, kmin);
+  uint64_t hi = (uint64_t)__reduce_max_sync(0xffffffffu, kmax) + 1;
   while (hi - lo > 1) {
-    const uint32_t mid = lo + ((hi - lo) >> 1);
-    if (count_ge(mid, false) >= kk) lo = mid;
+    const uint32_t mid = (uint32_t)(lo + ((hi - lo) >> 1));
+    const int c = count_ge(mid, false);
+    if (c >= kk) lo = mid;
     else hi = mid;
+    if (c == kk) break;
   }
   const uint32_t T = lo;
   int have = count_ge(T, true);

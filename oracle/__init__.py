@@ -30,11 +30,12 @@ from .route import (RouteCfg, pool_blocks, pool_frames, block_scores, row_softma
                     valid_near_tie_set, sasa_tile_augment, sasa_near_tie_rows, valid_sasa_row)
 from .attention import attention_sets, attention_token_mask, attention_rows, selected_flops
 from .schedule import csr_from_mask, head_loads, tile_costs, lpt_order
+from .rlb import imbalance, rlb_plan
 
 __all__ = [
     "RouteCfg", "pool_blocks", "pool_frames", "block_scores", "row_softmax", "topp_row", "topk_row",
     "forced_blocks", "frame_topk_select", "route", "near_tie_rows", "valid_near_tie_set",
     "sasa_tile_augment", "sasa_near_tie_rows", "valid_sasa_row",
     "attention_sets", "attention_token_mask", "attention_rows", "selected_flops",
-    "csr_from_mask", "head_loads", "tile_costs", "lpt_order",
+    "csr_from_mask", "head_loads", "tile_costs", "lpt_order", "imbalance", "rlb_plan",
 ]

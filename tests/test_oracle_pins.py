@@ -421,3 +421,52 @@ def test_sasa_ties_go_to_lower_block_and_route_integration():
     assert np.all(base["mask"] <= aug["mask"])
     assert aug["mask"].sum() > base["mask"].sum()
     assert np.array_equal(oracle.tile_costs(aug["mask"]), oracle.tile_costs(base["mask"]))
+
+
+# ---------------------------------------------------------------- runtime load balancing (RLB)
+
+def test_rlb_golden_hand_cases():
+    cases = json.load(open(os.path.join(GOLDEN, "rlb_hand_cases.json")))["cases"]
+    for c in cases:
+        moves, L = oracle.rlb_plan(np.array(c["loads"]), c["target"], c["budget"])
+        assert [list(mv) for mv in moves] == c["moves"], c["why"]
+        assert L == c["rank_loads"], c["why"]
+
+
+def test_rlb_imbalance_definition():
+    assert oracle.imbalance([10, 10, 10]) == 1.0
+    assert oracle.imbalance([3, 1]) == 1.5                 # max / mean = 3 / 2
+    assert oracle.imbalance([0, 0]) == 1.0
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_rlb_invariants_random(seed):
+    # Every move lowers the pair's maximum, so the maximum never rises and the imbalance never
+    # grows; total load is conserved; a head moves at most once and only from its own rank; the
+    # per-rank budget holds; the plan stops at the target or when the sender has no such head.
+    rng = np.random.default_rng(seed)
+    R, Hl = int(rng.integers(2, 9)), int(rng.integers(1, 7))
+    loads = rng.integers(0, 1000, size=(R, Hl)) * (rng.random((R, Hl)) < 0.8)
+    budget = int(rng.integers(0, 3))
+    target = float(rng.choice([1.0, 1.05, 1.2]))
+    moves, L = oracle.rlb_plan(loads, target, budget)
+    cur = [int(x) for x in loads.sum(axis=1)]
+    seen = set()
+    sent = [0] * R
+    for s, h, d in moves:
+        assert (s, h) not in seen and s != d
+        seen.add((s, h))
+        w = int(loads[s, h])
+        assert cur[d] + w < cur[s]
+        before = max(cur)
+        cur[s] -= w
+        cur[d] += w
+        assert max(cur) <= before
+        sent[s] += 1
+    assert cur == L and sum(L) == int(loads.sum())
+    assert all(x <= budget for x in sent)
+    assert oracle.imbalance(L) <= oracle.imbalance(loads.sum(axis=1))
+    if moves == [] and budget > 0 and oracle.imbalance(L) > target:
+        s = max(range(R), key=lambda r: (L[r], -r))
+        d = min(range(R), key=lambda r: (L[r], r))
+        assert all(not (L[d] + int(loads[s, h]) < L[s]) for h in range(Hl))
