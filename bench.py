@@ -233,6 +233,66 @@ def run_reference(args, w):
 
 # ------------------------------------------------------------------ GPU arm
 
+def emulate_ranks(fv, q, k, v, cfg, csr, out, stream, R: int, target: float, budget: int, reps: int = 5):
+    """Runtime load balancing over R ranks, emulated on this GPU: the layer's H heads are split
+    into R contiguous groups (the heads each rank holds under sequence parallelism), the
+    migration plan is made from the routed layer's per-head loads, and the attention of each
+    rank's head set is timed on this GPU (CUDA events), before and after the plan. The step of
+    an R-GPU job waits for its slowest rank: the critical path is the maximum over ranks."""
+    import numpy as np
+    import torch
+    from block_sparse_top_fvattn_b200 import rlb
+    B, H, S, d = q.shape
+    if B != 1 or H % R:
+        return {"skipped": f"H={H} is not a multiple of {R} ranks"}
+    Hl = H // R
+    fv.route(q, k, cfg, csr=csr)
+    torch.cuda.synchronize()
+    loads = csr.head_load.cpu().numpy().reshape(R, Hl)
+    plan = rlb.make_plan(loads, target, budget)
+    full_order = csr.tile_order.clone()
+    n_all = int(csr.status[3].item())
+    owner = np.repeat(np.arange(R), Hl)
+    after = owner.copy()
+    for s_, h, dst in plan.moves:
+        after[s_ * Hl + h] = dst
+
+    def rank_ms(owners, r):
+        act = torch.tensor((owners == r).astype(np.uint8), device=q.device)
+        times = []
+        for it in range(reps + 1):
+            csr.tile_order.copy_(full_order)
+            csr.status[3].fill_(n_all)
+            fv.select_heads(csr, act)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fv.sparse_attn(q, k, v, csr, out=out)
+            b.record(stream)
+            torch.cuda.synchronize()
+            if it:
+                times.append(a.elapsed_time(b))
+        return float(np.median(times))
+
+    t_before = [rank_ms(owner, r) for r in range(R)]
+    t_after = [rank_ms(after, r) for r in range(R)]
+    csr.tile_order.copy_(full_order)
+    csr.status[3].fill_(n_all)
+    esize = q.element_size()
+    return {
+        "ranks": R, "heads_per_rank": Hl, "target_imbalance": target, "max_moves_per_rank": budget,
+        "moves": len(plan.moves), "load_imbalance_before": plan.imbalance_before,
+        "load_imbalance_after": plan.imbalance_after,
+        "rank_attn_ms_before": t_before, "rank_attn_ms_after": t_after,
+        "critical_path_ms_before": max(t_before), "critical_path_ms_after": max(t_after),
+        "time_imbalance_before": max(t_before) / (sum(t_before) / R),
+        "time_imbalance_after": max(t_after) / (sum(t_after) / R),
+        "migrated_bytes": len(plan.moves) * 4 * S * d * esize,
+        "note": "per-rank attention of each rank's head set timed on one B200; migration traffic (Q, K, V out, O "
+                "back) not included in the times",
+    }
+
+
 def run_ours(args, w):
     import numpy as np
     import torch
@@ -346,6 +406,11 @@ def run_ours(args, w):
                "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                "d2h_bytes_per_step": out.numel() * out.element_size()}
 
+    rlb_em = None
+    if args.emulate_ranks > 1 and world == 1:
+        rlb_em = emulate_ranks(fv, q, k, v, cfg, csr, out, stream, args.emulate_ranks, args.rlb_target,
+                               args.rlb_budget)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_layer, desc, threads, _ = cpu_oracle_run(w, q.cpu(), k.cpu(), v.cpu(), n_items=160)
@@ -379,6 +444,7 @@ def run_ours(args, w):
                             "frac": router_gbs / pk["hbm_gbs"], "algorithmic_bytes": rbytes,
                             "peak_kind": f"hbm copy ({pk_src})"},
         "e2e": e2e, "cpu_baseline": cpu,
+        **({"rlb_emulated": rlb_em} if rlb_em is not None else {}),
         "gpu_launches": 5 * args.steps,
         "clocks": clocks,
     }
@@ -401,6 +467,10 @@ def main():
     ap.add_argument("--topk-frames", type=int, default=4)
     ap.add_argument("--sasa-coef", type=float, default=0.0, help="tile slack augmentation coefficient (0: off)")
     ap.add_argument("--sasa-trigger", type=int, default=1)
+    ap.add_argument("--emulate-ranks", type=int, default=0,
+                    help="emulate runtime load balancing over this many ranks on one GPU (0: off)")
+    ap.add_argument("--rlb-target", type=float, default=1.05)
+    ap.add_argument("--rlb-budget", type=int, default=1, help="heads a rank may send")
     args = ap.parse_args()
     from workloads import get_workload
     w = get_workload(args.workload)

@@ -15,7 +15,7 @@ from __future__ import annotations
 
 import ctypes
 import dataclasses
-from typing import Optional
+from typing import List, Optional, Tuple
 
 import torch
 
@@ -24,7 +24,7 @@ from ._lib import (FVATTN_BF16, FVATTN_F32, FVATTN_MODE_FRAME_TOPK, FVATTN_MODE_
                    load, status_string)
 
 __all__ = ["RouteConfig", "CsrBuffers", "alloc_csr", "route", "sparse_attn", "block_means", "read_status",
-           "workspace_bytes", "shape_of", "load", "FvattnError", "status_string"]
+           "workspace_bytes", "shape_of", "load", "FvattnError", "status_string", "rlb_plan", "select_heads"]
 
 BLOCK = 64
 
@@ -182,3 +182,34 @@ def block_means(x: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> 
 def read_status(csr: CsrBuffers, stream: Optional[torch.cuda.Stream] = None) -> int:
     """Synchronise the stream and return the device status word (0 = ok)."""
     return int(load().fvattn_read_status(ctypes.byref(csr.to_c()), _stream(stream)))
+
+
+def select_heads(csr: CsrBuffers, active: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """fvattn_select_heads: restrict the next sparse_attn on `csr` to the heads bh with
+    active[bh] != 0 (active: CUDA uint8/bool tensor [B*H]). The next route on `csr` undoes it."""
+    if not active.is_cuda or active.numel() != csr.B * csr.H:
+        raise ValueError("active must be a CUDA tensor of B*H flags")
+    act = active.to(torch.uint8).contiguous()
+    shp = _lib.Shape(csr.B, csr.H, csr.S, 64, BLOCK, FVATTN_BF16, 0.0)    # only B, H, S are read
+    check(load().fvattn_select_heads(ctypes.byref(shp), ctypes.byref(csr.to_c()), act.data_ptr(), _stream(stream)),
+          "fvattn_select_heads")
+    csr._active = act                 # keep the flags alive until the kernel has run
+
+
+def rlb_plan(loads, target: float = 1.05, max_moves_per_rank: int = 1) -> Tuple[List[Tuple[int, int, int]], List[int]]:
+    """fvattn_rlb_plan on a [ranks, heads_per_rank] array of per-head loads (host). Returns the
+    moves (sender rank, sender's local head, receiver rank) in plan order and the rank loads
+    after them."""
+    import numpy as np
+    L = np.ascontiguousarray(np.asarray(loads, dtype=np.int64))
+    if L.ndim != 2:
+        raise ValueError("loads must be [ranks, heads_per_rank]")
+    R, Hl = L.shape
+    cap = max(1, R * min(max_moves_per_rank, Hl))
+    moves = np.zeros(3 * cap, dtype=np.int32)
+    rl = np.zeros(R, dtype=np.int64)
+    n = ctypes.c_int32(0)
+    check(load().fvattn_rlb_plan(L.ctypes.data, R, Hl, float(target), int(max_moves_per_rank), moves.ctypes.data, cap,
+                                 ctypes.byref(n), rl.ctypes.data), "fvattn_rlb_plan")
+    mv = moves[: 3 * n.value].reshape(-1, 3)
+    return [(int(a), int(b), int(c)) for a, b, c in mv], [int(x) for x in rl]

@@ -78,6 +78,11 @@ def load() -> ctypes.CDLL:
     lib.fvattn_read_status.argtypes = [P(Csr), vp]
     lib.fvattn_route_static_scratch.restype = ctypes.c_int
     lib.fvattn_route_static_scratch.argtypes = [vp, vp, P(Shape), P(RouteCfg), P(Csr), vp]
+    lib.fvattn_rlb_plan.restype = ctypes.c_int
+    lib.fvattn_rlb_plan.argtypes = [vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_double, ctypes.c_int32, vp,
+                                    ctypes.c_int64, P(ctypes.c_int32), vp]
+    lib.fvattn_select_heads.restype = ctypes.c_int
+    lib.fvattn_select_heads.argtypes = [P(Shape), P(Csr), vp, vp]
     _lib = lib
     return lib
 

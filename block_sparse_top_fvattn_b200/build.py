@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfvattn.so")
 
-SOURCES = ["api.cu", "route.cu", "attn_f32.cu", "attn_tc.cu", "route_static.cu"]
+SOURCES = ["api.cu", "route.cu", "attn_f32.cu", "attn_tc.cu", "route_static.cu", "balance.cu"]
 HEADERS = ["common.cuh", "route.cuh", "tc_ptx.cuh"]
 
 NVCC_FLAGS = [

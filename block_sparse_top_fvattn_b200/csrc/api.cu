@@ -202,13 +202,25 @@ int fvattn_sparse_attn(const void* Q, const void* K, const void* V, const fvattn
   cudaError_t e;
   if (shape->dtype == FVATTN_F32) {
     e = launch_attn_f32(static_cast<const float*>(Q), static_cast<const float*>(K), static_cast<const float*>(V), m,
-                        scale, csr->row_ptr, csr->col_idx, static_cast<float*>(O), lse, s);
+                        scale, csr->row_ptr, csr->col_idx, csr->tile_order, csr->status, static_cast<float*>(O),
+                        lse, s);
   } else {
     const int nsm = num_sms();
     if (nsm <= 0) return FVATTN_ERR_CUDA;
     if (cudaMemsetAsync(csr->status + 2, 0, sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
     e = launch_attn_tc(Q, K, V, m, scale, csr->row_ptr, csr->col_idx, csr->tile_order, csr->status, O, lse, nsm, s);
   }
+  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
+int fvattn_select_heads(const fvattn_shape* shape, const fvattn_csr* csr, const uint8_t* active,
+                        fvattn_stream_t stream) {
+  const int st = validate_shape(shape);
+  if (st != FVATTN_OK) return st;
+  if (!csr || !csr->tile_order || !csr->status || !active) return FVATTN_ERR_INVALID;
+  const Dims m = make_dims(*shape, 0);
+  if (m.BH * m.nt > 0x7fffffff) return FVATTN_ERR_UNSUPPORTED;
+  cudaError_t e = launch_select_heads(csr->tile_order, m, active, csr->status, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
 }
 

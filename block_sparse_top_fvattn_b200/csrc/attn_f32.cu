@@ -2,9 +2,11 @@
 //
 // Exact softmax attention of each query token over the tokens of the key blocks that the
 // router kept for its query block (FVAttn blog summary, section "AI视频生成的阿喀琉斯之踵";
-// the masked attention of the wzjinhao.cn notes §5.2). One CTA per (head, query block);
-// four threads share one query row, each owning d/4 output columns; keys are visited in
-// ascending block order with an online (running max / running sum) softmax.
+// the masked attention of the wzjinhao.cn notes §5.2). One CTA per query block of the tiles
+// in the router's tile order (the first control[3] entries: every tile, or the tiles of the
+// heads kept by fvattn_select_heads); four threads share one query row, each owning d/4
+// output columns; keys are visited in ascending block order with an online (running max /
+// running sum) softmax.
 #include <math.h>
 
 #include "common.cuh"
@@ -17,6 +19,8 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float* __restrict__
                                                        const float* __restrict__ V, Dims m, float scale,
                                                        const int32_t* __restrict__ row_ptr,
                                                        const int32_t* __restrict__ col_idx,
+                                                       const int32_t* __restrict__ tile_order,
+                                                       const int32_t* __restrict__ control,
                                                        float* __restrict__ O, float* __restrict__ lse) {
   constexpr int DQ = D / 4;
   constexpr int KCH = D == 128 ? 32 : 64;     // keys staged per step (shared memory <= 48 KB)
@@ -24,8 +28,14 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float* __restrict__
   __shared__ float sV[KCH][D];
   const int tid = threadIdx.x;
   const int r = tid >> 2, part = tid & 3;
-  const int64_t bh = blockIdx.y;
-  const int i = blockIdx.x;
+  const int64_t ntiles = m.BH * m.nt;
+  const int64_t k = blockIdx.x;
+  if (k >= imin<int64_t>(ntiles, control[3])) return;
+  const int tile = tile_order[k];
+  if (tile < 0 || tile >= ntiles) return;
+  const int64_t bh = tile / m.nt;
+  const int i = 2 * (int)(tile - bh * m.nt) + (int)blockIdx.y;
+  if (i >= m.nb) return;
   const int64_t t = (int64_t)i * kBlock + r;
   const bool valid_row = t < m.S;
   const int64_t base = bh * m.S * D;
@@ -78,13 +88,15 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float* __restrict__
 }
 
 cudaError_t launch_attn_f32(const float* Q, const float* K, const float* V, const Dims& m, float scale,
-                            const int32_t* row_ptr, const int32_t* col_idx, float* O, float* lse,
-                            cudaStream_t st) {
-  dim3 grid((unsigned)m.nb, (unsigned)m.BH);
+                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_order,
+                            const int32_t* control, float* O, float* lse, cudaStream_t st) {
+  const int64_t ntiles = m.BH * m.nt;
+  if (ntiles > 0x7fffffff) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)ntiles, 2);
   if (m.d == 128)
-    attn_f32_kernel<128><<<grid, 256, 0, st>>>(Q, K, V, m, scale, row_ptr, col_idx, O, lse);
+    attn_f32_kernel<128><<<grid, 256, 0, st>>>(Q, K, V, m, scale, row_ptr, col_idx, tile_order, control, O, lse);
   else
-    attn_f32_kernel<64><<<grid, 256, 0, st>>>(Q, K, V, m, scale, row_ptr, col_idx, O, lse);
+    attn_f32_kernel<64><<<grid, 256, 0, st>>>(Q, K, V, m, scale, row_ptr, col_idx, tile_order, control, O, lse);
   return cudaGetLastError();
 }
 

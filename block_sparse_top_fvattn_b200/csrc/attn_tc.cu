@@ -209,13 +209,16 @@ __global__ void __launch_bounds__(192, 2)
       // The record ring is deep enough that a record is never overwritten before every
       // reader has taken it: record g+NI is written only after S_{g+NI-3} was issued, which
       // follows P_{g+NI-5} of the softmax warps.
+      // Entries of the order to process: every tile, or those of the heads kept by
+      // fvattn_select_heads (control[3]).
+      const int64_t count = imin<int64_t>(ntiles, imax<int64_t>(0, *reinterpret_cast<volatile int32_t*>(&control[3])));
       uint32_t g = 0;
       for (uint32_t n = 0;; ++n) {
         const int s = n & 1;
         if (!tc::mbar_wait(&bars->sched_empty[s], ((n >> 1) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 1); break; }
         const int k = atomicAdd(&control[2], 1);
         int tile = -1;
-        if (k < ntiles) {
+        if (k < count) {
           tile = tile_order[k];
           if (tile < 0 || tile >= ntiles) { fail(bars, 11); tile = -1; }
         }

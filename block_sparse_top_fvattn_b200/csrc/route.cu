@@ -906,6 +906,7 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int32_t* __restric
     row_ptr[N] = (int32_t)carry;
     *nnz_out = carry;
     if (carry > capacity) report_error(status, FVATTN_ERR_CAPACITY, 1);
+    status[3] = (int32_t)(m.BH * m.nt);     // the attention takes every tile of the order
   }
   __syncthreads();
   for (int64_t bh = tid; bh < m.BH; bh += 1024)

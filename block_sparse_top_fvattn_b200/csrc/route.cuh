@@ -38,10 +38,14 @@ cudaError_t launch_schedule(const int32_t* counts, const int32_t* tile_cost, con
 cudaError_t launch_csr(const uint32_t* bits, const int32_t* row_ptr, const Dims& m, int32_t* col_idx,
                        int64_t capacity, int nsm, cudaStream_t st);
 
+// Compacts the tile order to the tiles of heads with active[bh] != 0 (balance.cu).
+cudaError_t launch_select_heads(int32_t* tile_order, const Dims& m, const uint8_t* active, int32_t* control,
+                                cudaStream_t st);
+
 // Attention (attn_f32.cu, attn_tc.cu).
 cudaError_t launch_attn_f32(const float* Q, const float* K, const float* V, const Dims& m, float scale,
-                            const int32_t* row_ptr, const int32_t* col_idx, float* O, float* lse,
-                            cudaStream_t st);
+                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_order,
+                            const int32_t* control, float* O, float* lse, cudaStream_t st);
 cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const Dims& m, float scale,
                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_order,
                            int32_t* control, void* O, float* lse, int nsm, cudaStream_t st);

@@ -115,7 +115,9 @@ typedef struct {
  *                                 the attention kernel's persistent CTAs take tiles.
  *  nnz        int64 [1]           total selected pairs (= row_ptr[BH*nb]).
  *  status     int32 [4]           control block: [0] device status (fvattn_status), [1] error
- *                                 detail, [2] tile ticket of the attention scheduler, [3] 0.
+ *                                 detail, [2] tile ticket of the attention scheduler, [3] number
+ *                                 of tile_order entries the attention processes (ntiles after
+ *                                 fvattn_route; fewer after fvattn_select_heads).
  */
 typedef struct {
   int32_t* row_ptr;
@@ -189,6 +191,43 @@ int fvattn_block_means(const void* X, const fvattn_shape* shape, double* out,
 /* Synchronises `stream`, then returns the device status word status[0] (FVATTN_OK or a
  * negative fvattn_status written by a kernel). FVATTN_ERR_CUDA if the copy fails. */
 int fvattn_read_status(const fvattn_csr* csr, fvattn_stream_t stream);
+
+/*
+ * fvattn_rlb_plan -- runtime load balancing of heads across ranks (FVAttn blog summary,
+ * section "RLB"), on the host; makes no CUDA call. With the per-head loads of every rank
+ * gathered (each rank's fvattn_csr.head_load: selected block pairs per head), it repeatedly
+ * takes the most loaded rank as the sender and the least loaded as the receiver and moves the
+ * sender's heaviest head whose move keeps the receiver's load below the sender's, until
+ * max / mean of the rank loads is <= target_imbalance, the sender has sent
+ * max_moves_per_rank heads, or no head of the sender qualifies. Ties go to the lower rank or
+ * head index; a head moves at most once. The plan is a pure function of its inputs, so every
+ * rank computes the same one.
+ *  loads         host int64 [ranks * heads_per_rank]: load of local head h of rank r at
+ *                r * heads_per_rank + h (0 <= load <= 2^40).
+ *  moves         host int32 [3 * moves_capacity]: (sender rank, sender's local head, receiver
+ *                rank) of each move, in plan order; moves_capacity must be at least
+ *                ranks * min(max_moves_per_rank, heads_per_rank).
+ *  n_moves       host out: number of moves written.
+ *  rank_loads    host int64 [ranks] out (may be NULL): the loads after the moves.
+ * Returns FVATTN_OK, FVATTN_ERR_INVALID (null pointer, ranks or heads_per_rank < 1, a load
+ * out of range, target_imbalance < 1 or not finite, max_moves_per_rank < 0) or
+ * FVATTN_ERR_CAPACITY (moves_capacity too small); nothing is written on error.
+ */
+int fvattn_rlb_plan(const int64_t* loads, int32_t ranks, int32_t heads_per_rank, double target_imbalance,
+                    int32_t max_moves_per_rank, int32_t* moves, int64_t moves_capacity, int32_t* n_moves,
+                    int64_t* rank_loads);
+
+/*
+ * fvattn_select_heads -- restricts the following fvattn_sparse_attn calls on `csr` to the
+ * heads bh with active[bh] != 0 (active: device uint8 [B*H]): compacts csr->tile_order in
+ * place, keeping the longest-first order of the kept tiles, and sets csr->status[3] to their
+ * number. Output rows of the other heads are left untouched. The next fvattn_route on `csr`
+ * selects every head again. Under runtime load balancing a rank skips the heads it sends to
+ * other ranks this way. One single-CTA kernel on `stream`; an entry of tile_order that is out
+ * of range is dropped and reported as FVATTN_ERR_INVALID in the device status.
+ */
+int fvattn_select_heads(const fvattn_shape* shape, const fvattn_csr* csr, const uint8_t* active,
+                        fvattn_stream_t stream);
 
 /*
  * fvattn_route_static_scratch -- fvattn_route without a caller workspace. The pages have no

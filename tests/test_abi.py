@@ -130,3 +130,43 @@ def test_attention_and_status_reject_on_host(lib):
     assert lib.fvattn_sparse_attn(P, P, P, ctypes.byref(shape(d=80)), ctypes.byref(csr), P, None, None) == -2
     assert lib.fvattn_block_means(None, ctypes.byref(s), P, None) == -1
     assert lib.fvattn_read_status(None, None) == -1
+
+
+# ---------------------------------------------------------------- runtime load balancing plan (host)
+
+@pytest.mark.parametrize("seed", range(25))
+def test_rlb_plan_matches_oracle(lib, seed):
+    import numpy as np
+    import oracle
+    import block_sparse_top_fvattn_b200 as fv
+    rng = np.random.default_rng(seed)
+    R, Hl = int(rng.integers(1, 9)), int(rng.integers(1, 9))
+    loads = rng.integers(0, 5000, size=(R, Hl)) * (rng.random((R, Hl)) < 0.85)
+    if seed % 5 == 0:
+        loads[:, :] = rng.integers(0, 3, size=(R, Hl))       # many ties
+    target = float(rng.choice([1.0, 1.02, 1.1, 1.3]))
+    budget = int(rng.integers(0, 4))
+    got = fv.rlb_plan(loads, target, budget)
+    want = oracle.rlb_plan(loads, target, budget)
+    assert got[0] == [tuple(m) for m in want[0]]
+    assert got[1] == want[1]
+
+
+def test_rlb_plan_rejects_bad_arguments(lib):
+    import numpy as np
+    loads = np.array([[5, 1], [1, 1]], dtype=np.int64)
+    moves = np.zeros(3 * 4, dtype=np.int32)
+    n = ctypes.c_int32(-7)
+
+    def call(ld=loads, R=2, Hl=2, target=1.05, budget=1, mv=moves, cap=4):
+        return lib.fvattn_rlb_plan(ld.ctypes.data if ld is not None else None, R, Hl, target, budget,
+                                   mv.ctypes.data if mv is not None else None, cap, ctypes.byref(n), None)
+
+    assert call() == 0 and n.value == 1
+    assert call(ld=None) == -1
+    assert call(R=0) == -1 and call(Hl=0) == -1
+    assert call(target=0.99) == -1 and call(target=float("nan")) == -1 and call(target=float("inf")) == -1
+    assert call(budget=-1) == -1
+    assert call(ld=np.array([[5, -1], [1, 1]], dtype=np.int64)) == -1
+    assert call(cap=1) == -3                              # needs ranks * min(budget, heads) = 2 entries
+    assert call(budget=0, cap=0, mv=None) == 0 and n.value == 0

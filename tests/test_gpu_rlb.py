@@ -1,0 +1,76 @@
+"""GPU side of runtime load balancing: fvattn_select_heads restricts the attention to a subset
+of heads (the heads a rank keeps), leaves the other heads' output rows untouched and keeps the
+longest-first order of the kept tiles; balanced_attention runs end to end on one rank."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_top_fvattn_b200 as fv
+from workloads import get_workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    fv.load()
+
+
+def _inputs(name, **kw):
+    w = get_workload(name, **kw)
+    x = make_inputs(w)
+    return w, x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+
+
+@pytest.mark.parametrize("name,kw,active", [
+    ("single", {"H": 4, "S": 2000}, [1, 0, 1, 0]),
+    ("single", {"H": 3, "S": 64 * 9 + 7, "d": 64}, [0, 0, 1]),
+    ("tiny", {}, [0, 1]),                                   # fp32 path
+    ("single", {"H": 2, "S": 1024}, [0, 0]),                # nothing kept
+])
+def test_select_heads(name, kw, active):
+    w, q, k, v = _inputs(name, **kw)
+    H = q.shape[1]
+    cfg = fv.RouteConfig(p=0.9)
+    csr = fv.route(q, k, cfg)
+    full = fv.sparse_attn(q, k, v, csr).clone()
+    assert fv.read_status(csr) == 0
+    nt = -(-w.nb // 2)
+    assert int(csr.status[3].item()) == H * nt
+    order = csr.tile_order.cpu().numpy().copy()
+    fv.select_heads(csr, torch.tensor(active, dtype=torch.uint8, device="cuda"))
+    out = torch.full_like(q, 7.0)
+    fv.sparse_attn(q, k, v, csr, out=out)
+    assert fv.read_status(csr) == 0
+    kept = [h for h in range(H) if active[h]]
+    dropped = [h for h in range(H) if not active[h]]
+    n = int(csr.status[3].item())
+    assert n == len(kept) * nt
+    want = [t for t in order if active[t // nt]]
+    np.testing.assert_array_equal(csr.tile_order[:n].cpu().numpy(), np.array(want, dtype=np.int32))
+    for h in kept:
+        assert torch.equal(out[:, h], full[:, h])           # same kernels, same tiles: bit-identical
+    for h in dropped:
+        assert bool((out[:, h] == 7.0).all())
+    fv.route(q, k, cfg, csr=csr)                            # routing again selects every head
+    torch.cuda.synchronize()
+    assert int(csr.status[3].item()) == H * nt
+
+
+def test_balanced_attention_one_rank_nccl(tmp_path):
+    import torch.distributed as dist
+    from block_sparse_top_fvattn_b200 import rlb
+    w, q, k, v = _inputs("single", H=3, S=1500)
+    dist.init_process_group("nccl", init_method=f"file://{tmp_path}/pg", rank=0, world_size=1)
+    try:
+        out, plan = rlb.balanced_attention(q, k, v, fv.RouteConfig(p=0.9), target=1.0, max_moves_per_rank=1)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    assert plan.moves == [] and plan.imbalance_before == 1.0
+    csr = fv.route(q, k, fv.RouteConfig(p=0.9))
+    ref = fv.sparse_attn(q, k, v, csr)
+    assert torch.equal(out, ref)
+    np.testing.assert_array_equal(plan.loads[0], csr.head_load.cpu().numpy())

@@ -32,7 +32,7 @@ def _worker(rank, world, port, out):
 
 def test_two_rank_reduction_gloo():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn", join=True)
     assert out[0] == (5.0, 30.0) and out[1] == (5.0, 30.0)
