@@ -24,7 +24,8 @@ from ._lib import (FVATTN_BF16, FVATTN_F32, FVATTN_MODE_FRAME_TOPK, FVATTN_MODE_
                    load, status_string)
 
 __all__ = ["RouteConfig", "CsrBuffers", "alloc_csr", "route", "sparse_attn", "block_means", "read_status",
-           "workspace_bytes", "shape_of", "load", "FvattnError", "status_string", "rlb_plan", "select_heads"]
+           "workspace_bytes", "shape_of", "load", "FvattnError", "status_string", "rlb_plan", "select_heads",
+           "LazyRouter"]
 
 BLOCK = 64
 
@@ -213,3 +214,45 @@ def rlb_plan(loads, target: float = 1.05, max_moves_per_rank: int = 1) -> Tuple[
                                  ctypes.byref(n), rl.ctypes.data), "fvattn_rlb_plan")
     mv = moves[: 3 * n.value].reshape(-1, 3)
     return [(int(a), int(b), int(c)) for a, b, c in mv], [int(x) for x in rl]
+
+
+class LazyRouter:
+    """Routing reuse across diffusion steps for one attention layer: the block selection (and
+    its tile schedule) is recomputed only every `refresh_every` steps and reused in between
+    (the video-generation acceleration notes' "lazy" mask update, e.g. every 4 diffusion
+    steps, to save the cost of generating the mask). Holds the layer's CSR and workspace.
+
+        layer = LazyRouter(RouteConfig(p=0.9), refresh_every=4)
+        for step in range(n_steps):
+            o = layer(q, k, v, step)
+    """
+
+    def __init__(self, cfg: Optional[RouteConfig] = None, refresh_every: int = 4):
+        if refresh_every < 1:
+            raise ValueError("refresh_every must be >= 1")
+        self.cfg = cfg or RouteConfig()
+        self.refresh_every = int(refresh_every)
+        self.csr: Optional[CsrBuffers] = None
+        self.workspace: Optional[torch.Tensor] = None
+        self.last_refresh: Optional[int] = None
+        self.routed = 0
+
+    def should_refresh(self, step: int, shape) -> bool:
+        if self.csr is None or self.last_refresh is None:
+            return True
+        if (self.csr.B, self.csr.H, self.csr.S) != tuple(shape[:3]):
+            return True
+        return step < self.last_refresh or step - self.last_refresh >= self.refresh_every
+
+    def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, step: int, *,
+                 out: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        if self.should_refresh(step, q.shape):
+            B, H, S, _ = q.shape
+            if self.csr is None or (self.csr.B, self.csr.H, self.csr.S) != (B, H, S):
+                self.csr = alloc_csr(B, H, S, q.device)
+                self.workspace = None
+            route(q, k, self.cfg, csr=self.csr, workspace=self.workspace, stream=stream)
+            self.workspace = self.csr._workspace
+            self.last_refresh = step
+            self.routed += 1
+        return sparse_attn(q, k, v, self.csr, out=out, stream=stream)

@@ -170,3 +170,22 @@ def test_rlb_plan_rejects_bad_arguments(lib):
     assert call(ld=np.array([[5, -1], [1, 1]], dtype=np.int64)) == -1
     assert call(cap=1) == -3                              # needs ranks * min(budget, heads) = 2 entries
     assert call(budget=0, cap=0, mv=None) == 0 and n.value == 0
+
+
+def test_lazy_router_refresh_schedule():
+    # which diffusion steps recompute the routing (no GPU needed: the schedule only)
+    import block_sparse_top_fvattn_b200 as fv
+
+    class FakeCsr:
+        B, H, S = 1, 2, 1000
+
+    lr = fv.LazyRouter(fv.RouteConfig(), refresh_every=4)
+    assert lr.should_refresh(0, (1, 2, 1000))                  # nothing routed yet
+    lr.csr, lr.last_refresh = FakeCsr(), 0
+    assert [s for s in range(1, 10) if lr.should_refresh(s, (1, 2, 1000))] == [4, 5, 6, 7, 8, 9]
+    lr.last_refresh = 4
+    assert [s for s in range(5, 13) if lr.should_refresh(s, (1, 2, 1000))] == [8, 9, 10, 11, 12]
+    assert lr.should_refresh(5, (1, 2, 2000))                  # a new shape always routes
+    assert lr.should_refresh(3, (1, 2, 1000))                  # a step before the last refresh
+    with pytest.raises(ValueError):
+        fv.LazyRouter(refresh_every=0)

@@ -74,3 +74,31 @@ def test_balanced_attention_one_rank_nccl(tmp_path):
     ref = fv.sparse_attn(q, k, v, csr)
     assert torch.equal(out, ref)
     np.testing.assert_array_equal(plan.loads[0], csr.head_load.cpu().numpy())
+
+
+def test_lazy_router_reuses_the_routing():
+    # Diffusion steps with new inputs: steps between refreshes attend with the last refresh's
+    # selection, exactly as the oracle does with that (stale) mask.
+    import oracle
+    w = get_workload("single", H=2, S=1100)
+    layer = fv.LazyRouter(fv.RouteConfig(p=0.9), refresh_every=3)
+    masks = {}
+    for step in range(5):
+        x = make_inputs(w, seed=100 + step)
+        q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+        o = layer(q, k, v, step)
+        assert fv.read_status(layer.csr) == 0
+        B, H, S, d = q.shape
+        if step % 3 == 0:
+            masks["cur"] = oracle.route(x["q"].reshape(B * H, S, d), x["k"].reshape(B * H, S, d),
+                                        oracle.RouteCfg(p=0.9))
+        r = masks["cur"]
+        assert not r["near_tie"].any()                         # these seeds have no near-tie rows
+        rp, ci = oracle.csr_from_mask(r["mask"])
+        np.testing.assert_array_equal(layer.csr.row_ptr.cpu().numpy(), rp)
+        np.testing.assert_array_equal(layer.csr.col_idx[: len(ci)].cpu().numpy(), ci)
+        ref = oracle.attention_sets(x["q"].reshape(B * H, S, d), x["k"].reshape(B * H, S, d),
+                                    x["v"].reshape(B * H, S, d), r["mask"], 1.0 / np.sqrt(d))
+        e = np.abs(o.reshape(B * H, S, d).float().cpu().numpy() - ref)
+        assert e.max() <= 2e-2 and e.mean() <= 2e-3
+    assert layer.routed == 2                                   # steps 0 and 3
