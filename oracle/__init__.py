@@ -27,15 +27,17 @@ routines (torch scaled_dot_product_attention). No function is unpinned.
 """
 from .route import (RouteCfg, pool_blocks, pool_frames, block_scores, row_softmax,
                     topp_row, topk_row, forced_blocks, frame_topk_select, route, near_tie_rows,
-                    valid_near_tie_set, sasa_tile_augment, sasa_near_tie_rows, valid_sasa_row)
-from .attention import attention_sets, attention_token_mask, attention_rows, selected_flops
+                    valid_near_tie_set, sasa_tile_augment, sasa_near_tie_rows, valid_sasa_row, frame_sets,
+                    block_forced, frame_token_mask, frame_entry_code)
+from .attention import attention_sets, attention_token_mask, attention_rows, selected_flops, attention_dense_mask
 from .schedule import csr_from_mask, head_loads, tile_costs, lpt_order
 from .rlb import imbalance, rlb_plan
 
 __all__ = [
     "RouteCfg", "pool_blocks", "pool_frames", "block_scores", "row_softmax", "topp_row", "topk_row",
     "forced_blocks", "frame_topk_select", "route", "near_tie_rows", "valid_near_tie_set",
-    "sasa_tile_augment", "sasa_near_tie_rows", "valid_sasa_row",
+    "sasa_tile_augment", "sasa_near_tie_rows", "valid_sasa_row", "frame_sets", "block_forced",
+    "frame_token_mask", "frame_entry_code", "attention_dense_mask",
     "attention_sets", "attention_token_mask", "attention_rows", "selected_flops",
     "csr_from_mask", "head_loads", "tile_costs", "lpt_order", "imbalance", "rlb_plan",
 ]

@@ -79,3 +79,17 @@ def selected_flops(mask, S: int, block: int, d: int) -> int:
     n = np.array([min(S, (j + 1) * block) - j * block for j in range(nb)], dtype=np.int64)
     pairs = np.einsum("bij,i,j->", mask.astype(np.int64), n, n)
     return int(4 * d * pairs)
+
+
+def attention_dense_mask(Q, K, V, tokmask, scale: float) -> np.ndarray:
+    """Softmax attention of every query token over the key tokens its row of `tokmask`
+    ([BH, S, S] bool) allows (the token-exact frame mode's definition). Small inputs only."""
+    Qd, Kd, Vd = _f64(Q), _f64(K), _f64(V)
+    out = np.empty_like(Qd)
+    for bh in range(Qd.shape[0]):
+        s = (Qd[bh] @ Kd[bh].T) * scale
+        s = np.where(tokmask[bh], s, -np.inf)
+        s = s - s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        out[bh] = (p / p.sum(axis=1, keepdims=True)) @ Vd[bh]
+    return out

@@ -34,6 +34,8 @@ class RouteCfg:
     sasa_coef    augmentation coefficient in [0, 1] of slack-aware sparse augmentation
                  (sasa_tile_augment); 0 disables it. Top-p and "topk" modes only.
     sasa_trigger smallest slack, in key blocks, at which a row is augmented.
+    frame_exact  frame mode: attention is token-exact (frame_token_mask) instead of over whole
+                 key blocks.
     """
     mode: str = "topp"
     p: float = 0.9
@@ -48,6 +50,7 @@ class RouteCfg:
     scale: Optional[float] = None
     sasa_coef: float = 0.0
     sasa_trigger: int = 1
+    frame_exact: bool = False
 
 
 def _f64(x) -> np.ndarray:
@@ -240,6 +243,8 @@ def route(Q, K, cfg: RouteCfg):
         qf, kf = pool_frames(Q, cfg.frame_len), pool_frames(K, cfg.frame_len)
         routed, fs, chosen = frame_topk_select(qf, kf, S, cfg, scale)
         out.update(frame_scores=fs, chosen=chosen)
+        if cfg.frame_exact:
+            out["frame_sets"] = np.stack([frame_sets(chosen[bh], cfg) for bh in range(BH)])
     else:
         raise ValueError(cfg.mode)
     out["routed"] = routed
@@ -451,3 +456,64 @@ def valid_near_tie_set(r: dict, bh: int, i: int, gpu_row: np.ndarray, S: int, cf
         must = _blocks_touching_frames(fm, inc) | forced
         may = _blocks_touching_frames(fy, inc) | forced
     return bool(np.all(gpu_row[must]) and not np.any(gpu_row & ~may))
+
+
+# ---------------------------------------------------------------- token-exact frame selection
+
+def frame_sets(chosen_bh: np.ndarray, cfg: RouteCfg) -> np.ndarray:
+    """G [F, F] bool for one head: key frames a query token of frame f may attend in the
+    token-exact frame mode: its top-k frames (Sol-Attn §2.1), the frames within +-frame_window
+    of f (§2.2, neighbouring frames) and frame 0 when force_first_frame (§5.2)."""
+    F = chosen_bh.shape[0]
+    G = chosen_bh.astype(bool).copy()
+    for f in range(F):
+        if cfg.frame_window >= 0:
+            G[f, max(0, f - cfg.frame_window):min(F - 1, f + cfg.frame_window) + 1] = True
+        if cfg.force_first_frame:
+            G[f, 0] = True
+    return G
+
+
+def block_forced(S: int, cfg: RouteCfg) -> np.ndarray:
+    """[nb, nb] bool: the block-level forced blocks (diagonal, band |i-j| <= local_window)."""
+    nb = -(-S // cfg.block)
+    out = np.zeros((nb, nb), dtype=bool)
+    for i in range(nb):
+        if cfg.force_diag:
+            out[i, i] = True
+        if cfg.local_window > 0:
+            out[i, max(0, i - cfg.local_window):min(nb - 1, i + cfg.local_window) + 1] = True
+    return out
+
+
+def frame_token_mask(G: np.ndarray, S: int, cfg: RouteCfg) -> np.ndarray:
+    """[S, S] bool for one head, token-exact frame mode: query token t may attend key token u
+    when frame(u) is in G[frame(t)], or when u's key block is a block-level forced block of t's
+    query block (those are kept whole)."""
+    fl, bs = cfg.frame_len, cfg.block
+    fr = np.arange(S) // fl
+    allowed = G[fr][:, fr]
+    bf = block_forced(S, cfg)
+    blk = np.arange(S) // bs
+    return allowed | bf[blk][:, blk]
+
+
+def frame_entry_code(G: np.ndarray, bf: np.ndarray, i: int, j: int, S: int, cfg: RouteCfg) -> int:
+    """The 32-bit code of CSR entry (query block i, key block j) in token-exact frame mode:
+    bits 0-3 allow[a][b] at bit 2a+b (a: the query block's first (0) or second (1) frame, b the
+    same for the key block; a block spans at most two frames since frames are >= 64 tokens),
+    bits 8-15 the first column of the key block's second frame (64 when it has one frame), bits
+    16-23 the first row of the query block's second frame (64 likewise). A block-level forced
+    entry allows all four."""
+    fl, bs = cfg.frame_len, cfg.block
+    qa, qb = _frames_of_block(i, S, bs, fl)
+    ka, kb = _frames_of_block(j, S, bs, fl)
+    qf, kf = (qa, qb), (ka, kb)
+    bits = 0
+    for a in range(2):
+        for b in range(2):
+            if bf[i, j] or G[qf[a], kf[b]]:
+                bits |= 1 << (2 * a + b)
+    kcol = kb * fl - j * bs if kb != ka else bs
+    qrow = qb * fl - i * bs if qb != qa else bs
+    return bits | (kcol << 8) | (qrow << 16)

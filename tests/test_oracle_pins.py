@@ -470,3 +470,82 @@ def test_rlb_invariants_random(seed):
         s = max(range(R), key=lambda r: (L[r], -r))
         d = min(range(R), key=lambda r: (L[r], r))
         assert all(not (L[d] + int(loads[s, h]) < L[s]) for h in range(Hl))
+
+
+# ---------------------------------------------------------------- token-exact frame selection
+
+def _exact_cfg(fl, **kw):
+    base = dict(mode="frame_topk", frame_len=fl, topk_frames=1, force_diag=False, frame_exact=True)
+    base.update(kw)
+    return oracle.RouteCfg(**base)
+
+
+def test_frame_exact_golden_hand_case():
+    c = json.load(open(os.path.join(GOLDEN, "frame_exact_hand_case.json")))
+    S, fl = c["S"], c["frame_len"]
+    cfg = _exact_cfg(fl)
+    G = np.array(c["G"], dtype=bool)
+    tm = oracle.frame_token_mask(G, S, cfg)
+    want = np.zeros((S, S), dtype=bool)
+    want[0:96, 0:96] = True
+    want[96:192, 192:256] = True
+    want[192:256, 96:192] = True
+    assert np.array_equal(tm, want), c["token_rule"]
+    nb = S // 64
+    support = [[j for j in range(nb) if tm[i * 64:(i + 1) * 64, j * 64:(j + 1) * 64].any()] for i in range(nb)]
+    assert support == c["block_support"]
+    bf = oracle.block_forced(S, cfg)
+    for e in c["codes"]:
+        code = oracle.frame_entry_code(G, bf, e["i"], e["j"], S, cfg)
+        assert (code & 15, (code >> 8) & 255, (code >> 16) & 255) == (e["allow"], e["kcol"], e["qrow"]), e["why"]
+
+
+@pytest.mark.parametrize("fl,seed", [(900, 0), (640, 1), (200, 2)])
+def test_frame_exact_invariants(fl, seed):
+    # The block support of the token mask is the block-granular frame selection; the entry codes
+    # expand to exactly the token mask's 64 x 64 tiles; frames that are whole blocks give the
+    # block mask itself; topk >= F allows everything.
+    rng = np.random.default_rng(seed)
+    S, d, BH = 1800, 16, 2
+    Q = rng.standard_normal((BH, S, d))
+    K = rng.standard_normal((BH, S, d))
+    cfg = _exact_cfg(fl, topk_frames=2, frame_window=0 if seed == 1 else -1, force_first_frame=seed == 2,
+                     force_diag=seed != 0, local_window=1 if seed == 2 else 0)
+    r = oracle.route(Q, K, cfg)
+    nb = -(-S // 64)
+    bf = oracle.block_forced(S, cfg)
+    for bh in range(BH):
+        tm = oracle.frame_token_mask(r["frame_sets"][bh], S, cfg)
+        for i in range(nb):
+            for j in range(nb):
+                tile = tm[i * 64:(i + 1) * 64, j * 64:(j + 1) * 64]
+                assert tile.any() == r["mask"][bh, i, j], (bh, i, j)
+                if r["mask"][bh, i, j]:
+                    code = oracle.frame_entry_code(r["frame_sets"][bh], bf, i, j, S, cfg)
+                    rows = np.arange(tile.shape[0]) >= ((code >> 16) & 255)
+                    cols = np.arange(tile.shape[1]) >= ((code >> 8) & 255)
+                    expand = (code >> (2 * rows[:, None] + cols[None, :])) & 1
+                    assert np.array_equal(expand.astype(bool), tile), (bh, i, j)
+    # frames of whole blocks: exact == block granular
+    cfg64 = _exact_cfg(640, topk_frames=2)
+    r64 = oracle.route(Q, K, cfg64)
+    tm = oracle.frame_token_mask(r64["frame_sets"][0], S, cfg64)
+    blk = np.arange(S) // 64
+    assert np.array_equal(tm, r64["mask"][0][blk][:, blk])
+    # every frame kept: dense
+    rall = oracle.route(Q, K, _exact_cfg(fl, topk_frames=99))
+    assert oracle.frame_token_mask(rall["frame_sets"][1], S, _exact_cfg(fl)).all()
+
+
+def test_attention_dense_mask_matches_sdpa():
+    rng = np.random.default_rng(5)
+    Q, K, V = (torch.from_numpy(rng.standard_normal((2, 150, 32))) for _ in range(3))
+    full = np.ones((2, 150, 150), dtype=bool)
+    out = oracle.attention_dense_mask(Q, K, V, full, 1 / math.sqrt(32))
+    ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V).numpy()
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    m = rng.random((2, 150, 150)) < 0.3
+    m[:, np.arange(150), np.arange(150)] = True
+    out = oracle.attention_dense_mask(Q, K, V, m, 0.2)
+    ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=torch.from_numpy(m), scale=0.2).numpy()
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
