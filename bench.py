@@ -46,9 +46,10 @@ def env_rank():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
 
 
-def workload_desc(w, mode: str = "topp", topk_frames: int = 4, sasa_coef: float = 0.0, sasa_trigger: int = 1) -> str:
+def workload_desc(w, mode: str = "topp", topk_frames: int = 4, sasa_coef: float = 0.0, sasa_trigger: int = 1,
+                  frame_exact: bool = False) -> str:
     sel = (f"p={w.p},diag forced" if mode == "topp" else
-           f"frame top-k={topk_frames} + frames +-1 + frame 0 + diag")
+           f"frame top-k={topk_frames} + frames +-1 + frame 0 + diag" + (", token-exact" if frame_exact else ""))
     if sasa_coef > 0:
         sel += f",tile slack augmentation coef={sasa_coef} trigger={sasa_trigger}"
     return (f"{w.name}: B={w.B},H={w.H},S={w.S} ({w.frames} frames x {w.frame_len} tokens),d={w.d},{w.dtype},"
@@ -124,6 +125,29 @@ def selected_flops_from_csr(csr, S: int, d: int):
     padded = int(counts.sum().item()) * 64 * 64
     kv_tokens = int(n[kj].sum().item())
     return 4 * d * pairs, nnz, 4 * d * padded, kv_tokens
+
+
+def selected_flops_exact(csr, S: int, d: int) -> int:
+    """4*d * the (query token, key token) pairs that token-exact frame mode attends: per CSR
+    entry, the allowed (query frame side, key frame side) quarters of the block pair, counted
+    over valid tokens only (the codes of fvattn_csr.col_code)."""
+    import torch
+    nb = csr.nb
+    rp = csr.row_ptr.long()
+    nnz = int(csr.nnz.item())
+    counts = rp[1:] - rp[:-1]
+    rows = torch.repeat_interleave(torch.arange(counts.numel(), device=rp.device), counts)
+    i = rows % nb
+    j = csr.col_idx[:nnz].long()
+    code = csr.col_code[:nnz].long()
+    nq = torch.clamp(S - 64 * i, max=64)
+    nk = torch.clamp(S - 64 * j, max=64)
+    qrow = torch.minimum((code >> 16) & 255, nq)
+    kcol = torch.minimum((code >> 8) & 255, nk)
+    rq = (qrow, nq - qrow)
+    ck = (kcol, nk - kcol)
+    pairs = sum(((code >> (2 * a + b)) & 1) * rq[a] * ck[b] for a in range(2) for b in range(2))
+    return 4 * d * int(pairs.sum().item())
 
 
 def tile_mma_flops(csr, d: int) -> int:
@@ -316,10 +340,10 @@ def run_ours(args, w):
     BH = B * H
     if args.mode == "frame_topk":
         cfg = fv.RouteConfig(mode="frame_topk", topk_frames=args.topk_frames, frame_len=w.frame_len, frame_window=1,
-                             force_first_frame=True, force_diag=True)
+                             force_first_frame=True, force_diag=True, frame_exact=args.frame_exact)
     else:
         cfg = fv.RouteConfig(p=w.p, force_diag=True, sasa_coef=args.sasa_coef, sasa_trigger=args.sasa_trigger)
-    csr = fv.alloc_csr(B, H, S, dev)
+    csr = fv.alloc_csr(B, H, S, dev, codes=cfg.frame_exact)
     ws = torch.empty(fv.workspace_bytes(q, cfg), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
@@ -334,6 +358,8 @@ def run_ours(args, w):
     if fv.read_status(csr) != 0:
         raise RuntimeError(f"device status {fv.read_status(csr)}")
     flops, nnz, flops_padded, kv_tokens = selected_flops_from_csr(csr, S, d)
+    if cfg.frame_exact:
+        flops = selected_flops_exact(csr, S, d)
     density = nnz / (BH * csr.nb * csr.nb)
     mma_flops = tile_mma_flops(csr, d)
 
@@ -429,7 +455,8 @@ def run_ours(args, w):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": workload_desc(w, args.mode, args.topk_frames, args.sasa_coef, args.sasa_trigger),
+        "config": {"workload": workload_desc(w, args.mode, args.topk_frames, args.sasa_coef, args.sasa_trigger,
+                                             args.frame_exact),
                    "l2": f"inputs larger than L2 (Q,K,V = {3 * q.numel() * q.element_size() / 1e9:.2f} GB per layer)",
                    "parallelism": f"independent layer per GPU x{world}",
                    **({"routing_refresh_every": args.refresh_every} if args.refresh_every > 1 else {})},
@@ -469,6 +496,7 @@ def main():
     ap.add_argument("--p", type=float, default=0.0, help="override the Top-p threshold")
     ap.add_argument("--mode", default="topp", choices=["topp", "frame_topk"])
     ap.add_argument("--topk-frames", type=int, default=4)
+    ap.add_argument("--frame-exact", action="store_true", help="token-exact frame mode (with --mode frame_topk)")
     ap.add_argument("--sasa-coef", type=float, default=0.0, help="tile slack augmentation coefficient (0: off)")
     ap.add_argument("--sasa-trigger", type=int, default=1)
     ap.add_argument("--refresh-every", type=int, default=1,

@@ -44,13 +44,15 @@ class RouteConfig:
     topk_blocks: int = 0
     sasa_coef: float = 0.0
     sasa_trigger: int = 1
+    frame_exact: bool = False
 
     def to_c(self) -> _lib.RouteCfg:
         mode = {"topp": FVATTN_MODE_TOPP, "frame_topk": FVATTN_MODE_FRAME_TOPK,
                 "topk": _lib.FVATTN_MODE_TOPK_BLOCKS}[self.mode]
         return _lib.RouteCfg(mode, float(self.p), int(self.force_diag), int(self.local_window), int(self.frame_len),
                              int(self.topk_frames), int(self.frame_window), int(self.force_first_frame),
-                             int(self.topk_blocks), float(self.sasa_coef), int(self.sasa_trigger))
+                             int(self.topk_blocks), float(self.sasa_coef), int(self.sasa_trigger),
+                             int(self.frame_exact))
 
 
 @dataclasses.dataclass
@@ -66,6 +68,7 @@ class CsrBuffers:
     B: int
     H: int
     S: int
+    col_code: Optional[torch.Tensor] = None   # int32 [BH*nb*nb]: per-entry token masks (frame_exact)
 
     @property
     def nb(self) -> int:
@@ -74,7 +77,8 @@ class CsrBuffers:
     def to_c(self) -> _lib.Csr:
         return _lib.Csr(self.row_ptr.data_ptr(), self.col_idx.data_ptr(), self.col_idx.numel(),
                         self.head_load.data_ptr(), self.tile_cost.data_ptr(), self.tile_order.data_ptr(),
-                        self.nnz.data_ptr(), self.status.data_ptr())
+                        self.nnz.data_ptr(), self.status.data_ptr(),
+                        self.col_code.data_ptr() if self.col_code is not None else None)
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -104,11 +108,14 @@ def _check_tensor(t: torch.Tensor, name: str) -> None:
         raise ValueError(f"{name} must be contiguous [B, H, S, d]")
 
 
-def alloc_csr(B: int, H: int, S: int, device="cuda") -> CsrBuffers:
+def alloc_csr(B: int, H: int, S: int, device="cuda", codes: bool = False) -> CsrBuffers:
+    """Router output buffers; `codes` adds the per-entry token masks that token-exact frame
+    mode (RouteConfig.frame_exact) writes and the attention applies."""
     nb = -(-S // BLOCK)
     nt = B * H * (-(-nb // 2))
     i32, i64 = torch.int32, torch.int64
     return CsrBuffers(
+        col_code=torch.empty(B * H * nb * nb, dtype=i32, device=device) if codes else None,
         row_ptr=torch.empty(B * H * nb + 1, dtype=i32, device=device),
         col_idx=torch.empty(B * H * nb * nb, dtype=i32, device=device),
         head_load=torch.empty(B * H, dtype=i64, device=device),
@@ -139,7 +146,9 @@ def route(q: torch.Tensor, k: torch.Tensor, cfg: Optional[RouteConfig] = None, *
         raise ValueError("q and k must have the same shape and dtype")
     B, H, S, _ = q.shape
     if csr is None:
-        csr = alloc_csr(B, H, S, q.device)
+        csr = alloc_csr(B, H, S, q.device, codes=cfg.frame_exact)
+    elif cfg.frame_exact and csr.col_code is None:
+        raise ValueError("token-exact frame mode needs CSR buffers with col_code (alloc_csr(..., codes=True))")
     shp = shape_of(q, scale)
     c_cfg = cfg.to_c()
     nws = workspace_bytes(q, cfg)
@@ -249,7 +258,7 @@ class LazyRouter:
         if self.should_refresh(step, q.shape):
             B, H, S, _ = q.shape
             if self.csr is None or (self.csr.B, self.csr.H, self.csr.S) != (B, H, S):
-                self.csr = alloc_csr(B, H, S, q.device)
+                self.csr = alloc_csr(B, H, S, q.device, codes=self.cfg.frame_exact)
                 self.workspace = None
             route(q, k, self.cfg, csr=self.csr, workspace=self.workspace, stream=stream)
             self.workspace = self.csr._workspace

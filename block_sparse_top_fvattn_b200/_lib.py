@@ -30,13 +30,14 @@ class RouteCfg(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("p", ctypes.c_float), ("force_diag", ctypes.c_int32),
                 ("local_window", ctypes.c_int32), ("frame_len", ctypes.c_int32), ("topk_frames", ctypes.c_int32),
                 ("frame_window", ctypes.c_int32), ("force_first_frame", ctypes.c_int32),
-                ("topk_blocks", ctypes.c_int32), ("sasa_coef", ctypes.c_float), ("sasa_trigger", ctypes.c_int32)]
+                ("topk_blocks", ctypes.c_int32), ("sasa_coef", ctypes.c_float), ("sasa_trigger", ctypes.c_int32),
+                ("frame_exact", ctypes.c_int32)]
 
 
 class Csr(ctypes.Structure):
     _fields_ = [("row_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p), ("col_capacity", ctypes.c_int64),
                 ("head_load", ctypes.c_void_p), ("tile_cost", ctypes.c_void_p), ("tile_order", ctypes.c_void_p),
-                ("nnz", ctypes.c_void_p), ("status", ctypes.c_void_p)]
+                ("nnz", ctypes.c_void_p), ("status", ctypes.c_void_p), ("col_code", ctypes.c_void_p)]
 
 
 class FvattnError(RuntimeError):

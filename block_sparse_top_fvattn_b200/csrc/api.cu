@@ -10,7 +10,7 @@ using namespace fv;
 
 namespace {
 
-constexpr int kVersion = (1 << 16) | 1;
+constexpr int kVersion = (1 << 16) | 2;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -43,6 +43,8 @@ int validate_cfg(const fvattn_shape* s, const fvattn_route_cfg* c) {
   if (c->force_first_frame != 0 && c->force_first_frame != 1) return FVATTN_ERR_INVALID;
   if ((c->frame_window >= 0 || c->force_first_frame) && c->frame_len == 0) return FVATTN_ERR_INVALID;
   if (!(c->sasa_coef >= 0.f && c->sasa_coef <= 1.f) || c->sasa_trigger < 0) return FVATTN_ERR_INVALID;
+  if (c->frame_exact != 0 && c->frame_exact != 1) return FVATTN_ERR_INVALID;
+  if (c->frame_exact && c->mode != FVATTN_MODE_FRAME_TOPK) return FVATTN_ERR_INVALID;
   if (c->sasa_coef > 0.f) {
     if (c->mode == FVATTN_MODE_FRAME_TOPK) return FVATTN_ERR_UNSUPPORTED;
     if ((s->S + kBlock - 1) / kBlock > 1280) return FVATTN_ERR_UNSUPPORTED;
@@ -56,7 +58,7 @@ int validate_cfg(const fvattn_shape* s, const fvattn_route_cfg* c) {
 }
 
 struct WsLayout {
-  size_t qlo, klo, qhi, khi, qf, kf, logits, bits, counts, total;
+  size_t qlo, klo, qhi, khi, qf, kf, fsel, logits, bits, counts, total;
 };
 
 size_t take(size_t& off, size_t bytes) {
@@ -78,6 +80,7 @@ WsLayout ws_layout(const Dims& m, int mode) {
     const size_t fm = (size_t)m.BH * m.F * m.d * sizeof(double);
     L.qf = take(off, fm);
     L.kf = take(off, fm);
+    L.fsel = take(off, (size_t)m.BH * m.F * ((m.F + 31) / 32) * sizeof(uint32_t));
   }
   if (scored) L.logits = take(off, logits_elems(m) * sizeof(double));
   L.bits = take(off, (size_t)m.BH * m.nb * m.nw * sizeof(uint32_t));
@@ -146,6 +149,7 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const 
   if (!out->row_ptr || !out->col_idx || !out->head_load || !out->tile_cost || !out->tile_order || !out->nnz ||
       !out->status)
     return FVATTN_ERR_INVALID;
+  if (cfg->frame_exact && out->col_code == nullptr) return FVATTN_ERR_INVALID;
   const Dims m = make_dims(*shape, cfg->frame_len);
   const WsLayout L = ws_layout(m, cfg->mode);
   if (workspace_bytes < L.total) return FVATTN_ERR_CAPACITY;
@@ -179,12 +183,16 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const 
     e = launch_pool(Q, K, 2, shape->dtype, m, 2, cfg->frame_len, qlo, klo, qhi, khi, nsm, s);
     if (e == cudaSuccess)
       e = launch_frame(qlo, qhi, klo, khi, qf, kf, m, cfg->frame_len, cfg->topk_frames, scale, fc, bits, counts,
-                       out->tile_cost, s);
+                       out->tile_cost, reinterpret_cast<uint32_t*>(ws + L.fsel), s);
   }
   if (e == cudaSuccess)
     e = launch_schedule(counts, out->tile_cost, m, out->row_ptr, out->head_load, out->nnz, out->tile_order,
                         out->col_capacity, out->status, s);
   if (e == cudaSuccess) e = launch_csr(bits, out->row_ptr, m, out->col_idx, out->col_capacity, nsm, s);
+  if (e == cudaSuccess && out->col_code != nullptr)
+    e = launch_codes(out->row_ptr, out->col_idx, m, cfg->frame_exact ? reinterpret_cast<const uint32_t*>(ws + L.fsel)
+                                                                     : nullptr,
+                     cfg->frame_len, fc, out->col_code, out->col_capacity, nsm, s);
   return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
 }
 
@@ -202,13 +210,14 @@ int fvattn_sparse_attn(const void* Q, const void* K, const void* V, const fvattn
   cudaError_t e;
   if (shape->dtype == FVATTN_F32) {
     e = launch_attn_f32(static_cast<const float*>(Q), static_cast<const float*>(K), static_cast<const float*>(V), m,
-                        scale, csr->row_ptr, csr->col_idx, csr->tile_order, csr->status, static_cast<float*>(O),
-                        lse, s);
+                        scale, csr->row_ptr, csr->col_idx, csr->col_code, csr->tile_order, csr->status,
+                        static_cast<float*>(O), lse, s);
   } else {
     const int nsm = num_sms();
     if (nsm <= 0) return FVATTN_ERR_CUDA;
     if (cudaMemsetAsync(csr->status + 2, 0, sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
-    e = launch_attn_tc(Q, K, V, m, scale, csr->row_ptr, csr->col_idx, csr->tile_order, csr->status, O, lse, nsm, s);
+    e = launch_attn_tc(Q, K, V, m, scale, csr->row_ptr, csr->col_idx, csr->col_code, csr->tile_order, csr->status, O,
+                       lse, nsm, s);
   }
   return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
 }

@@ -19,6 +19,7 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float* __restrict__
                                                        const float* __restrict__ V, Dims m, float scale,
                                                        const int32_t* __restrict__ row_ptr,
                                                        const int32_t* __restrict__ col_idx,
+                                                       const int32_t* __restrict__ col_code,
                                                        const int32_t* __restrict__ tile_order,
                                                        const int32_t* __restrict__ control,
                                                        float* __restrict__ O, float* __restrict__ lse) {
@@ -51,6 +52,11 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float* __restrict__
   const int e0 = row_ptr[row], e1 = row_ptr[row + 1];
   for (int e = e0; e < e1; ++e) {
     const int j = col_idx[e];
+    // token-exact frame mode: which side of the key block this row may see (col_code)
+    const int code = col_code != nullptr ? col_code[e] : kCodeAll;
+    const int side = r >= ((code >> 16) & 0xFF) ? 1 : 0;
+    const bool keep0 = (code >> (2 * side)) & 1, keep1 = (code >> (2 * side + 1)) & 1;
+    const int kcol = (code >> 8) & 0xFF;
     const int64_t k0 = (int64_t)j * kBlock;
     const int nk_blk = (int)imin<int64_t>(kBlock, m.S - k0);
     for (int c0 = 0; c0 < nk_blk; c0 += KCH) {
@@ -69,13 +75,15 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float* __restrict__
       for (int c = 0; c < DQ; ++c) s = fmaf(q[c], sK[u][part * DQ + c], s);
       s += __shfl_xor_sync(0xffffffffu, s, 1);
       s += __shfl_xor_sync(0xffffffffu, s, 2);
-      const float mn = fmaxf(mx, s);
-      const float a = expf(mx - mn);
-      const float pu = expf(s - mn);
-      l = l * a + pu;
+      if (c0 + u < kcol ? keep0 : keep1) {
+        const float mn = fmaxf(mx, s);
+        const float a = expf(mx - mn);
+        const float pu = expf(s - mn);
+        l = l * a + pu;
 #pragma unroll
-      for (int c = 0; c < DQ; ++c) o[c] = fmaf(pu, sV[u][part * DQ + c], o[c] * a);
-      mx = mn;
+        for (int c = 0; c < DQ; ++c) o[c] = fmaf(pu, sV[u][part * DQ + c], o[c] * a);
+        mx = mn;
+      }
     }
     }
   }
@@ -88,15 +96,18 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float* __restrict__
 }
 
 cudaError_t launch_attn_f32(const float* Q, const float* K, const float* V, const Dims& m, float scale,
-                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_order,
-                            const int32_t* control, float* O, float* lse, cudaStream_t st) {
+                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
+                            const int32_t* tile_order, const int32_t* control, float* O, float* lse,
+                            cudaStream_t st) {
   const int64_t ntiles = m.BH * m.nt;
   if (ntiles > 0x7fffffff) return cudaErrorInvalidValue;
   dim3 grid((unsigned)ntiles, 2);
   if (m.d == 128)
-    attn_f32_kernel<128><<<grid, 256, 0, st>>>(Q, K, V, m, scale, row_ptr, col_idx, tile_order, control, O, lse);
+    attn_f32_kernel<128><<<grid, 256, 0, st>>>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O,
+                                               lse);
   else
-    attn_f32_kernel<64><<<grid, 256, 0, st>>>(Q, K, V, m, scale, row_ptr, col_idx, tile_order, control, O, lse);
+    attn_f32_kernel<64><<<grid, 256, 0, st>>>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O,
+                                              lse);
   return cudaGetLastError();
 }
 

@@ -63,6 +63,9 @@ struct TcBars {
   uint64_t info_full[NI];
   int sched_tile[2];
   int step_info[NI];          // key block j | membership mask << 28 | last step of tile << 30
+  int step_code[NI];          // token mask of the step: allow bits of block 2t (0-3) and 2t+1 (4-7),
+                              // key-frame boundary column (8-15), query-frame boundary rows (16-23,
+                              // 24-31); see fvattn_csr.col_code
   uint32_t tmem_base;
   int abort;
 };
@@ -85,12 +88,15 @@ struct PairMerge {
     }
   }
   __device__ __forceinline__ bool more() const { return a < ae || b < be; }
-  __device__ __forceinline__ bool next(int& j, int& mask) {
+  // ea / eb: the entry of j in the two lists (-1 where the list lacks j).
+  __device__ __forceinline__ bool next(int& j, int& mask, int& ea, int& eb) {
     if (a >= ae && b >= be) return false;
     const int ja = a < ae ? ci[a] : 0x7fffffff;
     const int jb = b < be ? ci[b] : 0x7fffffff;
     j = min(ja, jb);
     mask = (ja == j ? 1 : 0) | (jb == j ? 2 : 0);
+    ea = ja == j ? a : -1;
+    eb = jb == j ? b : -1;
     a += (ja == j);
     b += (jb == j);
     return true;
@@ -150,8 +156,8 @@ __global__ void __launch_bounds__(192, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, Dims m, float scale_log2,
                    const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
-                   const int32_t* __restrict__ tile_order, int32_t* __restrict__ control,
-                   __nv_bfloat16* __restrict__ O, float* __restrict__ lse) {
+                   const int32_t* __restrict__ col_code, const int32_t* __restrict__ tile_order,
+                   int32_t* __restrict__ control, __nv_bfloat16* __restrict__ O, float* __restrict__ lse) {
   using L = TcLayout<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -234,10 +240,18 @@ __global__ void __launch_bounds__(192, 2)
             tc::tma_load_3d(sQ + c * L::kQChunk + h * L::kKVChunk, &tmQ, &bars->q_full, c * 64,
                             t * kTileRows + h * kBlock, (int)bh);
         PairMerge mg(row_ptr, col_idx, bh, t, m.nb);
-        int j, mask;
+        int j, mask, ea, eb;
         bool ok = true;
-        while (mg.next(j, mask)) {
+        while (mg.next(j, mask, ea, eb)) {
           bars->step_info[g % NI] = j | (mask << 28) | (mg.more() ? 0 : (1 << 30));
+          int code = 0xFF | (kBlock << 8) | (kBlock << 16) | (kBlock << 24);
+          if (col_code != nullptr) {
+            const int ca = ea >= 0 ? col_code[ea] : kCodeAll;
+            const int cb = eb >= 0 ? col_code[eb] : kCodeAll;
+            code = (ca & 0xF) | ((cb & 0xF) << 4) | ((((ea >= 0 ? ca : cb) >> 8) & 0xFF) << 8) |
+                   (((ca >> 16) & 0xFF) << 16) | (((cb >> 16) & 0xFF) << 24);
+          }
+          bars->step_code[g % NI] = code;
           tc::mbar_arrive(&bars->info_full[g % NI]);
           const int st = g % NS;
           if (!tc::mbar_wait(&bars->k_empty[st], ((g / NS) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 3); ok = false; break; }
@@ -261,9 +275,9 @@ __global__ void __launch_bounds__(192, 2)
         const int64_t bh = tile / m.nt;
         const int t = (int)(tile - bh * m.nt);
         PairMerge mg(row_ptr, col_idx, bh, t, m.nb);
-        int j, mask;
+        int j, mask, ea, eb;
         bool ok = true;
-        while (mg.next(j, mask)) {
+        while (mg.next(j, mask, ea, eb)) {
           const int st = g % NS;
           if (!tc::mbar_wait(&bars->v_empty[st], ((g / NS) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 16); ok = false; break; }
           tc::mbar_expect_tx(&bars->v_full[st], L::kKBytes);
@@ -370,6 +384,7 @@ __global__ void __launch_bounds__(192, 2)
         // The step record published by the loader names the key block and its row halves.
         if (!warp_wait(&bars->info_full[gi % NI], (gi / NI) & 1, abort)) { fail(bars, 14); ok = false; break; }
         const int info = bars->step_info[gi % NI];
+        const int code = bars->step_code[gi % NI];
         const int j = info & 0x0fffffff, mask = (info >> 28) & 3;
         last = (info >> 30) & 1;
         if (!warp_wait(&bars->s_full[sb], (gi >> 1) & 1, abort)) { fail(bars, 10); ok = false; break; }
@@ -390,6 +405,21 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
             for (int c = 0; c < 64; ++c)
               if (c >= nk) sraw[c] = __float_as_uint(-INFINITY);
+          }
+          // Token-exact frame mode: the keys of a frame not kept for this row's frame.
+          const int hsel = half_bit - 1;                       // 0: block 2t, 1: block 2t+1
+          const int allow = (code >> (4 * hsel)) & 0xF;        // uniform across the warp
+          if (allow != 0xF) {
+            const int side = (r & (kBlock - 1)) >= ((code >> (16 + 8 * hsel)) & 0xFF) ? 1 : 0;
+            const int kcol = (code >> 8) & 0xFF;
+            const uint64_t low = kcol >= 64 ? ~0ull : ((1ull << kcol) - 1ull);   // columns of the first frame
+            const uint64_t keep = (((allow >> (2 * side)) & 1) ? low : 0ull) | (((allow >> (2 * side + 1)) & 1) ? ~low : 0ull);
+            const uint32_t klo = (uint32_t)keep, khi = (uint32_t)(keep >> 32);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              if (!((klo >> c) & 1u)) sraw[c] = __float_as_uint(-INFINITY);
+              if (!((khi >> c) & 1u)) sraw[32 + c] = __float_as_uint(-INFINITY);
+            }
           }
           float m21[21];
 #pragma unroll
@@ -426,7 +456,10 @@ __global__ void __launch_bounds__(192, 2)
             lsum = f2(l0 * alpha, l1 * alpha);
           }
           if (raise) mrow = mx;
-          const uint64_t negm = f2(-mrow, -mrow);
+          // A row whose keys of every step so far are masked keeps mrow = -inf; its weights
+          // are exp2(-inf) = 0 against an offset of 0.
+          const float nm = mrow == -INFINITY ? 0.f : -mrow;
+          const uint64_t negm = f2(nm, nm);
           uint64_t acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
@@ -527,8 +560,9 @@ bool make_map(CUtensorMap* map, const void* base, const Dims& m) {
 
 template <int D>
 cudaError_t launch_tc_d(const void* Q, const void* K, const void* V, const Dims& m, float scale,
-                        const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_order,
-                        int32_t* control, void* O, float* lse, int nsm, cudaStream_t st) {
+                        const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
+                        const int32_t* tile_order, int32_t* control, void* O, float* lse, int nsm,
+                        cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, Q, m) || !make_map(&mk, K, m) || !make_map(&mv, V, m)) return cudaErrorInvalidValue;
   const size_t smem = TcLayout<D>::kBytes + 1024;
@@ -537,18 +571,19 @@ cudaError_t launch_tc_d(const void* Q, const void* K, const void* V, const Dims&
   const int64_t ntiles = m.BH * m.nt;
   const int grid = (int)imin<int64_t>(ntiles, (int64_t)nsm * 2);
   attn_tc_kernel<D><<<grid, 192, smem, st>>>(mq, mk, mv, m, scale * 1.4426950408889634f, row_ptr, col_idx,
-                                             tile_order, control, static_cast<__nv_bfloat16*>(O), lse);
+                                             col_code, tile_order, control, static_cast<__nv_bfloat16*>(O), lse);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const Dims& m, float scale,
-                           const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_order,
-                           int32_t* control, void* O, float* lse, int nsm, cudaStream_t st) {
+                           const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
+                           const int32_t* tile_order, int32_t* control, void* O, float* lse, int nsm,
+                           cudaStream_t st) {
   if (m.d == 128)
-    return launch_tc_d<128>(Q, K, V, m, scale, row_ptr, col_idx, tile_order, control, O, lse, nsm, st);
-  return launch_tc_d<64>(Q, K, V, m, scale, row_ptr, col_idx, tile_order, control, O, lse, nsm, st);
+    return launch_tc_d<128>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O, lse, nsm, st);
+  return launch_tc_d<64>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O, lse, nsm, st);
 }
 
 }  // namespace fv

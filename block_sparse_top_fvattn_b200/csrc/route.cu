@@ -766,7 +766,8 @@ __global__ void __launch_bounds__(256) frame_select_kernel(const double* __restr
                                                            Dims m, int frame_len, int topk, double scale,
                                                            ForceCfg fc, uint32_t* __restrict__ bits,
                                                            int32_t* __restrict__ counts,
-                                                           int32_t* __restrict__ tile_cost) {
+                                                           int32_t* __restrict__ tile_cost,
+                                                           uint32_t* __restrict__ fsel) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int F = m.F, fwords = (F + 31) / 32;
   double* sS = reinterpret_cast<double*>(smem_raw);                     // [F][F]
@@ -808,6 +809,7 @@ __global__ void __launch_bounds__(256) frame_select_kernel(const double* __restr
     }
   }
   __syncthreads();
+  for (int x = tid; x < F * fwords; x += blockDim.x) fsel[bh * F * fwords + x] = sCh[x];
 
   uint32_t* w0 = sW + warp * 2 * m.nw;
   for (int t = warp; t < m.nt; t += NWARP) {
@@ -981,6 +983,54 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int32_t* __restric
   }
 }
 
+// ------------------------------------------------------------------ token-exact frame codes
+
+// One warp per CSR row: the code of every entry (fvattn_csr.col_code). Token-exact frame mode
+// (fsel != null): a query token of frame f may attend the key tokens of the frames kept for f
+// (its top-k frames, the frames within +-frame_window, frame 0 when forced); the entry's
+// blocks span at most two frames each, so the code holds allow[a][b] for the query block's
+// frame a and the key block's frame b and the two in-block boundaries. Block-level forced
+// entries (diagonal, band) and every entry outside that mode allow the whole key block.
+__global__ void __launch_bounds__(256) code_kernel(const int32_t* __restrict__ row_ptr,
+                                                   const int32_t* __restrict__ col_idx, Dims m,
+                                                   const uint32_t* __restrict__ fsel, int frame_len, ForceCfg fc,
+                                                   int32_t* __restrict__ col_code, int64_t capacity) {
+  const int lane = threadIdx.x & 31;
+  const int64_t N = m.BH * m.nb;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int fwords = (m.F + 31) / 32;
+  for (int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < N; row += nwarps) {
+    const int64_t e0 = row_ptr[row], e1 = imin<int64_t>(row_ptr[row + 1], capacity);
+    if (fsel == nullptr) {
+      for (int64_t e = e0 + lane; e < e1; e += 32) col_code[e] = kCodeAll;
+      continue;
+    }
+    const int64_t bh = row / m.nb;
+    const int i = (int)(row - bh * m.nb);
+    const int64_t fl = frame_len;
+    const int64_t ti = (int64_t)i * kBlock;
+    const int qf0 = (int)(ti / fl), qf1 = (int)((min(m.S, ti + kBlock) - 1) / fl);
+    const int qrow = qf1 != qf0 ? (int)(qf1 * fl - ti) : kBlock;
+    const uint32_t* G = fsel + bh * m.F * fwords;
+    auto kept = [&](int f, int g) -> bool {
+      if (fc.frame_window >= 0 && g >= f - fc.frame_window && g <= f + fc.frame_window) return true;
+      if (fc.force_first && g == 0) return true;
+      return (G[f * fwords + (g >> 5)] >> (g & 31)) & 1u;
+    };
+    for (int64_t e = e0 + lane; e < e1; e += 32) {
+      const int j = col_idx[e];
+      const bool forced = (fc.force_diag && j == i) || (fc.local_window > 0 && abs(i - j) <= fc.local_window);
+      const int64_t tj = (int64_t)j * kBlock;
+      const int kf0 = (int)(tj / fl), kf1 = (int)((min(m.S, tj + kBlock) - 1) / fl);
+      const int kcol = kf1 != kf0 ? (int)(kf1 * fl - tj) : kBlock;
+      int allow = 0xF;
+      if (!forced)
+        allow = (kept(qf0, kf0) ? 1 : 0) | (kept(qf0, kf1) ? 2 : 0) | (kept(qf1, kf0) ? 4 : 0) | (kept(qf1, kf1) ? 8 : 0);
+      col_code[e] = allow | (kcol << 8) | (qrow << 16);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ K4: CSR columns
 
 __global__ void __launch_bounds__(256) csr_kernel(const uint32_t* __restrict__ bits,
@@ -1057,7 +1107,7 @@ cudaError_t launch_topp(const double* qT, const double* kT, double* logits, cons
 cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,
                          double* qf, double* kf, const Dims& m, int frame_len, int topk, double scale,
                          const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
-                         cudaStream_t st) {
+                         uint32_t* fsel, cudaStream_t st) {
   dim3 g1((unsigned)m.F, (unsigned)m.BH, 2);
   const size_t smem = frame_smem_bytes(m);
   cudaError_t e;
@@ -1066,13 +1116,13 @@ cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo
     e = cudaFuncSetAttribute(frame_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     frame_select_kernel<128><<<(unsigned)m.BH, 256, smem, st>>>(qf, kf, m, frame_len, topk, scale, fc, bits, counts,
-                                                                tile_cost);
+                                                                tile_cost, fsel);
   } else {
     frame_means_kernel<64><<<g1, 64, 0, st>>>(qlo, qhi, klo, khi, m, frame_len, qf, kf);
     e = cudaFuncSetAttribute(frame_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     frame_select_kernel<64><<<(unsigned)m.BH, 256, smem, st>>>(qf, kf, m, frame_len, topk, scale, fc, bits, counts,
-                                                               tile_cost);
+                                                               tile_cost, fsel);
   }
   return cudaGetLastError();
 }
@@ -1086,6 +1136,15 @@ cudaError_t launch_schedule(const int32_t* counts, const int32_t* tile_cost, con
   if (e != cudaSuccess) return e;
   schedule_kernel<<<1, 1024, smem, st>>>(counts, tile_cost, m, groups, row_ptr, head_load, nnz, tile_order,
                                          capacity, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_codes(const int32_t* row_ptr, const int32_t* col_idx, const Dims& m, const uint32_t* fsel,
+                         int frame_len, const ForceCfg& fc, int32_t* col_code, int64_t capacity, int nsm,
+                         cudaStream_t st) {
+  const int64_t rows = m.BH * m.nb;
+  const int grid = (int)imin<int64_t>((rows + 7) / 8, (int64_t)nsm * 8);
+  code_kernel<<<grid, 256, 0, st>>>(row_ptr, col_idx, m, fsel, frame_len, fc, col_code, capacity);
   return cudaGetLastError();
 }
 

@@ -10,6 +10,9 @@ struct ForceCfg {
   int force_diag, local_window, frame_len, frame_window, force_first;
 };
 
+// Code of an entry whose key block is attended whole (all four allow bits, no boundaries).
+constexpr int32_t kCodeAll = 0xF | (64 << 8) | (64 << 16);
+
 size_t means_t_elems(const Dims& m);     // doubles of one transposed block-mean array
 size_t logits_elems(const Dims& m);      // doubles of the fp64 block-score matrix
 size_t frame_smem_bytes(const Dims& m);
@@ -28,9 +31,15 @@ struct SasaCfg {
 cudaError_t launch_topp(const double* qT, const double* kT, double* logits, const Dims& m, double p, int kblocks,
                         double scale, const ForceCfg& fc, const SasaCfg& sasa, uint32_t* bits, int32_t* counts,
                         int32_t* tile_cost, cudaStream_t st);
+// fsel: per head, the top-k key frames of every query frame ([BH][F][ceil(F/32)] bits).
 cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,
                          double* qf, double* kf, const Dims& m, int frame_len, int topk, double scale,
                          const ForceCfg& fc, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
+                         uint32_t* fsel, cudaStream_t st);
+// Per-entry token-mask codes (fvattn_csr.col_code): token-exact frame codes from fsel, or
+// "allow all" when fsel is null.
+cudaError_t launch_codes(const int32_t* row_ptr, const int32_t* col_idx, const Dims& m, const uint32_t* fsel,
+                         int frame_len, const ForceCfg& fc, int32_t* col_code, int64_t capacity, int nsm,
                          cudaStream_t st);
 cudaError_t launch_schedule(const int32_t* counts, const int32_t* tile_cost, const Dims& m, int32_t* row_ptr,
                             int64_t* head_load, int64_t* nnz, int32_t* tile_order, int64_t capacity,
@@ -43,11 +52,14 @@ cudaError_t launch_select_heads(int32_t* tile_order, const Dims& m, const uint8_
                                 cudaStream_t st);
 
 // Attention (attn_f32.cu, attn_tc.cu).
+// col_code may be null (every entry allows its whole key block).
 cudaError_t launch_attn_f32(const float* Q, const float* K, const float* V, const Dims& m, float scale,
-                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_order,
-                            const int32_t* control, float* O, float* lse, cudaStream_t st);
+                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
+                            const int32_t* tile_order, const int32_t* control, float* O, float* lse,
+                            cudaStream_t st);
 cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const Dims& m, float scale,
-                           const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_order,
-                           int32_t* control, void* O, float* lse, int nsm, cudaStream_t st);
+                           const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
+                           const int32_t* tile_order, int32_t* control, void* O, float* lse, int nsm,
+                           cudaStream_t st);
 
 }  // namespace fv

@@ -37,7 +37,7 @@ class Kernels:
 
     def route(self, q: torch.Tensor, k: torch.Tensor):
         B, H, S, _ = q.shape
-        return route(q, k, self.cfg, csr=alloc_csr(B, H, S, q.device))
+        return route(q, k, self.cfg, csr=alloc_csr(B, H, S, q.device, codes=self.cfg.frame_exact))
 
     @staticmethod
     def head_load(state) -> torch.Tensor:

@@ -84,6 +84,13 @@ typedef struct {
  *                    exactly from the float value. Both rows are augmented from their sets
  *                    before augmentation, so the union (the tile's cost) does not change.
  *  sasa_trigger      smallest slack, in key blocks, at which a row is augmented (>= 0).
+ *  frame_exact       frame mode only, 0 or 1. 1: token-exact attention (Sol-Attn's semantics,
+ *                    vLLM-Omni article §2.1-§2.2): a query token of frame f attends exactly the
+ *                    key tokens of the frames kept for f (its top-k frames, the frames within
+ *                    +-frame_window of f, frame 0 when force_first_frame), plus the whole of
+ *                    its block-level forced blocks (diagonal, band). The CSR rows are the same
+ *                    as with 0; each entry also gets a code in fvattn_csr.col_code, which must
+ *                    then be non-NULL. With 0 a kept key block is attended whole.
  * Forced blocks are added after the cut (a union); they do not count toward p or k.
  */
 typedef struct {
@@ -98,6 +105,7 @@ typedef struct {
   int32_t topk_blocks;
   float sasa_coef;
   int32_t sasa_trigger;
+  int32_t frame_exact;
 } fvattn_route_cfg;
 
 /*
@@ -118,6 +126,15 @@ typedef struct {
  *                                 detail, [2] tile ticket of the attention scheduler, [3] number
  *                                 of tile_order entries the attention processes (ntiles after
  *                                 fvattn_route; fewer after fvattn_select_heads).
+ *  col_code   int32 [col_capacity] or NULL: per-entry token mask of the key block, written by
+ *                                 fvattn_route when non-NULL and applied by fvattn_sparse_attn.
+ *                                 Bits 0-3: allow[a][b] at bit 2a+b, a = the query block's
+ *                                 first (0) or second (1) frame, b the same for the key block
+ *                                 (a 64-token block spans at most two frames of >= 64 tokens);
+ *                                 bits 8-15: first column of the key block's second frame, bits
+ *                                 16-23: first row of the query block's second frame (64 when the
+ *                                 block lies in one frame). Outside token-exact frame mode every
+ *                                 entry allows all (0x40400F).
  */
 typedef struct {
   int32_t* row_ptr;
@@ -128,6 +145,7 @@ typedef struct {
   int32_t* tile_order;
   int64_t* nnz;
   int32_t* status;
+  int32_t* col_code;
 } fvattn_csr;
 
 /* Library version, (major << 16) | minor. */

@@ -84,6 +84,8 @@ def test_invalid_shapes(lib, bad, code):
     dict(mode=1, frame_len=256, topk_frames=0),
     dict(sasa_coef=-0.1), dict(sasa_coef=1.5), dict(sasa_coef=float("nan")), dict(sasa_trigger=-1),
     dict(mode=1, frame_len=256, topk_frames=2, sasa_coef=0.5),   # frame mode has no per-block order
+    dict(frame_exact=1),                                          # token-exact needs frame mode
+    dict(mode=1, frame_len=256, topk_frames=2, frame_exact=2),
 ])
 def test_invalid_configs(lib, bad):
     assert lib.fvattn_route_workspace_bytes(ctypes.byref(shape()), ctypes.byref(cfg(**bad))) == 0
@@ -117,6 +119,10 @@ def test_route_rejects_on_host_before_any_launch(lib):
     assert lib.fvattn_route(P, P, ctypes.byref(s), ctypes.byref(c), ctypes.byref(small), P, ws, None) == -3
     bad = cfg(p=0.0)
     assert lib.fvattn_route(P, P, ctypes.byref(s), ctypes.byref(bad), ctypes.byref(csr), P, ws, None) == -1
+    exact = cfg(mode=1, frame_len=256, topk_frames=2, frame_exact=1)       # col_code is NULL in csr
+    ws_e = lib.fvattn_route_workspace_bytes(ctypes.byref(s), ctypes.byref(exact))
+    assert ws_e > 0
+    assert lib.fvattn_route(P, P, ctypes.byref(s), ctypes.byref(exact), ctypes.byref(csr), P, ws_e, None) == -1
     assert lib.fvattn_route(P, P, ctypes.byref(shape(block=32)), ctypes.byref(c), ctypes.byref(csr), P, ws,
                             None) == -2
 

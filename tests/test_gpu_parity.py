@@ -44,7 +44,7 @@ def to_oracle_cfg(cfg: fv.RouteConfig) -> oracle.RouteCfg:
     return oracle.RouteCfg(mode=cfg.mode, p=cfg.p, force_diag=cfg.force_diag, local_window=cfg.local_window,
                            frame_len=cfg.frame_len, topk_frames=cfg.topk_frames, frame_window=cfg.frame_window,
                            force_first_frame=cfg.force_first_frame, topk_blocks=cfg.topk_blocks,
-                           sasa_coef=cfg.sasa_coef, sasa_trigger=cfg.sasa_trigger)
+                           sasa_coef=cfg.sasa_coef, sasa_trigger=cfg.sasa_trigger, frame_exact=cfg.frame_exact)
 
 
 def check_route(q, k, cfg: fv.RouteConfig, csr=None, r=None):
@@ -217,6 +217,44 @@ def test_sasa_parity(name, kw, cfg):
     np.testing.assert_array_equal(csr.row_ptr.cpu().numpy(), rp)
     np.testing.assert_array_equal(csr.col_idx[: len(ci)].cpu().numpy(), ci)
     check_attention(q, k, v, csr, gm, 1.0 / np.sqrt(d))
+
+
+# Token-exact frame mode: the same CSR as the block-granular frame mode, per-entry codes equal to
+# the oracle's, and attention against the oracle's dense token mask.
+EXACT_CASES = [
+    ("single", {"H": 2, "S": 3000, "frame_len": 900}, dict(topk_frames=2, frame_window=-1, force_first_frame=False)),
+    ("dit", {"H": 2, "S": 1560 * 2}, dict(topk_frames=1, frame_window=0, force_first_frame=True)),
+    ("single", {"H": 3, "S": 64 * 20 + 9, "d": 64, "frame_len": 200}, dict(topk_frames=1, frame_window=-1,
+                                                                         force_first_frame=False, local_window=1)),
+    ("tiny", {"frame_len": 200}, dict(topk_frames=2, frame_window=-1, force_first_frame=True)),   # fp32 path
+]
+
+
+@pytest.mark.parametrize("name,kw,extra", EXACT_CASES)
+def test_frame_exact_parity(name, kw, extra):
+    w, q, k, v = small_inputs(name, **kw)
+    B, H, S, d = q.shape
+    force_diag = extra.pop("force_diag", True)
+    cfg = fv.RouteConfig(mode="frame_topk", frame_len=w.frame_len, frame_exact=True, force_diag=force_diag, **extra)
+    csr, gm, r = check_route(q, k, cfg, csr=fv.alloc_csr(B, H, S, q.device, codes=True))
+    assert not r["near_tie"].any()                      # these cases have no near-tie frames
+    oc = to_oracle_cfg(cfg)
+    bf = oracle.block_forced(S, oc)
+    rp, ci = oracle.csr_from_mask(r["mask"])
+    want = np.array([oracle.frame_entry_code(r["frame_sets"][row // (w.nb)], bf, row % w.nb, int(ci[e]), S, oc)
+                     for row in range(B * H * w.nb) for e in range(rp[row], rp[row + 1])], dtype=np.int64)
+    np.testing.assert_array_equal(csr.col_code[: len(ci)].cpu().numpy().astype(np.int64), want)
+    o = fv.sparse_attn(q, k, v, csr)
+    assert fv.read_status(csr) == 0
+    Q, K, V = (t.reshape(B * H, S, d).cpu() for t in (q, k, v))
+    tok = np.stack([oracle.frame_token_mask(r["frame_sets"][bh], S, oc) for bh in range(B * H)])
+    ref = oracle.attention_dense_mask(Q, K, V, tok, 1.0 / np.sqrt(d))
+    e = np.abs(o.reshape(B * H, S, d).float().cpu().numpy() - ref)
+    lim = (MAX_ABS_F32, MAX_ABS_F32) if w.dtype == "f32" else (MAX_ABS_BF16, MEAN_ABS_BF16)
+    assert e.max() <= lim[0] and e.mean() <= lim[1], (e.max(), e.mean())
+    # the block-granular answer differs where a kept block straddles a frame that is not kept
+    blk = np.stack([np.repeat(np.repeat(r["mask"][bh], 64, 0), 64, 1)[:S, :S] for bh in range(B * H)])
+    assert (blk & ~tok).any()
 
 
 def test_route_deterministic():
