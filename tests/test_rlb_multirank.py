@@ -80,3 +80,38 @@ def test_balanced_attention_gloo(world):
         assert mv == moves                         # every rank computed the same plan
     assert len(moves) > 0 and all(s == 0 for s, _, _ in moves[:1])   # the heavy rank sends first
     assert out[0][3] < out[0][2]                  # the imbalance went down
+
+
+def _ulysses_worker(rank, world, port, balance, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from block_sparse_top_fvattn_b200 import ulysses
+        from workloads import get_workload, make_inputs
+        # one global layer (the same draw on every rank), sequence-sharded across the ranks
+        w = get_workload("tiny", H=2 * world, S=256 * world, alpha=("uniform", 0.0, 3.0), seed=21)
+        x = make_inputs(w)
+        Sl = w.S // world
+        shard = [t[:, :, rank * Sl:(rank + 1) * Sl].contiguous() for t in (x["q"], x["k"], x["v"])]
+        kern = OracleKernels(0.9)
+        o, plan = ulysses.ulysses_attention(*shard, group=None, balance=balance, target=1.0,
+                                            max_moves_per_rank=1, kernels=kern)
+        ref = torch.empty_like(x["q"])
+        kern.attend(x["q"], x["k"], x["v"], kern.route(x["q"], x["k"]), None, ref)
+        out[rank] = float((o - ref[:, :, rank * Sl:(rank + 1) * Sl]).abs().max())
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,balance", [(2, False), (2, True), (3, True)])
+def test_ulysses_attention_gloo(world, balance):
+    # sequence -> heads all-to-all, routing and attention of the local heads (with head migration
+    # when balance), heads -> sequence: each rank's output slice equals the single-process
+    # oracle attention of the whole layer
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_ulysses_worker, args=(world, _free_port(), balance, out), nprocs=world,
+                       start_method="spawn", join=True)
+    for r in range(world):
+        assert out[r] == 0.0, (r, out[r])
