@@ -58,7 +58,7 @@ int validate_cfg(const fvattn_shape* s, const fvattn_route_cfg* c) {
 }
 
 struct WsLayout {
-  size_t qlo, klo, qhi, khi, qf, kf, fsel, logits, bits, counts, total;
+  size_t qlo, klo, qhi, khi, qf, kf, fsel, qs, ks, eq, ek, logits, bits, counts, total;
 };
 
 size_t take(size_t& off, size_t bytes) {
@@ -71,9 +71,17 @@ WsLayout ws_layout(const Dims& m, int mode) {
   WsLayout L{};
   size_t off = 0;
   const bool scored = mode == FVATTN_MODE_TOPP || mode == FVATTN_MODE_TOPK_BLOCKS;
-  const size_t means = (scored ? means_t_elems(m) : (size_t)m.BH * m.nb * m.d) * sizeof(double);
-  L.qlo = take(off, means);
-  L.klo = take(off, means);
+  const size_t means = (size_t)m.BH * m.nb * m.d * sizeof(double);
+  if (scored) {
+    const size_t slices = (size_t)m.BH * kScoreSlices * m.nb * m.d * sizeof(__nv_bfloat16);
+    L.qs = take(off, slices);
+    L.ks = take(off, slices);
+    L.eq = take(off, (size_t)m.BH * m.nb * sizeof(int32_t));
+    L.ek = take(off, (size_t)m.BH * m.nb * sizeof(int32_t));
+  } else {
+    L.qlo = take(off, means);
+    L.klo = take(off, means);
+  }
   if (mode == FVATTN_MODE_FRAME_TOPK) {
     L.qhi = take(off, means);
     L.khi = take(off, means);
@@ -170,17 +178,19 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const 
   cudaError_t e;
   if (cfg->mode == FVATTN_MODE_TOPP || cfg->mode == FVATTN_MODE_TOPK_BLOCKS) {
     const int kblocks = cfg->mode == FVATTN_MODE_TOPK_BLOCKS ? cfg->topk_blocks : 0;
-    e = launch_pool(Q, K, 2, shape->dtype, m, 1, 0, qlo, klo, nullptr, nullptr, nsm, s);
+    const SliceOut so{reinterpret_cast<__nv_bfloat16*>(ws + L.qs), reinterpret_cast<__nv_bfloat16*>(ws + L.ks),
+                      reinterpret_cast<int32_t*>(ws + L.eq), reinterpret_cast<int32_t*>(ws + L.ek)};
+    e = launch_pool(Q, K, 2, shape->dtype, m, 1, 0, nullptr, nullptr, nullptr, nullptr, so, nsm, s);
     if (e == cudaSuccess)
-      e = launch_topp(qlo, klo, reinterpret_cast<double*>(ws + L.logits), m, cfg->p >= 1.f ? 1.0 : (double)cfg->p,
-                      kblocks, scale, fc, SasaCfg{cfg->sasa_coef, cfg->sasa_trigger}, bits, counts, out->tile_cost,
-                      s);
+      e = launch_topp(so, reinterpret_cast<double*>(ws + L.logits), m, cfg->p >= 1.f ? 1.0 : (double)cfg->p, kblocks,
+                      scale, fc, SasaCfg{cfg->sasa_coef, cfg->sasa_trigger}, bits, counts, out->tile_cost,
+                      out->status, s);
   } else {
     double* qhi = reinterpret_cast<double*>(ws + L.qhi);
     double* khi = reinterpret_cast<double*>(ws + L.khi);
     double* qf = reinterpret_cast<double*>(ws + L.qf);
     double* kf = reinterpret_cast<double*>(ws + L.kf);
-    e = launch_pool(Q, K, 2, shape->dtype, m, 2, cfg->frame_len, qlo, klo, qhi, khi, nsm, s);
+    e = launch_pool(Q, K, 2, shape->dtype, m, 2, cfg->frame_len, qlo, klo, qhi, khi, SliceOut{}, nsm, s);
     if (e == cudaSuccess)
       e = launch_frame(qlo, qhi, klo, khi, qf, kf, m, cfg->frame_len, cfg->topk_frames, scale, fc, bits, counts,
                        out->tile_cost, reinterpret_cast<uint32_t*>(ws + L.fsel), s);
@@ -240,7 +250,7 @@ int fvattn_block_means(const void* X, const fvattn_shape* shape, double* out, fv
   const Dims m = make_dims(*shape, 0);
   const int nsm = num_sms();
   if (nsm <= 0) return FVATTN_ERR_CUDA;
-  cudaError_t e = launch_pool(X, nullptr, 1, shape->dtype, m, 0, 0, out, nullptr, nullptr, nullptr, nsm,
+  cudaError_t e = launch_pool(X, nullptr, 1, shape->dtype, m, 0, 0, out, nullptr, nullptr, nullptr, SliceOut{}, nsm,
                               reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
 }

@@ -26,6 +26,7 @@
 #include "common.cuh"
 #include "route.cuh"
 #include "tc_ptx.cuh"
+#include "tmap.cuh"
 
 namespace fv {
 
@@ -528,34 +529,10 @@ __global__ void __launch_bounds__(192, 2)
   if (threadIdx.x == 0 && bars->abort) report_error(control, FVATTN_ERR_TIMEOUT, bars->abort);
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
 // [BH, S, d] bf16 viewed as a 3-D tensor (d innermost); 64 x 64 boxes with the 128-byte
 // swizzle; rows past S read as zeros and never reach the next head.
 bool make_map(CUtensorMap* map, const void* base, const Dims& m) {
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)m.d, (cuuint64_t)m.S, (cuuint64_t)m.BH};
-  cuuint64_t strides[2] = {(cuuint64_t)m.d * 2, (cuuint64_t)m.S * (cuuint64_t)m.d * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)kBlock, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return make_map_bf16_3d(map, base, (uint64_t)m.d, (uint64_t)m.S, (uint64_t)m.BH, (uint32_t)kBlock);
 }
 
 template <int D>

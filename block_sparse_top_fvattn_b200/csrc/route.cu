@@ -69,13 +69,14 @@ __device__ __forceinline__ void unpack(const uint4& v, double (&o)[4], const flo
   o[3] = __uint_as_float(v.w);
 }
 
-enum PoolOut { kMeans = 0, kMeansT = 1, kFrameSums = 2 };
+enum PoolOut { kMeans = 0, kSliced = 1, kFrameSums = 2 };
 
 template <typename T, int D, int OUT>
 __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ Q, const T* __restrict__ K,
-                                                   int ntensors, Dims m, int frame_len, int ld,
+                                                   int ntensors, Dims m, int frame_len,
                                                    double* __restrict__ qo, double* __restrict__ ko,
-                                                   double* __restrict__ qhi, double* __restrict__ khi) {
+                                                   double* __restrict__ qhi, double* __restrict__ khi,
+                                                   SliceOut so) {
   using AccT = typename Acc<T>::type;
   constexpr int VEC = Acc<T>::kVec;
   constexpr int CPR = D / VEC;         // 16-byte vectors per row
@@ -139,15 +140,48 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ Q, cons
         lo[e] += __shfl_xor_sync(0xffffffffu, lo[e], off);
         if (FRAME) hi[e] += __shfl_xor_sync(0xffffffffu, hi[e], off);
       }
-    if (r0 == 0) {
+    if (OUT == kSliced) {
+      // The mean as a power-of-two scale 2^ex (max|x| < 2^ex) and kScoreSlices base-256 digits
+      // in [-128, 128] (exact in bf16): N = rint(x 2^(39-ex)), |N| < 2^39, written as
+      // N = X_0 2^32 + X_1 2^24 + X_2 2^16 + X_3 2^8 + X_4, i.e. x ~ 2^ex sum_a X_a 2^(-7-8a), by
+      // integer shifts (digits rounded half up from the top).
+      double r[VEC], mx = 0.0;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        r[e] = lo[e] / (double)nvalid;
+        mx = fmax(mx, fabs(r[e]));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      // ex = floor(log2(mx)) + 1 from the exponent field; means below 2^-900 count as 0
+      const int ex = max(-900, mx > 0.0 ? (int)((__double_as_longlong(mx) >> 52) & 0x7ff) - 1022 : 0);
+      if (r0 == 0) {
+        __nv_bfloat16* dst = (isK ? so.ks : so.qs) + ((bh * kScoreSlices) * m.nb + blk) * (int64_t)D + c * VEC;
+        const double sc = __longlong_as_double((int64_t)(1023 + 39 - ex) << 52);   // 2^(39-ex)
+        long long n[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) n[e] = __double2ll_rn(r[e] * sc);
+#pragma unroll
+        for (int a = 0; a < kScoreSlices; ++a) {
+          const int sh = 8 * (kScoreSlices - 1 - a);
+          __nv_bfloat16 h[VEC];
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) {
+            const long long x = sh ? (n[e] + (1ll << (sh - 1))) >> sh : n[e];
+            n[e] -= x << sh;
+            h[e] = __int2bfloat16_rn((int)x);
+          }
+          __nv_bfloat16* d = dst + (int64_t)a * m.nb * D;
+          if (VEC == 8) *reinterpret_cast<uint4*>(d) = *reinterpret_cast<const uint4*>(h);
+          else *reinterpret_cast<uint2*>(d) = *reinterpret_cast<const uint2*>(h);
+        }
+        if (c == 0) (isK ? so.ek : so.eq)[row] = ex;
+      }
+    } else if (r0 == 0) {
       double* o = isK ? ko : qo;
       if (OUT == kMeans) {
 #pragma unroll
         for (int e = 0; e < VEC; ++e) o[row * D + c * VEC + e] = lo[e] / (double)nvalid;
-      } else if (OUT == kMeansT) {
-        double* ot = o + bh * (int64_t)D * ld + blk;
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) ot[(int64_t)(c * VEC + e) * ld] = lo[e] / (double)nvalid;
       } else {
         double* oh = isK ? khi : qhi;
 #pragma unroll
@@ -332,94 +366,7 @@ __device__ void topp_select(double* E, int n, double p, uint32_t* w, int lane) {
   __syncwarp();
 }
 
-// Transposed block means are stored with a row stride of nb rounded up to 32.
-__host__ __device__ __forceinline__ int means_ld(int nb) { return (nb + 31) & ~31; }
-
 size_t logits_elems(const Dims& m) { return (size_t)m.BH * m.nb * means_ld(m.nb); }
-
-constexpr int ST = 64;      // score GEMM output tile: 64 query blocks x 64 key blocks
-constexpr int SKC = 16;     // head-dim depth of one pipelined operand chunk
-constexpr int SNS = 3;      // pipeline stages
-
-__device__ __forceinline__ void cp_async_wait2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
-
-// Sc[bh][i][j] = <qbar_i, kbar_j> * scale in fp64 for all i, j < nb, written row-major with row
-// stride ld. One 64 x 64 tile per CTA; warps in a 4 x 2 grid of 16 rows x 32 keys; each lane
-// 4 rows (lm * 4 ..) by 4 keys (2 ln, 2 ln + 1, 16 + 2 ln, 17 + 2 ln), so that every shared
-// load of an operand is a single wavefront. Operands stream from the transposed block means
-// [bh][d][ld] through a 3-stage cp.async ring of 16-deep head-dim chunks. FMAs accumulate in
-// ascending head-dim order.
-template <int D>
-__global__ void __launch_bounds__(256) score_kernel(const double* __restrict__ qT, const double* __restrict__ kT,
-                                                    Dims m, double scale, double* __restrict__ logits) {
-  __shared__ __align__(16) double sA[SNS][SKC][ST];
-  __shared__ __align__(16) double sB[SNS][SKC][ST];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wr = warp >> 1, wc = warp & 1;
-  const int lm = lane >> 3, ln = lane & 7;
-  const int64_t bh = blockIdx.z;
-  const int i0 = blockIdx.y * ST, j0 = blockIdx.x * ST;
-  const int ld = means_ld(m.nb);
-  const double* qh = qT + bh * (int64_t)D * ld;
-  const double* kh = kT + bh * (int64_t)D * ld;
-  constexpr int NCH = D / SKC;
-
-  auto issue = [&](int ch) {
-    const int st = ch % SNS, k0 = ch * SKC;
-    for (int x = tid; x < SKC * ST / 2; x += 256) {
-      const int kk = x / (ST / 2), c = (x % (ST / 2)) * 2;
-      const int i = i0 + c, j = j0 + c;
-      const int vi = imax(0, imin(2, m.nb - i)), vj = imax(0, imin(2, m.nb - j));
-      cp_async16(&sA[st][kk][c], qh + (int64_t)(k0 + kk) * ld + (vi ? i : 0), vi * 8);
-      cp_async16(&sB[st][kk][c], kh + (int64_t)(k0 + kk) * ld + (vj ? j : 0), vj * 8);
-    }
-    cp_async_commit();
-  };
-
-  double acc[4][4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) acc[r][c] = 0.0;
-  issue(0);
-  issue(1);
-  for (int ch = 0; ch < NCH; ++ch) {
-    if (ch + 2 < NCH) issue(ch + 2);
-    else cp_async_commit();
-    cp_async_wait2();
-    __syncthreads();
-    const int st = ch % SNS;
-#pragma unroll
-    for (int kk = 0; kk < SKC; ++kk) {
-      const double2 a01 = *reinterpret_cast<const double2*>(&sA[st][kk][wr * 16 + lm * 4]);
-      const double2 a23 = *reinterpret_cast<const double2*>(&sA[st][kk][wr * 16 + lm * 4 + 2]);
-      const double2 b01 = *reinterpret_cast<const double2*>(&sB[st][kk][wc * 32 + ln * 2]);
-      const double2 b23 = *reinterpret_cast<const double2*>(&sB[st][kk][wc * 32 + 16 + ln * 2]);
-      const double av[4] = {a01.x, a01.y, a23.x, a23.y};
-      const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] = fma(av[r], bv[c], acc[r][c]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int i = i0 + wr * 16 + lm * 4 + r;
-    if (i >= m.nb) continue;
-    double* row = logits + (bh * m.nb + i) * (int64_t)ld;
-#pragma unroll
-    for (int c2 = 0; c2 < 2; ++c2) {
-      const int j = j0 + wc * 32 + c2 * 16 + ln * 2;
-      if (j + 1 < m.nb) {
-        *reinterpret_cast<double2*>(row + j) = make_double2(acc[r][2 * c2] * scale, acc[r][2 * c2 + 1] * scale);
-      } else if (j < m.nb) {
-        row[j] = acc[r][2 * c2] * scale;
-      }
-    }
-  }
-}
 
 constexpr int SEL_WARPS = 8;
 
@@ -1063,41 +1010,39 @@ __global__ void __launch_bounds__(256) csr_kernel(const uint32_t* __restrict__ b
 
 template <typename T, int D>
 static cudaError_t launch_pool_td(const void* Q, const void* K, int ntensors, const Dims& m, int out, int frame_len,
-                                  double* qo, double* ko, double* qhi, double* khi, int nsm, cudaStream_t st) {
+                                  double* qo, double* ko, double* qhi, double* khi, const SliceOut& so, int nsm,
+                                  cudaStream_t st) {
   const int64_t units = m.BH * m.nb * ntensors;
   const int grid = (int)imin<int64_t>((units + 3) / 4, (int64_t)nsm * 16);
   const T* q = static_cast<const T*>(Q);
   const T* k = static_cast<const T*>(K);
-  const int ld = means_ld(m.nb);
-  if (out == kMeansT)
-    pool_kernel<T, D, kMeansT><<<grid, 128, 0, st>>>(q, k, ntensors, m, 0, ld, qo, ko, nullptr, nullptr);
+  if (out == kSliced)
+    pool_kernel<T, D, kSliced><<<grid, 128, 0, st>>>(q, k, ntensors, m, 0, nullptr, nullptr, nullptr, nullptr, so);
   else if (out == kFrameSums)
-    pool_kernel<T, D, kFrameSums><<<grid, 128, 0, st>>>(q, k, ntensors, m, frame_len, ld, qo, ko, qhi, khi);
+    pool_kernel<T, D, kFrameSums><<<grid, 128, 0, st>>>(q, k, ntensors, m, frame_len, qo, ko, qhi, khi, so);
   else
-    pool_kernel<T, D, kMeans><<<grid, 128, 0, st>>>(q, k, ntensors, m, 0, ld, qo, ko, nullptr, nullptr);
+    pool_kernel<T, D, kMeans><<<grid, 128, 0, st>>>(q, k, ntensors, m, 0, qo, ko, nullptr, nullptr, so);
   return cudaGetLastError();
 }
 
 // out: 0 = means [row][d], 1 = transposed means [bh][d][ld], 2 = frame segment sums.
 cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int out, int frame_len,
-                        double* qo, double* ko, double* qhi, double* khi, int nsm, cudaStream_t st) {
+                        double* qo, double* ko, double* qhi, double* khi, const SliceOut& so, int nsm,
+                        cudaStream_t st) {
   if (dtype == FVATTN_BF16) {
-    if (m.d == 128) return launch_pool_td<__nv_bfloat16, 128>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, nsm, st);
-    return launch_pool_td<__nv_bfloat16, 64>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, nsm, st);
+    if (m.d == 128)
+      return launch_pool_td<__nv_bfloat16, 128>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, so, nsm, st);
+    return launch_pool_td<__nv_bfloat16, 64>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, so, nsm, st);
   }
-  if (m.d == 128) return launch_pool_td<float, 128>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, nsm, st);
-  return launch_pool_td<float, 64>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, nsm, st);
+  if (m.d == 128) return launch_pool_td<float, 128>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, so, nsm, st);
+  return launch_pool_td<float, 64>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, so, nsm, st);
 }
 
-size_t means_t_elems(const Dims& m) { return (size_t)m.BH * m.d * means_ld(m.nb); }
 
-cudaError_t launch_topp(const double* qT, const double* kT, double* logits, const Dims& m, double p, int kblocks,
-                        double scale, const ForceCfg& fc, const SasaCfg& sasa, uint32_t* bits, int32_t* counts,
-                        int32_t* tile_cost, cudaStream_t st) {
-  dim3 g1((m.nb + ST - 1) / ST, (m.nb + ST - 1) / ST, (unsigned)m.BH);
-  if (m.d == 128) score_kernel<128><<<g1, 256, 0, st>>>(qT, kT, m, scale, logits);
-  else score_kernel<64><<<g1, 256, 0, st>>>(qT, kT, m, scale, logits);
-  cudaError_t e = cudaGetLastError();
+cudaError_t launch_topp(const SliceOut& so, double* logits, const Dims& m, double p, int kblocks, double scale,
+                        const ForceCfg& fc, const SasaCfg& sasa, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
+                        int32_t* status, cudaStream_t st) {
+  cudaError_t e = launch_score_tc(so.qs, so.ks, so.eq, so.ek, m, scale, logits, status, st);
   if (e != cudaSuccess) return e;
   if (m.nb <= 32 * 16) return launch_select_t<16>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost, st);
   if (m.nb <= 32 * 40) return launch_select_t<40>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost, st);

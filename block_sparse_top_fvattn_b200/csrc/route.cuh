@@ -13,24 +13,39 @@ struct ForceCfg {
 // Code of an entry whose key block is attended whole (all four allow bits, no boundaries).
 constexpr int32_t kCodeAll = 0xF | (64 << 8) | (64 << 16);
 
-size_t means_t_elems(const Dims& m);     // doubles of one transposed block-mean array
+// Row stride of the fp64 block-score matrix: nb rounded up to 32.
+__host__ __device__ __forceinline__ int means_ld(int nb) { return (nb + 31) & ~31; }
 size_t logits_elems(const Dims& m);      // doubles of the fp64 block-score matrix
 size_t frame_smem_bytes(const Dims& m);
 size_t schedule_smem_bytes(const Dims& m, int* groups);
 
-// out: 0 = means [row][d], 1 = means transposed per head [bh][d][ld], 2 = frame segment sums.
+// Block means as exact small-integer slices for the tensor-core score GEMM (score_tc.cu): per
+// block a power-of-two exponent and kScoreSlices bf16 planes, [BH][kScoreSlices][nb][d].
+constexpr int kScoreSlices = 5;
+struct SliceOut {
+  __nv_bfloat16* qs;
+  __nv_bfloat16* ks;
+  int32_t* eq;
+  int32_t* ek;
+};
+cudaError_t launch_score_tc(const __nv_bfloat16* qs, const __nv_bfloat16* ks, const int32_t* eq, const int32_t* ek,
+                            const Dims& m, double scale, double* logits, int32_t* status, cudaStream_t st);
+
+// out: 0 = means [row][d] (qo, ko), 1 = score slices and exponents (so), 2 = frame segment sums.
 cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int out, int frame_len,
-                        double* qo, double* ko, double* qhi, double* khi, int nsm, cudaStream_t st);
+                        double* qo, double* ko, double* qhi, double* khi, const SliceOut& so, int nsm,
+                        cudaStream_t st);
 // Slack-aware augmentation of 128-row tiles (fvattn_route_cfg.sasa_coef / sasa_trigger).
 struct SasaCfg {
   float coef;
   int trigger;
 };
 
-// kblocks > 0: keep the kblocks highest scores per row instead of the Top-p cut.
-cudaError_t launch_topp(const double* qT, const double* kT, double* logits, const Dims& m, double p, int kblocks,
-                        double scale, const ForceCfg& fc, const SasaCfg& sasa, uint32_t* bits, int32_t* counts,
-                        int32_t* tile_cost, cudaStream_t st);
+// Scores (tensor cores, from the slices), then the per-row cut. kblocks > 0: keep the kblocks
+// highest scores per row instead of the Top-p cut.
+cudaError_t launch_topp(const SliceOut& so, double* logits, const Dims& m, double p, int kblocks, double scale,
+                        const ForceCfg& fc, const SasaCfg& sasa, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
+                        int32_t* status, cudaStream_t st);
 // fsel: per head, the top-k key frames of every query frame ([BH][F][ceil(F/32)] bits).
 cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,
                          double* qf, double* kf, const Dims& m, int frame_len, int topk, double scale,
