@@ -89,7 +89,31 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ Q, cons
   const int64_t per = m.BH * m.nb;
   const int64_t units = per * ntensors;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t u = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); u < units; u += nwarps) {
+  // Software-pipelined over units: the first batch of the next unit is loaded before the current
+  // unit's reduction and epilogue, so the epilogue overlaps memory latency.
+  auto src_of = [&](int64_t uu) -> const T* {
+    const bool k_ = uu >= per;
+    const int64_t row_ = k_ ? uu - per : uu;
+    const int64_t bh_ = row_ / m.nb;
+    const int64_t t0_ = (row_ - bh_ * m.nb) * kBlock;
+    return (k_ ? K : Q) + (bh_ * m.S + t0_) * D + c * VEC;
+  };
+  auto nvalid_of = [&](int64_t uu) -> int {
+    const int64_t row_ = uu >= per ? uu - per : uu;
+    return (int)imin<int64_t>(kBlock, m.S - (row_ % m.nb) * kBlock);
+  };
+  uint4 v[BATCH];
+  int64_t u = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (u < units) {
+    const T* X0 = src_of(u);
+    const int nv0 = nvalid_of(u);
+#pragma unroll
+    for (int it = 0; it < BATCH; ++it) {
+      const int r = r0 + it * RPI;
+      v[it] = r < nv0 ? __ldg(reinterpret_cast<const uint4*>(X0 + (int64_t)r * D)) : make_uint4(0, 0, 0, 0);
+    }
+  }
+  for (; u < units; u += nwarps) {
     const bool isK = u >= per;
     const int64_t row = isK ? u - per : u;       // bh * nb + blk
     const int64_t bh = row / m.nb;
@@ -104,12 +128,7 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ Q, cons
     for (int e = 0; e < VEC; ++e) lo[e] = hi[e] = 0.0;
 #pragma unroll
     for (int b0 = 0; b0 < NIT; b0 += BATCH) {
-      uint4 v[BATCH];
-#pragma unroll
-      for (int it = 0; it < BATCH; ++it) {
-        const int r = r0 + (b0 + it) * RPI;
-        v[it] = r < nvalid ? __ldg(reinterpret_cast<const uint4*>(X + (int64_t)r * D)) : make_uint4(0, 0, 0, 0);
-      }
+      // v holds batch b0 of this unit (loaded by the previous iteration or the prologue)
 #pragma unroll
       for (int g = 0; g < BATCH; g += 4) {
         AccT sl[VEC], sh[VEC];
@@ -130,6 +149,19 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ Q, cons
         for (int e = 0; e < VEC; ++e) {
           lo[e] += (double)sl[e];
           if (FRAME) hi[e] += (double)sh[e];
+        }
+      }
+      // next batch: the rest of this unit, else the first batch of the next unit
+      const bool more = b0 + BATCH < NIT;
+      const int64_t un = u + nwarps;
+      if (more || un < units) {
+        const T* Xn = more ? X : src_of(un);
+        const int nvn = more ? nvalid : nvalid_of(un);
+        const int base = more ? b0 + BATCH : 0;
+#pragma unroll
+        for (int it = 0; it < BATCH; ++it) {
+          const int r = r0 + (base + it) * RPI;
+          v[it] = r < nvn ? __ldg(reinterpret_cast<const uint4*>(Xn + (int64_t)r * D)) : make_uint4(0, 0, 0, 0);
         }
       }
     }
