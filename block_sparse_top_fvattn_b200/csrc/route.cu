@@ -1,5 +1,7 @@
-// Router kernels: block pooling, fp64 block scores, row softmax, Top-p cut, frame-level
-// top-k, forced blocks, CSR rows, per-head loads, tile costs and the longest-first order.
+// Router kernels: block pooling (and the block means' integer slices for the tensor-core score
+// GEMM of score_tc.cu), row softmax, Top-p / top-k cut, slack-aware tile augmentation,
+// frame-level top-k, forced blocks, CSR rows, per-head loads, tile costs, the longest-first
+// order and the token-exact frame codes.
 //
 // Method: FVAttn blog summary ("腾讯+中山大学新作：视频生成提速2.11×，靠的是RLB和SASA"), section
 // "AI视频生成的阿喀琉斯之踵" (Top-p: smallest descending-importance prefix reaching p) and
@@ -45,9 +47,10 @@ __device__ __forceinline__ T warp_incl_scan(T v, int lane) {
 // is used, so every lane keeps 256 bytes in flight and no barrier is needed. Four rows are
 // summed in AccT (fp32 for bf16 input: exact unless the values' exponents are 16+ apart;
 // fp64 for fp32 input), the partial sums in fp64 in a fixed order, and the row groups of a
-// column are folded with shuffles. OUT selects what is written: means [row][d]; means
-// transposed per head, [bh][d][ld] with ld >= nb (the operand layout of the score GEMM); or
-// fp64 sums of the tokens before / after the block's first frame boundary, [row][d].
+// column are folded with shuffles. The next block's first batch is loaded before the current
+// block's epilogue. OUT selects what is written: means [row][d]; the means as exact bf16 integer
+// slices with power-of-two exponents (the operands of the score GEMM); or fp64 sums of the
+// tokens before / after the block's first frame boundary, [row][d].
 
 template <typename T> struct Acc;
 template <> struct Acc<__nv_bfloat16> { using type = float; static constexpr int kVec = 8; };
@@ -278,14 +281,6 @@ __device__ __forceinline__ int finalize_row(uint32_t* w, int i, const Dims& m, c
 
 constexpr int NWARP = 8;
 constexpr int kExtract = 16;   // max-extraction steps before the bisection fallback
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-               "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 // Order key of a probability weight: the bits of its fp32 rounding (non-negative floats order
 // like their bit patterns).
@@ -1057,7 +1052,7 @@ static cudaError_t launch_pool_td(const void* Q, const void* K, int ntensors, co
   return cudaGetLastError();
 }
 
-// out: 0 = means [row][d], 1 = transposed means [bh][d][ld], 2 = frame segment sums.
+// out: 0 = means [row][d], 1 = score slices and exponents, 2 = frame segment sums.
 cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int out, int frame_len,
                         double* qo, double* ko, double* qhi, double* khi, const SliceOut& so, int nsm,
                         cudaStream_t st) {
