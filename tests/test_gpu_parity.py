@@ -276,6 +276,7 @@ ATTN_CASES = [
     ("single", {"H": 3, "S": 64 * 7 + 5, "d": 64}, fv.RouteConfig(p=0.8, local_window=1)),
     ("single", {"H": 1, "S": 40}, fv.RouteConfig(p=0.9)),
     ("dit", {"H": 3, "S": 1560 * 2}, fv.RouteConfig(p=0.9)),
+    ("single", {"B": 2, "H": 2, "S": 64 * 9 + 30}, fv.RouteConfig(p=0.8)),        # B > 1, odd block count
 ]
 
 
@@ -348,3 +349,37 @@ def test_full_length_long_frame_mode_sampled_heads():
     rng = np.random.default_rng(1)
     items = [(int(bh), int(i)) for bh, i in zip(rng.integers(0, 4, 12), rng.integers(0, w.nb, 12))]
     check_attention(q, k, v, csr, gm, 1.0 / np.sqrt(128), items=items)
+
+
+# The three register/shared-memory variants of the per-row cut: rows of <= 512 blocks, of
+# 513..1280 blocks (the long layer's 1182) and of more than 1280 blocks (shared-memory cut),
+# each with the full block lists checked and attention on a sample of query blocks.
+@pytest.mark.slow
+@pytest.mark.parametrize("S,extra", [
+    (75600, {}),                                                        # nb = 1182
+    (1290 * 64 + 17, {}),                                               # nb = 1291: shared-memory cut
+    (700 * 64, {"mode": "topk", "topk_blocks": 40}),                    # nb = 700, top-k
+    (700 * 64 + 5, {"sasa_coef": 0.5, "sasa_trigger": 2}),               # nb = 701, tile augmentation
+])
+def test_long_rows_parity(S, extra):
+    w = get_workload("long", H=1, S=S, d=64)
+    x = make_inputs(w, device="cuda")
+    q, k, v = x["q"], x["k"], x["v"]
+    cfg = fv.RouteConfig(p=0.9, **extra)
+    if cfg.sasa_coef > 0:
+        B, H, S_, d = q.shape
+        _, gb, _ = check_route(q, k, dataclasses.replace(cfg, sasa_coef=0.0))
+        csr = fv.route(q, k, cfg)
+        assert fv.read_status(csr) == 0
+        gm = gpu_mask(csr)
+        r = oracle.route(q.reshape(B * H, S_, d), k.reshape(B * H, S_, d), to_oracle_cfg(cfg))
+        for i in range(w.nb):
+            if i ^ 1 < w.nb:
+                assert oracle.valid_sasa_row(r["pi"][0, i], gb[0, i], gb[0, i ^ 1], gm[0, i], cfg.sasa_coef,
+                                             cfg.sasa_trigger, "topp"), i
+        assert not (np.any(gm != r["mask"], axis=2) & ~r["near_tie"]).any()
+    else:
+        csr, gm, r = check_route(q, k, cfg)
+    rng = np.random.default_rng(2)
+    items = [(0, int(i)) for i in rng.integers(0, w.nb, 10)] + [(0, w.nb - 1)]
+    check_attention(q, k, v, csr, gm, 1.0 / np.sqrt(64), items=items)
