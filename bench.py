@@ -348,8 +348,17 @@ def run_ours(args, w):
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
 
-    def step():
+    # --plain-order: ascending tile ids instead of the router's longest-first order (to measure
+    # what the order buys; a diagnostic, not the product path)
+    plain = torch.arange(csr.tile_order.numel(), dtype=torch.int32, device=dev) if args.plain_order else None
+
+    def route_now():
         fv.route(q, k, cfg, csr=csr, workspace=ws)
+        if plain is not None:
+            csr.tile_order.copy_(plain)
+
+    def step():
+        route_now()
         fv.sparse_attn(q, k, v, csr, out=out)
 
     for _ in range(max(args.warmup, 3)):
@@ -378,7 +387,7 @@ def run_ours(args, w):
     for s in range(args.steps):
         ev[s][0].record(stream)
         if s % args.refresh_every == 0:              # routing reuse: refresh every N steps
-            fv.route(q, k, cfg, csr=csr, workspace=ws)
+            route_now()
             routed_steps += 1
         ev[s][1].record(stream)
         fv.sparse_attn(q, k, v, csr, out=out)
@@ -486,7 +495,8 @@ def run_ours(args, w):
                                              args.frame_exact),
                    "l2": f"inputs larger than L2 (Q,K,V = {3 * q.numel() * q.element_size() / 1e9:.2f} GB per layer)",
                    "parallelism": f"independent layer per GPU x{world}",
-                   **({"routing_refresh_every": args.refresh_every} if args.refresh_every > 1 else {})},
+                   **({"routing_refresh_every": args.refresh_every} if args.refresh_every > 1 else {}),
+                   "tile_order": "ascending tile id" if args.plain_order else "longest first"},
         "route_ms": route_avg, "attn_ms": attn_avg, "attn_tflops": attn_tflops,
         "pct_bf16_peak": 100.0 * value / pk["bf16_tflops"],
         "pct_bf16_peak_attn": 100.0 * attn_tflops / pk["bf16_tflops"],
@@ -528,6 +538,8 @@ def main():
     ap.add_argument("--sasa-trigger", type=int, default=1)
     ap.add_argument("--refresh-every", type=int, default=1,
                     help="recompute the routing every N steps and reuse it in between (1: every step)")
+    ap.add_argument("--plain-order", action="store_true",
+                    help="diagnostic: attention takes tiles in ascending id order instead of longest first")
     ap.add_argument("--emulate-ranks", type=int, default=0,
                     help="emulate runtime load balancing over this many ranks on one GPU (0: off)")
     ap.add_argument("--rlb-target", type=float, default=1.05)
