@@ -184,7 +184,7 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const 
     if (e == cudaSuccess)
       e = launch_topp(so, reinterpret_cast<double*>(ws + L.logits), m, cfg->p >= 1.f ? 1.0 : (double)cfg->p, kblocks,
                       scale, fc, SasaCfg{cfg->sasa_coef, cfg->sasa_trigger}, bits, counts, out->tile_cost,
-                      out->status, s);
+                      out->status, nsm, s);
   } else {
     double* qhi = reinterpret_cast<double*>(ws + L.qhi);
     double* khi = reinterpret_cast<double*>(ws + L.khi);

@@ -1068,8 +1068,8 @@ cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, c
 
 cudaError_t launch_topp(const SliceOut& so, double* logits, const Dims& m, double p, int kblocks, double scale,
                         const ForceCfg& fc, const SasaCfg& sasa, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
-                        int32_t* status, cudaStream_t st) {
-  cudaError_t e = launch_score_tc(so.qs, so.ks, so.eq, so.ek, m, scale, logits, status, st);
+                        int32_t* status, int nsm, cudaStream_t st) {
+  cudaError_t e = launch_score_tc(so.qs, so.ks, so.eq, so.ek, m, scale, logits, status, nsm, st);
   if (e != cudaSuccess) return e;
   if (m.nb <= 32 * 16) return launch_select_t<16>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost, st);
   if (m.nb <= 32 * 40) return launch_select_t<40>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost, st);

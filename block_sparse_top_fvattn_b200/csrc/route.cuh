@@ -29,7 +29,7 @@ struct SliceOut {
   int32_t* ek;
 };
 cudaError_t launch_score_tc(const __nv_bfloat16* qs, const __nv_bfloat16* ks, const int32_t* eq, const int32_t* ek,
-                            const Dims& m, double scale, double* logits, int32_t* status, cudaStream_t st);
+                            const Dims& m, double scale, double* logits, int32_t* status, int nsm, cudaStream_t st);
 
 // out: 0 = means [row][d] (qo, ko), 1 = score slices and exponents (so), 2 = frame segment sums.
 cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int out, int frame_len,
@@ -45,7 +45,7 @@ struct SasaCfg {
 // highest scores per row instead of the Top-p cut.
 cudaError_t launch_topp(const SliceOut& so, double* logits, const Dims& m, double p, int kblocks, double scale,
                         const ForceCfg& fc, const SasaCfg& sasa, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
-                        int32_t* status, cudaStream_t st);
+                        int32_t* status, int nsm, cudaStream_t st);
 // fsel: per head, the top-k key frames of every query frame ([BH][F][ceil(F/32)] bits).
 cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,
                          double* qf, double* kf, const Dims& m, int frame_len, int topk, double scale,

@@ -4,7 +4,7 @@
 //
 // The pool kernel writes each block mean x (fp64, d values) as a power-of-two scale 2^e with
 // max|x| < 2^e and five slices of integers in [-128, 128] (exact in bf16):
-//     x = 2^e * (X_0 2^-7 + X_1 2^-15 + X_2 2^-23 + X_3 2^-31 + X_4 2^-39) + (residual < 2^(e-46)).
+//     x = 2^e * (X_0 2^-7 + X_1 2^-15 + X_2 2^-23 + X_3 2^-31 + X_4 2^-39) + (residual < 2^(e-40)).
 // The dot product of two blocks is then a sum over slice pairs (a, b) of integer dot products
 // weighted 2^(e_i + f_j - 14 - 8(a + b)). Pairs of one level l = a + b share a weight, so their
 // sum is accumulated in one fp32 TMEM accumulator; every partial sum is an integer below
@@ -13,12 +13,14 @@
 // whose products the tensor cores compute exactly, in the manner of the Ozaki scheme for
 // accurate matrix products).
 //
-// One CTA per 128 x 32 tile of one head's score matrix, two CTAs per SM (5 levels x 32 columns
-// at 32-column offsets of a 256-column TMEM allocation): the five K slices stay in shared memory,
-// the Q slices stream in 64-dim chunks through four slots; one thread issues tcgen05.mma
-// (kind::f16, bf16 -> fp32); then every thread takes one row, combines its levels in fp64 into
-// the staging area (the K slices' space) and the CTA writes the fp64 logits row by row,
-// coalesced.
+// Work: the 128 x 32 output tiles of all heads in (head, row tile, column tile) order, split into
+// one contiguous range per CTA (one persistent CTA per SM), so a CTA loads the five Q slices of a
+// row tile once (160 KB, resident in shared memory) and only reloads them when its range enters
+// the next row tile. Per column tile the five K slices stream through a three-slot ring; one
+// thread issues tcgen05.mma (kind::f16, bf16 -> fp32) into one of two accumulator sets (5 levels
+// x 32 columns at 32-column TMEM offsets); eight epilogue warps drain the other set meanwhile
+// (two per TMEM lane quarter, 16 columns each), combine the levels in fp64, stage the tile in
+// shared memory and write the fp64 logit rows coalesced.
 #include <cuda.h>
 #include <math.h>
 
@@ -32,27 +34,31 @@ namespace fv {
 namespace {
 
 constexpr int kRowsQ = 128, kColsK = 32;
-constexpr int kQSlots = 4;
+constexpr int kKSlots = 3;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = (kEpiWarps + 2) * 32;          // + producer warp + MMA warp
+constexpr int kLevelCols = kScoreSlices * kColsK;       // one accumulator set: 160 TMEM columns
 constexpr uint32_t kWaitLimit = 1u << 22;
 
 template <int D>
 struct ScLayout {
   static constexpr int kChunks = D / 64;
   static constexpr int kQChunk = kRowsQ * 128;                  // [128 rows x 64 dims] bf16 = 16 KB
+  static constexpr int kQSlice = kChunks * kQChunk;
   static constexpr int kKChunk = kColsK * 128;                  // [32 rows x 64 dims] bf16 = 4 KB
-  static constexpr int kKSlice = kChunks * kKChunk;
-  static constexpr int kOffK = 0;                               // five K slices, later the staging
-  static constexpr int kKBytes = kScoreSlices * kKSlice;
-  static constexpr int kStage = kRowsQ * kColsK * 8;            // fp64 tile
-  static constexpr int kKRegion = ((kKBytes > kStage ? kKBytes : kStage) + 1023) & ~1023;
-  static constexpr int kOffQ = kKRegion;                        // Q chunk slots
-  static constexpr int kOffE = kOffQ + kQSlots * kQChunk;       // column exponents
-  static constexpr int kOffBar = kOffE + kColsK * 4;
-  static constexpr int kBytes = kOffBar + 128;
+  static constexpr int kKSlot = kChunks * kKChunk;              // one K slice of one column tile
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kScoreSlices * kQSlice;
+  static constexpr int kOffStage = kOffK + kKSlots * kKSlot;
+  static constexpr int kOffBar = kOffStage + kRowsQ * kColsK * 8;
+  static constexpr int kBytes = kOffBar + 256;
 };
 
 struct ScBars {
-  uint64_t k_full, q_full[kQSlots], q_empty[kQSlots], done;
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kKSlots], k_empty[kKSlots];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -60,139 +66,229 @@ struct ScBars {
 // 2^k for the exponent range of the logits (a normal double), exactly.
 __device__ __forceinline__ double pow2(int k) { return __longlong_as_double((long long)(1023 + k) << 52); }
 
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); }
+
+// A barrier of the epilogue warps that also returns whether every one of their threads passed
+// true, so that they take the same branch (leaving the tile loop) together.
+__device__ __forceinline__ bool epi_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kEpiWarps * 32)
+      : "memory");
+  return r != 0;
+}
+
 template <int D>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const int32_t* __restrict__ eq, const int32_t* __restrict__ ek, Dims m, double scale, int ld,
                     double* __restrict__ logits, int32_t* __restrict__ status) {
   using L = ScLayout<D>;
-  constexpr int NQ = kScoreSlices * L::kChunks;                 // Q chunks streamed: (slice, chunk)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   ScBars* bars = reinterpret_cast<ScBars*>(smem + L::kOffBar);
-  int32_t* sE = reinterpret_cast<int32_t*>(smem + L::kOffE);
-  double* stage = reinterpret_cast<double*>(smem + L::kOffK);
+  double* stage = reinterpret_cast<double*>(smem + L::kOffStage);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j0 = blockIdx.x * kColsK, i0 = blockIdx.y * kRowsQ;
-  const int64_t bh = blockIdx.z;
   volatile int* abort = &bars->abort;
 
+  // this CTA's contiguous range of tiles in (head, row tile, column tile) order
+  const int nrt = (m.nb + kRowsQ - 1) / kRowsQ, nct = (m.nb + kColsK - 1) / kColsK;
+  const int64_t T = m.BH * nrt * nct;
+  const int64_t t_begin = T * blockIdx.x / gridDim.x, t_end = T * (blockIdx.x + 1) / gridDim.x;
+  auto row_tile = [&](int64_t t) { return t / nct; };           // bh * nrt + rt
+
   if (threadIdx.x == 0) {
-    tc::mbar_init(&bars->k_full, 1);
-    for (int s = 0; s < kQSlots; ++s) {
-      tc::mbar_init(&bars->q_full[s], 1);
-      tc::mbar_init(&bars->q_empty[s], 1);
+    tc::mbar_init(&bars->q_full, 1);
+    tc::mbar_init(&bars->q_empty, 1);
+    for (int s = 0; s < kKSlots; ++s) {
+      tc::mbar_init(&bars->k_full[s], 1);
+      tc::mbar_init(&bars->k_empty[s], 1);
     }
-    tc::mbar_init(&bars->done, 1);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&bars->acc_full[s], 1);
+      tc::mbar_init(&bars->acc_empty[s], kEpiWarps);
+    }
+    tc::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 1) {
-    tc::tmem_alloc(&bars->tmem_base, 256);
+  if (warp == kEpiWarps + 1) {
+    tc::tmem_alloc(&bars->tmem_base, 512);
     tc::tmem_relinquish();
   }
-  if (threadIdx.x < kColsK) {
-    const int j = j0 + threadIdx.x;
-    sE[threadIdx.x] = j < m.nb ? ek[bh * m.nb + j] : 0;
-  }
-  const int r = warp * 32 + lane, i = i0 + r;
-  const int ei = i < m.nb ? eq[bh * m.nb + i] : 0;      // this thread's row exponent, read early
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tbase = bars->tmem_base;
 
-  if (warp == 0 && lane == 0) {
-    // ---- loads: the five K slices once; Q (slice a, 64-dim chunk c) through the slots
-    tc::mbar_expect_tx(&bars->k_full, L::kKBytes);
-    for (int b = 0; b < kScoreSlices; ++b)
-      for (int c = 0; c < L::kChunks; ++c)
-        tc::tma_load_3d(smem + L::kOffK + b * L::kKSlice + c * L::kKChunk, &tmK, &bars->k_full, c * 64, j0,
-                        (int)(bh * kScoreSlices + b));
-    for (int n = 0; n < NQ; ++n) {
-      const int s = n % kQSlots, a = n / L::kChunks, c = n % L::kChunks;
-      if (n >= kQSlots && !tc::mbar_wait(&bars->q_empty[s], (n / kQSlots - 1) & 1, abort, kWaitLimit)) {
-        atomicCAS(&bars->abort, 0, 1);
-        break;
-      }
-      tc::mbar_expect_tx(&bars->q_full[s], L::kQChunk);
-      for (int h = 0; h < 2; ++h)
-        tc::tma_load_3d(smem + L::kOffQ + s * L::kQChunk + h * 64 * 128, &tmQ, &bars->q_full[s], c * 64,
-                        i0 + h * 64, (int)(bh * kScoreSlices + a));
-    }
-  } else if (warp == 1 && lane == 0) {
-    // ---- MMAs: level a+b += Q_a K_b^T for a + b < 5, chunk by chunk of the head dimension; the
-    // first MMA into each level (a = 0, first chunk, first K16 step) overwrites it. The closing
-    // commit runs on every path, so the teardown can wait for whatever was issued.
-    constexpr uint32_t idesc = tc::idesc_bf16_f32(kRowsQ, kColsK, 0, 0);
-    const uint32_t kaddr = tc::smem_u32(smem + L::kOffK), qaddr = tc::smem_u32(smem + L::kOffQ);
-    bool ok = tc::mbar_wait(&bars->k_full, 0, abort, kWaitLimit);
-    for (int n = 0; ok && n < NQ; ++n) {
-      const int s = n % kQSlots, a = n / L::kChunks, c = n % L::kChunks;
-      if (!tc::mbar_wait(&bars->q_full[s], (n / kQSlots) & 1, abort, kWaitLimit)) {
-        ok = false;
-        break;
-      }
-      tc::fence_after_sync();
-      for (int b = 0; a + b < kScoreSlices; ++b) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = tc::smem_desc_sw128(qaddr + s * L::kQChunk + kk * 32, 16, 1024);
-          const uint64_t bd = tc::smem_desc_sw128(kaddr + b * L::kKSlice + c * L::kKChunk + kk * 32, 16, 1024);
-          tc::mma_f16(tbase + (a + b) * kColsK, ad, bd, idesc, (a > 0 || c > 0 || kk > 0) ? 1u : 0u);
+  if (warp == kEpiWarps) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- loads
+      uint32_t kc = 0, qc = 0;
+      int64_t cur = -1;
+      for (int64_t t = t_begin; t < t_end; ++t) {
+        const int64_t rtile = row_tile(t);
+        const int64_t bh = rtile / nrt;
+        const int i0 = (int)(rtile - bh * nrt) * kRowsQ, j0 = (int)(t - rtile * nct) * kColsK;
+        if (rtile != cur) {
+          // the previous row tile's MMAs are done with the Q slices before they are replaced
+          if (qc > 0 && !tc::mbar_wait(&bars->q_empty, (qc - 1) & 1, abort, kWaitLimit)) {
+            atomicCAS(&bars->abort, 0, 1);
+            break;
+          }
+          tc::mbar_expect_tx(&bars->q_full, kScoreSlices * L::kQSlice);
+          for (int a = 0; a < kScoreSlices; ++a)
+            for (int c = 0; c < L::kChunks; ++c)
+              for (int h = 0; h < 2; ++h)
+                tc::tma_load_3d(smem + L::kOffQ + a * L::kQSlice + c * L::kQChunk + h * 64 * 128, &tmQ, &bars->q_full,
+                                c * 64, i0 + h * 64, (int)(bh * kScoreSlices + a));
+          cur = rtile;
+          ++qc;
+        }
+        bool ok = true;
+        for (int b = 0; b < kScoreSlices; ++b, ++kc) {
+          const int s = kc % kKSlots;
+          if (!tc::mbar_wait(&bars->k_empty[s], ((kc / kKSlots) & 1) ^ 1, abort, kWaitLimit)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_expect_tx(&bars->k_full[s], L::kKSlot);
+          for (int c = 0; c < L::kChunks; ++c)
+            tc::tma_load_3d(smem + L::kOffK + s * L::kKSlot + c * L::kKChunk, &tmK, &bars->k_full[s], c * 64, j0,
+                            (int)(bh * kScoreSlices + b));
+        }
+        if (!ok) {
+          atomicCAS(&bars->abort, 0, 2);
+          break;
         }
       }
-      tc::mma_commit(&bars->q_empty[s]);
     }
-    if (!ok) atomicCAS(&bars->abort, 0, 2);
-    tc::mma_commit(&bars->done);
-  }
-  __syncwarp();
-
-  // ---- epilogue: one row per thread (TMEM lane) into the staging tile, then coalesced rows
-  const bool done = __all_sync(0xffffffffu, tc::mbar_wait(&bars->done, 0, abort, kWaitLimit));
-  tc::fence_after_sync();
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  if (done && !*abort) {
-#pragma unroll 1
-    for (int cc = 0; cc < kColsK / 16; ++cc) {
+  } else if (warp == kEpiWarps + 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMAs
+      // Column tile j (local index) goes to accumulator set j % 2: level a+b += Q_a K_b^T for
+      // a + b < 5. With b outermost, b = 0 touches every level first (a = level), so those MMAs
+      // (first chunk, first K16 step) overwrite. The closing commit runs on every path, and the
+      // thread waits for it, so no MMA is in flight when TMEM is released.
+      constexpr uint32_t idesc = tc::idesc_bf16_f32(kRowsQ, kColsK, 0, 0);
+      // Shared-memory descriptors are linear in the start address (bits 0-13 hold address >> 4,
+      // and every operand lies below 256 KB), so they are made once and offset by constants.
+      const uint64_t qdesc0 = tc::smem_desc_sw128(tc::smem_u32(smem + L::kOffQ), 16, 1024);
+      const uint64_t kdesc0 = tc::smem_desc_sw128(tc::smem_u32(smem + L::kOffK), 16, 1024);
+      uint32_t kc = 0, qc = 0;
+      int64_t cur = -1;
+      bool ok = true;
+      for (int64_t t = t_begin; ok && t < t_end; ++t) {
+        const uint32_t j = (uint32_t)(t - t_begin), buf = j & 1;
+        const int64_t rtile = row_tile(t);
+        if (rtile != cur) {
+          if (!tc::mbar_wait(&bars->q_full, qc & 1, abort, kWaitLimit)) { ok = false; break; }
+          cur = rtile;
+          ++qc;
+        }
+        if (!tc::mbar_wait(&bars->acc_empty[buf], ((j >> 1) & 1) ^ 1, abort, kWaitLimit)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t dbase = tbase + buf * kLevelCols;
+#pragma unroll
+        for (int b = 0; b < kScoreSlices; ++b, ++kc) {
+          const int s = kc % kKSlots;
+          if (!tc::mbar_wait(&bars->k_full[s], (kc / kKSlots) & 1, abort, kWaitLimit)) { ok = false; break; }
+          tc::fence_after_sync();
+          const uint64_t kd = kdesc0 + (uint64_t)((s * L::kKSlot) >> 4);
+#pragma unroll
+          for (int a = 0; a < kScoreSlices; ++a) {
+            if (a + b >= kScoreSlices) continue;
+#pragma unroll
+            for (int c = 0; c < L::kChunks; ++c)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                tc::mma_f16(dbase + (a + b) * kColsK, qdesc0 + ((a * L::kQSlice + c * L::kQChunk + kk * 32) >> 4),
+                            kd + ((c * L::kKChunk + kk * 32) >> 4), idesc, (b > 0 || c > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc::mma_commit(&bars->k_empty[s]);
+        }
+        if (!ok) break;
+        tc::mma_commit(&bars->acc_full[buf]);
+        if (t + 1 == t_end || row_tile(t + 1) != rtile) tc::mma_commit(&bars->q_empty);
+      }
+      if (!ok) atomicCAS(&bars->abort, 0, 3);
+      tc::mma_commit(&bars->drain);
+      tc::mbar_wait(&bars->drain, 0, abort, kWaitLimit);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 0-7)
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;                           // tile row == TMEM lane
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    int64_t cur = -1;
+    int ei = 0;
+    for (int64_t t = t_begin; t < t_end; ++t) {
+      const uint32_t j = (uint32_t)(t - t_begin), buf = j & 1;
+      const int64_t rtile = row_tile(t);
+      const int64_t bh = rtile / nrt;
+      const int i0 = (int)(rtile - bh * nrt) * kRowsQ, j0 = (int)(t - rtile * nct) * kColsK;
+      if (rtile != cur) {
+        ei = i0 + r < m.nb ? eq[bh * m.nb + i0 + r] : 0;
+        cur = rtile;
+      }
+      // the 16 column exponents of this warp's half, one per lane 0-15
+      const int jl = j0 + half * 16 + (lane & 15);
+      const int ej_l = jl < m.nb ? ek[bh * m.nb + jl] : 0;
+      const bool ready = tc::mbar_wait(&bars->acc_full[buf], (j >> 1) & 1, abort, kWaitLimit);
+      if (!epi_all(ready && !*abort)) break;                      // every epilogue warp leaves together
+      tc::fence_after_sync();
       uint32_t acc[kScoreSlices][16];
 #pragma unroll
-      for (int l = 0; l < kScoreSlices; ++l) tc::tmem_ld16(tbase + lane_off + l * kColsK + cc * 16, acc[l]);
+      for (int l = 0; l < kScoreSlices; ++l)
+        tc::tmem_ld16(tbase + lane_off + buf * kLevelCols + l * kColsK + half * 16, acc[l]);
       tc::tmem_ld_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bars->acc_empty[buf]);     // the set can take the next tile
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const int jj = cc * 16 + e;
         // levels combined from the finest: v = A_0 + 2^-8 (A_1 + 2^-8 (A_2 + ...))
         double v = (double)__uint_as_float(acc[kScoreSlices - 1][e]);
 #pragma unroll
         for (int l = kScoreSlices - 2; l >= 0; --l) v = fma(v, 0x1p-8, (double)__uint_as_float(acc[l][e]));
-        const int k = ei + sE[jj] - 14;
-        stage[r * kColsK + ((jj + r) % kColsK)] = (v * scale) * pow2(max(-1000, min(1000, k)));
+        const int k = ei + __shfl_sync(0xffffffffu, ej_l, e) - 14;
+        const int col = half * 16 + e;
+        stage[r * kColsK + ((col + r) & (kColsK - 1))] = (v * scale) * pow2(max(-1000, min(1000, k)));
       }
+      epi_sync();
+      // coalesced rows: 128 rows x 32 doubles, 256 threads, two consecutive doubles each
+      const int ncol = min(kColsK, m.nb - j0);
+      for (int x = threadIdx.x; x < kRowsQ * kColsK / 2; x += kEpiWarps * 32) {
+        const int rr = x / (kColsK / 2), cc = 2 * (x - rr * (kColsK / 2));
+        if (i0 + rr < m.nb) {
+          double* dst = logits + (bh * m.nb + i0 + rr) * (int64_t)ld + j0 + cc;
+          const double v0 = stage[rr * kColsK + ((cc + rr) & (kColsK - 1))];
+          const double v1 = stage[rr * kColsK + ((cc + 1 + rr) & (kColsK - 1))];
+          if (cc + 1 < ncol) *reinterpret_cast<double2*>(dst) = make_double2(v0, v1);
+          else if (cc < ncol) dst[0] = v0;
+        }
+      }
+      epi_sync();
     }
   }
+
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  if (done && !*abort) {
-    const int ncol = min(kColsK, m.nb - j0);
-    for (int x = threadIdx.x; x < kRowsQ * kColsK; x += blockDim.x) {
-      const int rr = x / kColsK, jj = x - rr * kColsK;
-      if (i0 + rr < m.nb && jj < ncol)
-        logits[(bh * m.nb + i0 + rr) * (int64_t)ld + j0 + jj] = stage[rr * kColsK + ((jj + rr) % kColsK)];
-    }
-  }
-  if (warp == 1) tc::tmem_dealloc(tbase, 256);
+  if (warp == kEpiWarps + 1) tc::tmem_dealloc(tbase, 512);
   if (threadIdx.x == 0 && bars->abort) report_error(status, FVATTN_ERR_TIMEOUT, 30 + bars->abort);
 }
 
 template <int D>
 cudaError_t launch_score_tc_d(const __nv_bfloat16* qs, const __nv_bfloat16* ks, const int32_t* eq,
                               const int32_t* ek, const Dims& m, double scale, double* logits, int32_t* status,
-                              cudaStream_t st) {
-  if (m.BH > 65535) return cudaErrorInvalidValue;
+                              int nsm, cudaStream_t st) {
   CUtensorMap mq, mk;
   const uint64_t planes = (uint64_t)m.BH * kScoreSlices;
   if (!make_map_bf16_3d(&mq, qs, (uint64_t)D, (uint64_t)m.nb, planes, 64) ||
@@ -201,17 +297,18 @@ cudaError_t launch_score_tc_d(const __nv_bfloat16* qs, const __nv_bfloat16* ks, 
   const size_t smem = ScLayout<D>::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((m.nb + kColsK - 1) / kColsK, (m.nb + kRowsQ - 1) / kRowsQ, (unsigned)m.BH);
-  score_tc_kernel<D><<<grid, 128, smem, st>>>(mq, mk, eq, ek, m, scale, means_ld(m.nb), logits, status);
+  const int64_t tiles = m.BH * ((m.nb + kRowsQ - 1) / kRowsQ) * ((m.nb + kColsK - 1) / kColsK);
+  const int grid = (int)imin<int64_t>(tiles, nsm);
+  score_tc_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, eq, ek, m, scale, means_ld(m.nb), logits, status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_score_tc(const __nv_bfloat16* qs, const __nv_bfloat16* ks, const int32_t* eq, const int32_t* ek,
-                            const Dims& m, double scale, double* logits, int32_t* status, cudaStream_t st) {
-  if (m.d == 128) return launch_score_tc_d<128>(qs, ks, eq, ek, m, scale, logits, status, st);
-  return launch_score_tc_d<64>(qs, ks, eq, ek, m, scale, logits, status, st);
+                            const Dims& m, double scale, double* logits, int32_t* status, int nsm, cudaStream_t st) {
+  if (m.d == 128) return launch_score_tc_d<128>(qs, ks, eq, ek, m, scale, logits, status, nsm, st);
+  return launch_score_tc_d<64>(qs, ks, eq, ek, m, scale, logits, status, nsm, st);
 }
 
 }  // namespace fv
