@@ -2,9 +2,11 @@
 
 Block selections must match bit for bit except on near-tie rows (a cumulative mass within
 1e-5 of p at the cut, or a probability gap under 1e-6 at the boundary), where the GPU's set
-must be a valid selection and is then fed to the attention oracle. Attention outputs must
-be within max-abs 2e-2 and mean-abs 2e-3 of the oracle for bf16 inputs (fp32 inputs: the
-notes' own full-coverage bound, max-abs 1e-4)."""
+must be a valid selection. Every expected value comes from the oracle on the same inputs: the
+attention reference uses the oracle's selection, and query blocks whose GPU selection
+(legitimately) differs are left out of that comparison. Attention outputs must be within
+max-abs 2e-2 and mean-abs 2e-3 of the oracle for bf16 inputs (fp32 inputs: the notes' own
+full-coverage bound, max-abs 1e-4)."""
 import dataclasses
 
 import numpy as np
@@ -47,8 +49,33 @@ def to_oracle_cfg(cfg: fv.RouteConfig) -> oracle.RouteCfg:
                            sasa_coef=cfg.sasa_coef, sasa_trigger=cfg.sasa_trigger, frame_exact=cfg.frame_exact)
 
 
+def check_bookkeeping_properties(csr, gm):
+    """Invariants of the router's bookkeeping on its own selection, in plain NumPy: row offsets
+    are the prefix sums of the row counts, head loads their per-head sums, tile costs the sizes
+    of the unions of query blocks 2t and 2t+1, and the tile order is by cost, largest first,
+    ties by ascending tile id."""
+    BH, nb, _ = gm.shape
+    counts = gm.reshape(BH * nb, nb).sum(axis=1)
+    np.testing.assert_array_equal(csr.row_ptr.cpu().numpy()[1:], np.cumsum(counts))
+    np.testing.assert_array_equal(csr.head_load.cpu().numpy(), gm.sum(axis=(1, 2)))
+    nt = -(-nb // 2)
+    pair = np.zeros((BH, nt, nb), dtype=bool)
+    pair[:, :, :] = gm[:, 0::2]
+    pair[:, : nb // 2] |= gm[:, 1::2]
+    costs = pair.sum(axis=2).reshape(-1)
+    np.testing.assert_array_equal(csr.tile_cost.cpu().numpy(), costs)
+    order = csr.tile_order.cpu().numpy()
+    assert sorted(order.tolist()) == list(range(costs.size))
+    key = np.stack([-costs[order], order], axis=1)
+    assert all(tuple(key[t]) <= tuple(key[t + 1]) for t in range(len(order) - 1))
+    assert int(csr.nnz.item()) == int(counts.sum())
+
+
 def check_route(q, k, cfg: fv.RouteConfig, csr=None, r=None):
-    """Run the GPU router and compare with the oracle. Returns (gpu mask, oracle result)."""
+    """Run the GPU router and compare with the oracle. Returns (csr, gpu mask, oracle result).
+    Rows may differ only where the oracle flags a near-tie, and there the GPU's set must be a
+    valid selection; the bookkeeping equals the oracle's when no row differs, and satisfies its
+    invariants on the GPU's own selection in every case."""
     B, H, S, d = q.shape
     csr = fv.route(q, k, cfg, csr=csr)
     assert fv.read_status(csr) == 0
@@ -63,27 +90,35 @@ def check_route(q, k, cfg: fv.RouteConfig, csr=None, r=None):
     assert not bad.any(), f"{int(bad.sum())} non-tie rows differ, e.g. {np.argwhere(bad)[:5].tolist()}"
     for bh, i in np.argwhere(diff_rows):
         assert oracle.valid_near_tie_set(r, bh, i, gm[bh, i], S, oc), (bh, i)
-    # bookkeeping is bit-exact against the GPU's own selection
-    rp, ci = oracle.csr_from_mask(gm)
-    np.testing.assert_array_equal(csr.row_ptr.cpu().numpy(), rp)
-    np.testing.assert_array_equal(csr.col_idx[: len(ci)].cpu().numpy(), ci)
-    assert int(csr.nnz.item()) == len(ci)
-    np.testing.assert_array_equal(csr.head_load.cpu().numpy(), oracle.head_loads(gm))
-    costs = oracle.tile_costs(gm)
-    np.testing.assert_array_equal(csr.tile_cost.cpu().numpy(), costs.reshape(-1))
-    np.testing.assert_array_equal(csr.tile_order.cpu().numpy(), oracle.lpt_order(costs))
+    if not diff_rows.any():
+        rp, ci = oracle.csr_from_mask(om)
+        np.testing.assert_array_equal(csr.row_ptr.cpu().numpy(), rp)
+        np.testing.assert_array_equal(csr.col_idx[: len(ci)].cpu().numpy(), ci)
+        assert int(csr.nnz.item()) == len(ci)
+        np.testing.assert_array_equal(csr.head_load.cpu().numpy(), oracle.head_loads(om))
+        costs = oracle.tile_costs(om)
+        np.testing.assert_array_equal(csr.tile_cost.cpu().numpy(), costs.reshape(-1))
+        np.testing.assert_array_equal(csr.tile_order.cpu().numpy(), oracle.lpt_order(costs))
+    check_bookkeeping_properties(csr, gm)
     return csr, gm, r
 
 
-def check_attention(q, k, v, csr, gm, scale, items=None, max_abs=MAX_ABS_BF16, mean_abs=MEAN_ABS_BF16):
+def check_attention(q, k, v, csr, r, gm, scale, items=None, max_abs=MAX_ABS_BF16, mean_abs=MEAN_ABS_BF16):
+    """The library's attention against the oracle's attention under the oracle's selection
+    (r["mask"]). Query blocks whose GPU selection differs from the oracle's (near-tie rows,
+    validated by check_route) are left out of the element-wise comparison."""
     B, H, S, d = q.shape
     o = fv.sparse_attn(q, k, v, csr)
     assert fv.read_status(csr) == 0
     nb = -(-S // 64)
+    ref_mask = r["mask"]
+    differs = np.any(gm != ref_mask, axis=2)
     if items is None:
         items = [(bh, i) for bh in range(B * H) for i in range(nb)]
+    items = [(bh, i) for bh, i in items if not differs[bh, i]]
+    assert items, "no query block left to compare"
     Q, K, V = (t.reshape(B * H, S, d).cpu() for t in (q, k, v))
-    ref = oracle.attention_rows(Q, K, V, gm, scale, items)
+    ref = oracle.attention_rows(Q, K, V, ref_mask, scale, items)
     O = o.reshape(B * H, S, d).float().cpu().numpy()
     errs = []
     for (bh, i), blk in ref.items():
@@ -166,7 +201,7 @@ def test_topk_blocks_parity(name, kw, cfg):
     if cfg.topk_blocks >= w.nb:
         assert gm.all()
     if w.dtype == "bf16":
-        check_attention(q, k, v, csr, gm, 1.0 / np.sqrt(w.d))
+        check_attention(q, k, v, csr, r, gm, 1.0 / np.sqrt(w.d))
 
 
 # Slack-aware augmentation of 128-row tiles: the GPU's base routing is checked as above; the
@@ -208,15 +243,17 @@ def test_sasa_parity(name, kw, cfg):
     if cfg.sasa_trigger > nb:
         assert np.array_equal(gm, gb)
     # the tile costs (unions) do not change; the bookkeeping follows the augmented sets
-    costs = oracle.tile_costs(gm)
-    np.testing.assert_array_equal(costs, oracle.tile_costs(gb))
-    np.testing.assert_array_equal(csr.tile_cost.cpu().numpy(), costs.reshape(-1))
-    np.testing.assert_array_equal(csr.tile_order.cpu().numpy(), oracle.lpt_order(costs))
-    np.testing.assert_array_equal(csr.head_load.cpu().numpy(), oracle.head_loads(gm))
-    rp, ci = oracle.csr_from_mask(gm)
-    np.testing.assert_array_equal(csr.row_ptr.cpu().numpy(), rp)
-    np.testing.assert_array_equal(csr.col_idx[: len(ci)].cpu().numpy(), ci)
-    check_attention(q, k, v, csr, gm, 1.0 / np.sqrt(d))
+    base = fv.route(q, k, dataclasses.replace(cfg, sasa_coef=0.0))
+    np.testing.assert_array_equal(csr.tile_cost.cpu().numpy(), base.tile_cost.cpu().numpy())
+    check_bookkeeping_properties(csr, gm)
+    if not diff.any():
+        rp, ci = oracle.csr_from_mask(r["mask"])
+        np.testing.assert_array_equal(csr.row_ptr.cpu().numpy(), rp)
+        np.testing.assert_array_equal(csr.col_idx[: len(ci)].cpu().numpy(), ci)
+        np.testing.assert_array_equal(csr.head_load.cpu().numpy(), oracle.head_loads(r["mask"]))
+        costs = oracle.tile_costs(r["mask"])
+        np.testing.assert_array_equal(csr.tile_order.cpu().numpy(), oracle.lpt_order(costs))
+    check_attention(q, k, v, csr, r, gm, 1.0 / np.sqrt(d))
 
 
 # Token-exact frame mode: the same CSR as the block-granular frame mode, per-entry codes equal to
@@ -284,7 +321,7 @@ ATTN_CASES = [
 def test_attention_parity_bf16(name, kw, cfg):
     w, q, k, v = small_inputs(name, **kw)
     csr, gm, r = check_route(q, k, cfg)
-    check_attention(q, k, v, csr, gm, 1.0 / np.sqrt(w.d))
+    check_attention(q, k, v, csr, r, gm, 1.0 / np.sqrt(w.d))
 
 
 def test_attention_p1_equals_dense_bf16():
@@ -301,7 +338,7 @@ def test_attention_p1_equals_dense_bf16():
 def test_tiny_fp32_path(p):
     w, q, k, v = small_inputs("tiny", alpha=("const", 0.4))
     csr, gm, r = check_route(q, k, fv.RouteConfig(p=p))
-    check_attention(q, k, v, csr, gm, 1.0 / 8.0, max_abs=MAX_ABS_F32, mean_abs=MAX_ABS_F32)
+    check_attention(q, k, v, csr, r, gm, 1.0 / 8.0, max_abs=MAX_ABS_F32, mean_abs=MAX_ABS_F32)
 
 
 def test_attention_lse_and_determinism():
@@ -334,7 +371,7 @@ def test_full_size_dit_layer_sampled():
     rng = np.random.default_rng(0)
     items = [(int(bh), int(i)) for bh, i in zip(rng.integers(0, 40, 48), rng.integers(0, w.nb, 48))]
     items += [(0, w.nb - 1), (39, w.nb - 1)]                      # the ragged last block
-    _, emax, emean = check_attention(q, k, v, csr, gm, 1.0 / np.sqrt(128), items=items)
+    _, emax, emean = check_attention(q, k, v, csr, r, gm, 1.0 / np.sqrt(128), items=items)
 
 
 @pytest.mark.slow
@@ -348,7 +385,7 @@ def test_full_length_long_frame_mode_sampled_heads():
     csr, gm, r = check_route(q, k, cfg)
     rng = np.random.default_rng(1)
     items = [(int(bh), int(i)) for bh, i in zip(rng.integers(0, 4, 12), rng.integers(0, w.nb, 12))]
-    check_attention(q, k, v, csr, gm, 1.0 / np.sqrt(128), items=items)
+    check_attention(q, k, v, csr, r, gm, 1.0 / np.sqrt(128), items=items)
 
 
 # The three register/shared-memory variants of the per-row cut: rows of <= 512 blocks, of
@@ -382,4 +419,4 @@ def test_long_rows_parity(S, extra):
         csr, gm, r = check_route(q, k, cfg)
     rng = np.random.default_rng(2)
     items = [(0, int(i)) for i in rng.integers(0, w.nb, 10)] + [(0, w.nb - 1)]
-    check_attention(q, k, v, csr, gm, 1.0 / np.sqrt(64), items=items)
+    check_attention(q, k, v, csr, r, gm, 1.0 / np.sqrt(64), items=items)
