@@ -102,3 +102,17 @@ def test_lazy_router_reuses_the_routing():
         e = np.abs(o.reshape(B * H, S, d).float().cpu().numpy() - ref)
         assert e.max() <= 2e-2 and e.mean() <= 2e-3
     assert layer.routed == 2                                   # steps 0 and 3
+
+
+def test_select_heads_reports_a_bad_tile_order():
+    # The kernel checks every entry against the tile count before using it; a corrupted entry is
+    # dropped and reported as FVATTN_ERR_INVALID (-1) in the device status word.
+    w, q, k, v = _inputs("single", H=2, S=1000)
+    csr = fv.route(q, k, fv.RouteConfig(p=0.9))
+    assert fv.read_status(csr) == 0
+    n = csr.tile_order.numel()
+    csr.tile_order[0] = n + 5
+    csr.tile_order[1] = -3
+    fv.select_heads(csr, torch.ones(2, dtype=torch.uint8, device="cuda"))
+    assert fv.read_status(csr) == -1
+    assert int(csr.status[3].item()) == n - 2          # the other tiles are kept
