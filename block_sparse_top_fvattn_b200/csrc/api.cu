@@ -73,7 +73,7 @@ WsLayout ws_layout(const Dims& m, int mode) {
   const bool scored = mode == FVATTN_MODE_TOPP || mode == FVATTN_MODE_TOPK_BLOCKS;
   const size_t means = (size_t)m.BH * m.nb * m.d * sizeof(double);
   if (scored) {
-    const size_t slices = (size_t)m.BH * kScoreSlices * m.nb * m.d * sizeof(__nv_bfloat16);
+    const size_t slices = (size_t)m.BH * kScoreSlices * m.nb * kSliceRow;
     L.qs = take(off, slices);
     L.ks = take(off, slices);
     L.eq = take(off, (size_t)m.BH * m.nb * sizeof(int32_t));
@@ -178,7 +178,7 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const 
   cudaError_t e;
   if (cfg->mode == FVATTN_MODE_TOPP || cfg->mode == FVATTN_MODE_TOPK_BLOCKS) {
     const int kblocks = cfg->mode == FVATTN_MODE_TOPK_BLOCKS ? cfg->topk_blocks : 0;
-    const SliceOut so{reinterpret_cast<__nv_bfloat16*>(ws + L.qs), reinterpret_cast<__nv_bfloat16*>(ws + L.ks),
+    const SliceOut so{reinterpret_cast<int8_t*>(ws + L.qs), reinterpret_cast<int8_t*>(ws + L.ks),
                       reinterpret_cast<int32_t*>(ws + L.eq), reinterpret_cast<int32_t*>(ws + L.ek)};
     e = launch_pool(Q, K, 2, shape->dtype, m, 1, 0, nullptr, nullptr, nullptr, nullptr, so, nsm, s);
     if (e == cudaSuccess)

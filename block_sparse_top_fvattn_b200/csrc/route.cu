@@ -176,10 +176,11 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ Q, cons
         if (FRAME) hi[e] += __shfl_xor_sync(0xffffffffu, hi[e], off);
       }
     if (OUT == kSliced) {
-      // The mean as a power-of-two scale 2^ex (max|x| < 2^ex) and kScoreSlices base-256 digits
-      // in [-128, 128] (exact in bf16): N = rint(x 2^(39-ex)), |N| < 2^39, written as
-      // N = X_0 2^32 + X_1 2^24 + X_2 2^16 + X_3 2^8 + X_4, i.e. x ~ 2^ex sum_a X_a 2^(-7-8a), by
-      // integer shifts (digits rounded half up from the top).
+      // The mean as a power-of-two scale 2^ex and kScoreSlices signed 8-bit digits: with
+      // N = rint(x 2^(39-ex)), N = X_0 2^32 + X_1 2^24 + X_2 2^16 + X_3 2^8 + X_4, i.e.
+      // x ~ 2^ex sum_a X_a 2^(-7-8a). X_4..X_1 are the balanced base-256 digits (in [-128, 127],
+      // taken from the bottom), X_0 the rest. ex is the smallest power of two above max|x|,
+      // raised by one when max|N| > 127 * 2^32, so that X_0 stays in [-128, 127] too.
       double r[VEC], mx = 0.0;
 #pragma unroll
       for (int e = 0; e < VEC; ++e) {
@@ -189,26 +190,35 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ Q, cons
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       // ex = floor(log2(mx)) + 1 from the exponent field; means below 2^-900 count as 0
-      const int ex = max(-900, mx > 0.0 ? (int)((__double_as_longlong(mx) >> 52) & 0x7ff) - 1022 : 0);
+      int ex = max(-900, mx > 0.0 ? (int)((__double_as_longlong(mx) >> 52) & 0x7ff) - 1022 : 0);
+      if (__double2ll_rn(mx * __longlong_as_double((int64_t)(1023 + 39 - ex) << 52)) > (127ll << 32)) ++ex;
       if (r0 == 0) {
-        __nv_bfloat16* dst = (isK ? so.ks : so.qs) + ((bh * kScoreSlices) * m.nb + blk) * (int64_t)D + c * VEC;
+        int8_t* dst = (isK ? so.ks : so.qs) + ((bh * kScoreSlices) * m.nb + blk) * (int64_t)kSliceRow + c * VEC;
         const double sc = __longlong_as_double((int64_t)(1023 + 39 - ex) << 52);   // 2^(39-ex)
         long long n[VEC];
 #pragma unroll
         for (int e = 0; e < VEC; ++e) n[e] = __double2ll_rn(r[e] * sc);
 #pragma unroll
-        for (int a = 0; a < kScoreSlices; ++a) {
-          const int sh = 8 * (kScoreSlices - 1 - a);
-          __nv_bfloat16 h[VEC];
+        for (int a = kScoreSlices - 1; a >= 0; --a) {          // digits from the bottom
+          uint32_t word[VEC / 4];
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) {
-            const long long x = sh ? (n[e] + (1ll << (sh - 1))) >> sh : n[e];
-            n[e] -= x << sh;
-            h[e] = __int2bfloat16_rn((int)x);
+          for (int w = 0; w < VEC / 4; ++w) {
+            word[w] = 0;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              long long& x = n[4 * w + b];
+              const long long dgt = a > 0 ? ((x + 128) & 255) - 128 : x;
+              x = (x - dgt) >> 8;
+              word[w] |= ((uint32_t)dgt & 0xffu) << (8 * b);
+            }
           }
-          __nv_bfloat16* d = dst + (int64_t)a * m.nb * D;
-          if (VEC == 8) *reinterpret_cast<uint4*>(d) = *reinterpret_cast<const uint4*>(h);
-          else *reinterpret_cast<uint2*>(d) = *reinterpret_cast<const uint2*>(h);
+          int8_t* d = dst + (int64_t)a * m.nb * kSliceRow;
+          if (VEC == 8) *reinterpret_cast<uint2*>(d) = make_uint2(word[0], word[VEC / 4 - 1]);
+          else *reinterpret_cast<uint32_t*>(d) = word[0];
+          if (D < kSliceRow) {                                    // zero upper half (d = 64)
+            if (VEC == 8) *reinterpret_cast<uint2*>(d + D) = make_uint2(0u, 0u);
+            else *reinterpret_cast<uint32_t*>(d + D) = 0u;
+          }
         }
         if (c == 0) (isK ? so.ek : so.eq)[row] = ex;
       }
@@ -395,7 +405,7 @@ __device__ void topp_select(double* E, int n, double p, uint32_t* w, int lane) {
 
 size_t logits_elems(const Dims& m) { return (size_t)m.BH * m.nb * means_ld(m.nb); }
 
-constexpr int SEL_WARPS = 8;
+constexpr int SEL_WARPS = 4;
 
 // Pairwise (fixed-order) sum of the lane's masked weights, as fp64: at most log2(NE) + 1
 // roundings of fp32 relative error each.
@@ -636,7 +646,7 @@ __device__ void sasa_row(const double* __restrict__ src, const Dims& m, const Sa
 // warps 2w and 2w+1 hold the two rows of a 128-row tile and write its cost, then (register
 // path, sasa.coef > 0) augment each other's slack.
 template <int NE>
-__global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ logits, Dims m, double p,
+__global__ void __launch_bounds__(SEL_WARPS * 32) select_kernel(const double* __restrict__ logits, Dims m, double p,
                                                      int kblocks, ForceCfg fc, SasaCfg sasa,
                                                      uint32_t* __restrict__ bits, int32_t* __restrict__ counts,
                                                      int32_t* __restrict__ tile_cost) {
@@ -697,7 +707,7 @@ static cudaError_t launch_select_t(const double* logits, const Dims& m, double p
   cudaError_t e = cudaFuncSetAttribute(select_kernel<NE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 g((m.nb + SEL_WARPS - 1) / SEL_WARPS, (unsigned)m.BH);
-  select_kernel<NE><<<g, 256, smem, st>>>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost);
+  select_kernel<NE><<<g, SEL_WARPS * 32, smem, st>>>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost);
   return cudaGetLastError();
 }
 

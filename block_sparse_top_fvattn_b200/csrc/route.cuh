@@ -19,17 +19,19 @@ size_t logits_elems(const Dims& m);      // doubles of the fp64 block-score matr
 size_t frame_smem_bytes(const Dims& m);
 size_t schedule_smem_bytes(const Dims& m, int* groups);
 
-// Block means as exact small-integer slices for the tensor-core score GEMM (score_tc.cu): per
-// block a power-of-two exponent and kScoreSlices bf16 planes, [BH][kScoreSlices][nb][d].
+// Block means as exact 8-bit integer slices for the tensor-core score GEMM (score_tc.cu): per
+// block a power-of-two exponent and kScoreSlices int8 planes, [BH][kScoreSlices][nb][kSliceRow]
+// (rows of 128 bytes; for d = 64 the upper half of a row is zero).
 constexpr int kScoreSlices = 5;
+constexpr int kSliceRow = 128;
 struct SliceOut {
-  __nv_bfloat16* qs;
-  __nv_bfloat16* ks;
+  int8_t* qs;
+  int8_t* ks;
   int32_t* eq;
   int32_t* ek;
 };
-cudaError_t launch_score_tc(const __nv_bfloat16* qs, const __nv_bfloat16* ks, const int32_t* eq, const int32_t* ek,
-                            const Dims& m, double scale, double* logits, int32_t* status, int nsm, cudaStream_t st);
+cudaError_t launch_score_tc(const int8_t* qs, const int8_t* ks, const int32_t* eq, const int32_t* ek, const Dims& m,
+                            double scale, double* logits, int32_t* status, int nsm, cudaStream_t st);
 
 // out: 0 = means [row][d] (qo, ko), 1 = score slices and exponents (so), 2 = frame segment sums.
 cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int out, int frame_len,

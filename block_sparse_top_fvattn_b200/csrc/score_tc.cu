@@ -3,22 +3,23 @@
 // accuracy.
 //
 // The pool kernel writes each block mean x (fp64, d values) as a power-of-two scale 2^e with
-// max|x| < 2^e and five slices of integers in [-128, 128] (exact in bf16):
-//     x = 2^e * (X_0 2^-7 + X_1 2^-15 + X_2 2^-23 + X_3 2^-31 + X_4 2^-39) + (residual < 2^(e-40)).
+// max|x| < 2^e and five slices of signed 8-bit integers:
+//     x = 2^e * (X_0 2^-7 + X_1 2^-15 + X_2 2^-23 + X_3 2^-31 + X_4 2^-39) + (residual <= 2^(e-40)).
 // The dot product of two blocks is then a sum over slice pairs (a, b) of integer dot products
 // weighted 2^(e_i + f_j - 14 - 8(a + b)). Pairs of one level l = a + b share a weight, so their
-// sum is accumulated in one fp32 TMEM accumulator; every partial sum is an integer below
-// 5 * d * 128^2 < 2^24 and therefore exact. Levels 0-4 (15 MMA groups) are kept; the dropped
-// ones are below 2^-30 * 2^(e_i + f_j) (a splitting of the operands into small-integer slices
-// whose products the tensor cores compute exactly, in the manner of the Ozaki scheme for
-// accurate matrix products).
+// sum is accumulated in one int32 TMEM accumulator (tcgen05.mma kind::i8, exact; every partial
+// sum is below 5 * d * 128^2 < 2^24). Levels 0-4 (15 MMA groups) are kept; the dropped ones are
+// below 2^-30 * 2^(e_i + f_j) (a splitting of the operands into small-integer slices whose
+// products the tensor cores compute exactly, in the manner of the Ozaki scheme for accurate
+// matrix products).
 //
 // Work: the 128 x 32 output tiles of all heads in (head, row tile, column tile) order, split into
 // one contiguous range per CTA (one persistent CTA per SM), so a CTA loads the five Q slices of a
-// row tile once (160 KB, resident in shared memory) and only reloads them when its range enters
-// the next row tile. Per column tile the five K slices stream through a three-slot ring; one
-// thread issues tcgen05.mma (kind::f16, bf16 -> fp32) into one of two accumulator sets (5 levels
-// x 32 columns at 32-column TMEM offsets); eight epilogue warps drain the other set meanwhile
+// row tile once (80 KB, resident in shared memory; rows of 128 bytes, one 128-byte swizzle
+// span) and only reloads them when its range enters the next row tile. Per column tile the five
+// K slices stream through a ring of two tiles' slots; one thread issues tcgen05.mma (kind::i8,
+// K = 32 per instruction) into one of two accumulator sets (5 levels x 32 columns at 32-column
+// TMEM offsets); eight epilogue warps drain the other set meanwhile
 // (two per TMEM lane quarter, 16 columns each), combine the levels in fp64, stage the tile in
 // shared memory and write the fp64 logit rows coalesced.
 #include <cuda.h>
@@ -34,7 +35,7 @@ namespace fv {
 namespace {
 
 constexpr int kRowsQ = 128, kColsK = 32;
-constexpr int kKSlots = 3;
+constexpr int kKSlots = 2 * kScoreSlices;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = (kEpiWarps + 2) * 32;          // + producer warp + MMA warp
 constexpr int kLevelCols = kScoreSlices * kColsK;       // one accumulator set: 160 TMEM columns
@@ -42,11 +43,9 @@ constexpr uint32_t kWaitLimit = 1u << 22;
 
 template <int D>
 struct ScLayout {
-  static constexpr int kChunks = D / 64;
-  static constexpr int kQChunk = kRowsQ * 128;                  // [128 rows x 64 dims] bf16 = 16 KB
-  static constexpr int kQSlice = kChunks * kQChunk;
-  static constexpr int kKChunk = kColsK * 128;                  // [32 rows x 64 dims] bf16 = 4 KB
-  static constexpr int kKSlot = kChunks * kKChunk;              // one K slice of one column tile
+  static constexpr int kSteps = D / 32;                         // K = 32 bytes per MMA
+  static constexpr int kQSlice = kRowsQ * kSliceRow;            // [128 rows x 128 bytes] = 16 KB
+  static constexpr int kKSlot = kColsK * kSliceRow;             // one K slice of one column tile: 4 KB
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kScoreSlices * kQSlice;
   static constexpr int kOffStage = kOffK + kKSlots * kKSlot;
@@ -144,10 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc::mbar_expect_tx(&bars->q_full, kScoreSlices * L::kQSlice);
           for (int a = 0; a < kScoreSlices; ++a)
-            for (int c = 0; c < L::kChunks; ++c)
-              for (int h = 0; h < 2; ++h)
-                tc::tma_load_3d(smem + L::kOffQ + a * L::kQSlice + c * L::kQChunk + h * 64 * 128, &tmQ, &bars->q_full,
-                                c * 64, i0 + h * 64, (int)(bh * kScoreSlices + a));
+            tc::tma_load_3d(smem + L::kOffQ + a * L::kQSlice, &tmQ, &bars->q_full, 0, i0, (int)(bh * kScoreSlices + a));
           cur = rtile;
           ++qc;
         }
@@ -159,9 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc::mbar_expect_tx(&bars->k_full[s], L::kKSlot);
-          for (int c = 0; c < L::kChunks; ++c)
-            tc::tma_load_3d(smem + L::kOffK + s * L::kKSlot + c * L::kKChunk, &tmK, &bars->k_full[s], c * 64, j0,
-                            (int)(bh * kScoreSlices + b));
+          tc::tma_load_3d(smem + L::kOffK + s * L::kKSlot, &tmK, &bars->k_full[s], 0, j0, (int)(bh * kScoreSlices + b));
         }
         if (!ok) {
           atomicCAS(&bars->abort, 0, 2);
@@ -174,9 +168,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------------- MMAs
       // Column tile j (local index) goes to accumulator set j % 2: level a+b += Q_a K_b^T for
       // a + b < 5. With b outermost, b = 0 touches every level first (a = level), so those MMAs
-      // (first chunk, first K16 step) overwrite. The closing commit runs on every path, and the
-      // thread waits for it, so no MMA is in flight when TMEM is released.
-      constexpr uint32_t idesc = tc::idesc_bf16_f32(kRowsQ, kColsK, 0, 0);
+      // (first K32 step) overwrite. The closing commit runs on every path, and the thread waits
+      // for it, so no MMA is in flight when TMEM is released.
+      constexpr uint32_t idesc = tc::idesc_s8_s32(kRowsQ, kColsK);
       // Shared-memory descriptors are linear in the start address (bits 0-13 hold address >> 4,
       // and every operand lies below 256 KB), so they are made once and offset by constants.
       const uint64_t qdesc0 = tc::smem_desc_sw128(tc::smem_u32(smem + L::kOffQ), 16, 1024);
@@ -205,11 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int a = 0; a < kScoreSlices; ++a) {
             if (a + b >= kScoreSlices) continue;
 #pragma unroll
-            for (int c = 0; c < L::kChunks; ++c)
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                tc::mma_f16(dbase + (a + b) * kColsK, qdesc0 + ((a * L::kQSlice + c * L::kQChunk + kk * 32) >> 4),
-                            kd + ((c * L::kKChunk + kk * 32) >> 4), idesc, (b > 0 || c > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < L::kSteps; ++kk)
+              tc::mma_i8(dbase + (a + b) * kColsK, qdesc0 + ((a * L::kQSlice + kk * 32) >> 4), kd + ((kk * 32) >> 4),
+                         idesc, (b > 0 || kk > 0) ? 1u : 0u);
           }
           tc::mma_commit(&bars->k_empty[s]);
         }
@@ -254,9 +246,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         // levels combined from the finest: v = A_0 + 2^-8 (A_1 + 2^-8 (A_2 + ...))
-        double v = (double)__uint_as_float(acc[kScoreSlices - 1][e]);
+        double v = (double)(int32_t)acc[kScoreSlices - 1][e];
 #pragma unroll
-        for (int l = kScoreSlices - 2; l >= 0; --l) v = fma(v, 0x1p-8, (double)__uint_as_float(acc[l][e]));
+        for (int l = kScoreSlices - 2; l >= 0; --l) v = fma(v, 0x1p-8, (double)(int32_t)acc[l][e]);
         const int k = ei + __shfl_sync(0xffffffffu, ej_l, e) - 14;
         const int col = half * 16 + e;
         stage[r * kColsK + ((col + r) & (kColsK - 1))] = (v * scale) * pow2(max(-1000, min(1000, k)));
@@ -286,13 +278,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D>
-cudaError_t launch_score_tc_d(const __nv_bfloat16* qs, const __nv_bfloat16* ks, const int32_t* eq,
-                              const int32_t* ek, const Dims& m, double scale, double* logits, int32_t* status,
-                              int nsm, cudaStream_t st) {
+cudaError_t launch_score_tc_d(const int8_t* qs, const int8_t* ks, const int32_t* eq, const int32_t* ek, const Dims& m,
+                              double scale, double* logits, int32_t* status, int nsm, cudaStream_t st) {
   CUtensorMap mq, mk;
   const uint64_t planes = (uint64_t)m.BH * kScoreSlices;
-  if (!make_map_bf16_3d(&mq, qs, (uint64_t)D, (uint64_t)m.nb, planes, 64) ||
-      !make_map_bf16_3d(&mk, ks, (uint64_t)D, (uint64_t)m.nb, planes, kColsK))
+  if (!make_map_i8_3d(&mq, qs, (uint64_t)kSliceRow, (uint64_t)m.nb, planes, kRowsQ) ||
+      !make_map_i8_3d(&mk, ks, (uint64_t)kSliceRow, (uint64_t)m.nb, planes, kColsK))
     return cudaErrorInvalidValue;
   const size_t smem = ScLayout<D>::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -305,8 +296,8 @@ cudaError_t launch_score_tc_d(const __nv_bfloat16* qs, const __nv_bfloat16* ks, 
 
 }  // namespace
 
-cudaError_t launch_score_tc(const __nv_bfloat16* qs, const __nv_bfloat16* ks, const int32_t* eq, const int32_t* ek,
-                            const Dims& m, double scale, double* logits, int32_t* status, int nsm, cudaStream_t st) {
+cudaError_t launch_score_tc(const int8_t* qs, const int8_t* ks, const int32_t* eq, const int32_t* ek, const Dims& m,
+                            double scale, double* logits, int32_t* status, int nsm, cudaStream_t st) {
   if (m.d == 128) return launch_score_tc_d<128>(qs, ks, eq, ek, m, scale, logits, status, nsm, st);
   return launch_score_tc_d<64>(qs, ks, eq, ek, m, scale, logits, status, nsm, st);
 }

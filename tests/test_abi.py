@@ -56,8 +56,9 @@ def test_sizes_on_host(lib):
     s = shape(S=65)                      # nb = 2 with a 1-token tail
     assert lib.fvattn_num_tiles(ctypes.byref(s)) == 2 * 1
     ws = lib.fvattn_route_workspace_bytes(ctypes.byref(shape(S=1000)), ctypes.byref(cfg()))
-    means = 2 * 16 * 128 * 8
-    assert ws >= 2 * means + 2 * 16 * 1 * 4 + 2 * 16 * 4
+    # Q and K score slices (5 int8 planes of 128-byte rows), fp64 logits (rows of 32), bitmasks
+    slices = 2 * 5 * 16 * 128
+    assert ws >= 2 * slices + 2 * 16 * 32 * 8 + 2 * 16 * 1 * 4 + 2 * 16 * 4
     wf = lib.fvattn_route_workspace_bytes(ctypes.byref(shape(S=1000)),
                                           ctypes.byref(cfg(mode=1, frame_len=250, topk_frames=2)))
     assert wf > ws
