@@ -424,10 +424,13 @@ __device__ __forceinline__ double lane_sum(const float (&e)[NE], const uint32_t 
 
 // The Top-p cut of one row with its weights in registers (NE per lane, element j = lane + 32 i),
 // the same rule as topp_select: weights e_j = 2^((s_j - max) log2 e) from the SFU on fp64
-// logit differences, masses compared with p * sum(e). Peaked rows are cut by max extraction
-// (REDUX on the fp32 key = the weight's bits, lowest index on ties); rows with more than
-// kExtract weights above 1/64 go straight to a bisection over the 32-bit key space. Lane sums
-// are pairwise in fp32 and folded across the warp in fp64 in a fixed order (deterministic).
+// logit differences, masses compared with p * sum(e). Both ways below find the cut key T (the
+// fp32 key = the weight's bits) and the mass above it; the row then keeps every key > T and, in
+// ascending index, as many keys == T as the mass needs. Peaked rows peel key values from the
+// top (REDUX max over the lanes' largest remaining keys, all copies of a value at once) until
+// the mass reaches p; rows with more than kExtract weights above 1/64, or not done after
+// kExtract values, take a bisection over the 32-bit key space. Lane sums are pairwise in fp32
+// and folded across the warp in fp64 in a fixed order (deterministic).
 template <int NE>
 __device__ void topp_select_reg(const double* __restrict__ src, int n, double p, uint32_t* w, int lane) {
   const int nw = (n + 31) / 32;
@@ -462,52 +465,58 @@ __device__ void topp_select_reg(const double* __restrict__ src, int n, double p,
   const double P = p * z;
   big = warp_sum(big);
 
-  uint64_t taken = 0;
+  // T: the key of the cut; above: the mass of the keys > T.
+  uint32_t T = 0;
+  double above = 0.0;
   bool done = false;
   if (big <= kExtract) {
-    uint32_t bkey = 0;
-    int bslot = -1;
-    auto rescan = [&]() {
-      bkey = 0;
-      bslot = -1;
-#pragma unroll
-      for (int i = 0; i < NE; ++i)
-        if (lane + 32 * i < n && !((taken >> i) & 1ull) && (bslot < 0 || k[i] > bkey)) { bkey = k[i]; bslot = i; }
-    };
-    rescan();
-    double acc = 0.0;
-    for (int it = 0; it < kExtract && !done; ++it) {
-      const uint32_t gk = __reduce_max_sync(0xffffffffu, bslot >= 0 ? bkey : 0u);
-      const uint32_t cand = (bslot >= 0 && bkey == gk) ? (uint32_t)(lane + 32 * bslot) : 0xffffffffu;
-      const uint32_t gj = __reduce_min_sync(0xffffffffu, cand);
-      if (gj == 0xffffffffu) break;
-      acc += (double)__uint_as_float(gk);
-      if ((int)(gj & 31) == lane) {
-        taken |= 1ull << (gj >> 5);
-        rescan();
-      }
-      done = acc >= P;
-    }
-  }
-  if (done) {
+    // Peel the largest remaining key value, with all its copies, until the mass reaches P. Each
+    // lane keeps a copy of its keys with the peeled ones zeroed and their maximum.
+    uint32_t kx[NE];
+    uint32_t lmax = 0;
 #pragma unroll
     for (int i = 0; i < NE; ++i) {
-      const uint32_t word = __ballot_sync(0xffffffffu, (taken >> i) & 1ull);
-      if (lane == 0 && i < nw) w[i] = word;
+      kx[i] = k[i];
+      lmax = max(lmax, k[i]);
     }
-    __syncwarp();
-    return;
+    double acc = 0.0;
+    for (int it = 0; it < kExtract; ++it) {
+      const uint32_t gk = __reduce_max_sync(0xffffffffu, lmax);
+      if (gk == 0u) break;                       // only zero weights left
+      int cnt = 0;
+      if (lmax == gk) {
+        uint32_t nm = 0;
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+          const bool eq = kx[i] == gk;
+          cnt += eq;
+          kx[i] = eq ? 0u : kx[i];
+          nm = max(nm, kx[i]);
+        }
+        lmax = nm;
+      }
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      above = acc;
+      acc += (double)cnt * (double)__uint_as_float(gk);
+      if (acc >= P) {
+        T = gk;
+        done = true;
+        break;
+      }
+    }
   }
-  // Bisection: largest T with mass{key >= T} >= P. Weights are at most 1, so keys <= 0x3f800000.
-  uint32_t lo = 0, hi = 0x3f800001u;
-  while (hi - lo > 1) {
-    const uint32_t mid = lo + ((hi - lo) >> 1);
-    const double sm = warp_sum_d(lane_sum(e, k, mid, false));
-    if (sm >= P) lo = mid;
-    else hi = mid;
+  if (!done) {
+    // Bisection: largest T with mass{key >= T} >= P. Weights are at most 1, so keys <= 0x3f800000.
+    uint32_t lo = 0, hi = 0x3f800001u;
+    while (hi - lo > 1) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      const double sm = warp_sum_d(lane_sum(e, k, mid, false));
+      if (sm >= P) lo = mid;
+      else hi = mid;
+    }
+    T = lo;
+    above = warp_sum_d(lane_sum(e, k, T, true));
   }
-  const uint32_t T = lo;
-  double above = warp_sum_d(lane_sum(e, k, T, true));
   const double tval = (double)__uint_as_float(T);
 #pragma unroll
   for (int i = 0; i < NE; ++i) {
