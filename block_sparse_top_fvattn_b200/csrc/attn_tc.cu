@@ -13,11 +13,16 @@
 //   P = exp2(S*c - m)    one thread per row reads its TMEM lane, masks the half-tile whose
 //                        list lacks j and the keys >= S, keeps a running max m that is only
 //                        raised (with a rescale of O in TMEM) when it grows by more than
-//                        2^8, and writes P as bf16 into shared memory in the MMA's layout
-//   O += P V_j           tcgen05.mma M=128 N=d K=64, V MN-major, O accumulated in TMEM
+//                        2^8, and writes P as bf16 pairs over its S buffer in TMEM
+//   O += P V_j           tcgen05.mma M=128 N=d K=64, A = P read from TMEM, V MN-major, O
+//                        accumulated in TMEM
 // Warp roles: warp 0 issues TMA loads (lane 0: Q once per tile and K_j, lane 1: V_j, each into
 // its own 2-stage ring, so a K stage is reloaded as soon as its S MMA is done),
 // warp 1 allocates TMEM and issues the MMAs, warps 2-5 do softmax and the epilogue.
+// Every mbarrier wait of the MMA-issuing thread stalls its MMA stream for a few hundred cycles
+// even when the phase is already complete (measured), so that thread waits only twice per step:
+// once for K_j (whose barrier also publishes the step record) and once for P_j together with
+// V_j (one barrier); coincident events share one barrier and one commit.
 // Every mbarrier wait is bounded; a wait that runs out sets an abort flag, every role
 // unwinds, TMEM is freed and FVATTN_ERR_TIMEOUT is written to the device status word.
 #include <cuda.h>
@@ -33,6 +38,7 @@ namespace fv {
 namespace {
 
 constexpr int NS = 2;                        // K/V pipeline stages (two CTAs share an SM)
+static_assert(NS == 2, "the stage of a step doubles as its S / P buffer index");
 constexpr uint32_t kWaitLimit = 1u << 22;    // polls of a bounded wait (seconds, not minutes)
 constexpr float kRescaleLog2 = 8.0f;         // raise the running max only when it grows by > 2^8
 
@@ -57,7 +63,13 @@ constexpr int NI = 8;        // step records in flight
 
 struct TcBars {
   uint64_t q_full, q_empty;
-  uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
+  uint64_t k_full[NS];
+  // With NS == 2 the K/V stage and the S buffer of a step have the same index b = step & 1, so
+  // one barrier serves each pair of events that happen together:
+  //   s_full[b]:  S of the step done (softmax may read it; its K stage may be refilled)
+  //   p_full[b]:  P written by the four softmax warps AND V landed (the V loader's
+  //               arrive.expect_tx is the fifth arrival)
+  //   pv_done[b]: P.V done (O is stable; the V stage may be refilled)
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t o_full, o_empty;
   uint64_t sched_full[2], sched_empty[2];
@@ -176,13 +188,10 @@ __global__ void __launch_bounds__(192, 2)
     tc::mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < NS; ++s) {
       tc::mbar_init(&bars->k_full[s], 1);
-      tc::mbar_init(&bars->k_empty[s], 1);
-      tc::mbar_init(&bars->v_full[s], 1);
-      tc::mbar_init(&bars->v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->s_full[s], 1);
-      tc::mbar_init(&bars->p_full[s], 4);
+      tc::mbar_init(&bars->p_full[s], 5);
       tc::mbar_init(&bars->pv_done[s], 1);
       tc::mbar_init(&bars->sched_full[s], 1);
       tc::mbar_init(&bars->sched_empty[s], 6);    // V loader, MMA thread, four softmax warps
@@ -255,7 +264,7 @@ __global__ void __launch_bounds__(192, 2)
           bars->step_code[g % NI] = code;
           tc::mbar_arrive(&bars->info_full[g % NI]);
           const int st = g % NS;
-          if (!tc::mbar_wait(&bars->k_empty[st], ((g / NS) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 3); ok = false; break; }
+          if (!tc::mbar_wait(&bars->s_full[st], ((g / NS) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 3); ok = false; break; }
           tc::mbar_expect_tx(&bars->k_full[st], L::kKBytes);
           for (int c = 0; c < D / 64; ++c)
             tc::tma_load_3d(sK + st * L::kKBytes + c * L::kKVChunk, &tmK, &bars->k_full[st], c * 64, j * kBlock, (int)bh);
@@ -280,10 +289,10 @@ __global__ void __launch_bounds__(192, 2)
         bool ok = true;
         while (mg.next(j, mask, ea, eb)) {
           const int st = g % NS;
-          if (!tc::mbar_wait(&bars->v_empty[st], ((g / NS) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 16); ok = false; break; }
-          tc::mbar_expect_tx(&bars->v_full[st], L::kKBytes);
+          if (!tc::mbar_wait(&bars->pv_done[st], ((g / NS) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 16); ok = false; break; }
+          tc::mbar_expect_tx(&bars->p_full[st], L::kKBytes);
           for (int c = 0; c < D / 64; ++c)
-            tc::tma_load_3d(sV + st * L::kKBytes + c * L::kKVChunk, &tmV, &bars->v_full[st], c * 64, j * kBlock, (int)bh);
+            tc::tma_load_3d(sV + st * L::kKBytes + c * L::kKVChunk, &tmV, &bars->p_full[st], c * 64, j * kBlock, (int)bh);
           ++g;
         }
         if (!ok) break;
@@ -304,7 +313,6 @@ __global__ void __launch_bounds__(192, 2)
         const int pb = gs & 1, st = gs % NS;
         if (!tc::mbar_wait(&bars->p_full[pb], (gs >> 1) & 1, abort, kWaitLimit)) return false;
         if (first && !tc::mbar_wait(&bars->o_empty, (n & 1) ^ 1, abort, kWaitLimit)) return false;
-        if (!tc::mbar_wait(&bars->v_full[st], (gs / NS) & 1, abort, kWaitLimit)) return false;
         tc::fence_after_sync();
         const uint32_t vaddr = vaddr0 + st * L::kKBytes;
 #pragma unroll
@@ -313,7 +321,6 @@ __global__ void __launch_bounds__(192, 2)
           tc::mma_f16_tmem_a(tbase + L::kColO, tbase + pb * kBlock + kk * 8, b, idO, (first && kk == 0) ? 0u : 1u);
         }
         tc::mma_commit(&bars->pv_done[pb]);
-        tc::mma_commit(&bars->v_empty[st]);
         return true;
       };
       for (;; ++n) {
@@ -327,8 +334,10 @@ __global__ void __launch_bounds__(192, 2)
         for (bool last = false; !last;) {
           const uint32_t gi = g + i;
           const int st = gi % NS, sb = gi & 1;
-          if (!tc::mbar_wait(&bars->info_full[gi % NI], (gi / NI) & 1, abort, kWaitLimit) ||
-              !tc::mbar_wait(&bars->k_full[st], (gi / NS) & 1, abort, kWaitLimit)) {
+          // The loader writes the step record before its arrive.expect_tx on k_full (a release),
+          // so the record is visible once k_full completes; this thread does not wait on
+          // info_full (every mbarrier wait here stalls the MMA stream).
+          if (!tc::mbar_wait(&bars->k_full[st], (gi / NS) & 1, abort, kWaitLimit)) {
             fail(bars, 6);
             ok = false;
             break;
@@ -343,8 +352,7 @@ __global__ void __launch_bounds__(192, 2)
             const uint64_t b = tc::smem_desc_sw128(kaddr + c * L::kKVChunk + off, 16, 1024);
             tc::mma_f16(tbase + sb * kBlock, a, b, idS, kk > 0 ? 1u : 0u);
           }
-          tc::mma_commit(&bars->s_full[sb]);
-          tc::mma_commit(&bars->k_empty[st]);       // K_j may be replaced once S_i is done
+          tc::mma_commit(&bars->s_full[sb]);        // also frees K stage st (== sb)
           if (i > 0 && !pv(gi - 1, i == 1)) { fail(bars, 7); ok = false; break; }
           ++i;
         }

@@ -16,12 +16,12 @@
 // Work: the 128 x 32 output tiles of all heads in (head, row tile, column tile) order, split into
 // one contiguous range per CTA (one persistent CTA per SM), so a CTA loads the five Q slices of a
 // row tile once (80 KB, resident in shared memory; rows of 128 bytes, one 128-byte swizzle
-// span) and only reloads them when its range enters the next row tile. Per column tile the five
-// K slices stream through a ring of two tiles' slots; one thread issues tcgen05.mma (kind::i8,
-// K = 32 per instruction) into one of two accumulator sets (5 levels x 32 columns at 32-column
-// TMEM offsets); eight epilogue warps drain the other set meanwhile
-// (two per TMEM lane quarter, 16 columns each), combine the levels in fp64, stage the tile in
-// shared memory and write the fp64 logit rows coalesced.
+// span) and only reloads them when its range enters the next row tile. The five K slices of a
+// column tile stream through a ring of three tiles (one barrier per tile); one thread issues
+// tcgen05.mma (kind::i8, K = 32 per instruction) into one of two accumulator sets (5 levels x 32
+// columns at 32-column TMEM offsets); sixteen epilogue warps drain the other set meanwhile (four
+// per TMEM lane quarter, 8 columns each), combine the levels in fp64 and write each thread's 8
+// consecutive logits of its row (64 bytes) straight to global memory.
 #include <cuda.h>
 #include <math.h>
 
@@ -35,8 +35,9 @@ namespace fv {
 namespace {
 
 constexpr int kRowsQ = 128, kColsK = 32;
-constexpr int kKSlots = 2 * kScoreSlices;
-constexpr int kEpiWarps = 8;
+constexpr int kKTiles = 3;                              // K ring: three column tiles of five slices
+constexpr int kEpiWarps = 16;
+constexpr int kEpiCols = kColsK / (kEpiWarps / 4);      // columns of a tile per epilogue thread
 constexpr int kThreads = (kEpiWarps + 2) * 32;          // + producer warp + MMA warp
 constexpr int kLevelCols = kScoreSlices * kColsK;       // one accumulator set: 160 TMEM columns
 constexpr uint32_t kWaitLimit = 1u << 22;
@@ -48,14 +49,14 @@ struct ScLayout {
   static constexpr int kKSlot = kColsK * kSliceRow;             // one K slice of one column tile: 4 KB
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kScoreSlices * kQSlice;
-  static constexpr int kOffStage = kOffK + kKSlots * kKSlot;
-  static constexpr int kOffBar = kOffStage + kRowsQ * kColsK * 8;
+  static constexpr int kKTile = kScoreSlices * kKSlot;         // the five K slices of one column tile
+  static constexpr int kOffBar = kOffK + kKTiles * kKTile;
   static constexpr int kBytes = kOffBar + 256;
 };
 
 struct ScBars {
   uint64_t q_full, q_empty;
-  uint64_t k_full[kKSlots], k_empty[kKSlots];
+  uint64_t k_full[kKTiles], k_empty[kKTiles];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
@@ -65,22 +66,32 @@ struct ScBars {
 // 2^k for the exponent range of the logits (a normal double), exactly.
 __device__ __forceinline__ double pow2(int k) { return __longlong_as_double((long long)(1023 + k) << 52); }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); }
-
-// A barrier of the epilogue warps that also returns whether every one of their threads passed
-// true, so that they take the same branch (leaving the tile loop) together.
-__device__ __forceinline__ bool epi_all(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, %2, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v), "n"(kEpiWarps * 32)
-      : "memory");
-  return r != 0;
+// An int32 as a double, exactly, on the fp64 pipe: the bits 0x43300000:(x + 2^31) are the double
+// 2^52 + x + 2^31, from which the constant 2^52 + 2^31 is subtracted without rounding.
+__device__ __forceinline__ double i32_to_f64(uint32_t x) {
+  return __hiloint2double(0x43300000, (int)(x ^ 0x80000000u)) - 4503601774854144.0;
 }
+
+// Walks the tiles of a CTA's range in (head, row tile, column tile) order without divisions.
+struct TileCursor {
+  int64_t bh;
+  int rt, ct, nrt, nct;
+  __device__ TileCursor(int64_t t, int nrt_, int nct_) : nrt(nrt_), nct(nct_) {
+    const int64_t rtile = t / nct;
+    ct = (int)(t - rtile * nct);
+    bh = rtile / nrt;
+    rt = (int)(rtile - bh * nrt);
+  }
+  __device__ void next() {
+    if (++ct == nct) {
+      ct = 0;
+      if (++rt == nrt) {
+        rt = 0;
+        ++bh;
+      }
+    }
+  }
+};
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -92,7 +103,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   ScBars* bars = reinterpret_cast<ScBars*>(smem + L::kOffBar);
-  double* stage = reinterpret_cast<double*>(smem + L::kOffStage);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort = &bars->abort;
 
@@ -100,12 +110,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nrt = (m.nb + kRowsQ - 1) / kRowsQ, nct = (m.nb + kColsK - 1) / kColsK;
   const int64_t T = m.BH * nrt * nct;
   const int64_t t_begin = T * blockIdx.x / gridDim.x, t_end = T * (blockIdx.x + 1) / gridDim.x;
-  auto row_tile = [&](int64_t t) { return t / nct; };           // bh * nrt + rt
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&bars->q_full, 1);
     tc::mbar_init(&bars->q_empty, 1);
-    for (int s = 0; s < kKSlots; ++s) {
+    for (int s = 0; s < kKTiles; ++s) {
       tc::mbar_init(&bars->k_full[s], 1);
       tc::mbar_init(&bars->k_empty[s], 1);
     }
@@ -129,13 +138,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kEpiWarps) {
     if (lane == 0) {
       // ---------------------------------------------------------------- loads
-      uint32_t kc = 0, qc = 0;
-      int64_t cur = -1;
-      for (int64_t t = t_begin; t < t_end; ++t) {
-        const int64_t rtile = row_tile(t);
-        const int64_t bh = rtile / nrt;
-        const int i0 = (int)(rtile - bh * nrt) * kRowsQ, j0 = (int)(t - rtile * nct) * kColsK;
-        if (rtile != cur) {
+      uint32_t qc = 0, kph = 0;
+      int s = 0;
+      TileCursor tcur(t_begin, nrt, nct);
+      for (int64_t t = t_begin; t < t_end; ++t, tcur.next()) {
+        const int64_t bh = tcur.bh;
+        const int i0 = tcur.rt * kRowsQ, j0 = tcur.ct * kColsK;
+        if (t == t_begin || tcur.ct == 0) {
           // the previous row tile's MMAs are done with the Q slices before they are replaced
           if (qc > 0 && !tc::mbar_wait(&bars->q_empty, (qc - 1) & 1, abort, kWaitLimit)) {
             atomicCAS(&bars->abort, 0, 1);
@@ -144,22 +153,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::mbar_expect_tx(&bars->q_full, kScoreSlices * L::kQSlice);
           for (int a = 0; a < kScoreSlices; ++a)
             tc::tma_load_3d(smem + L::kOffQ + a * L::kQSlice, &tmQ, &bars->q_full, 0, i0, (int)(bh * kScoreSlices + a));
-          cur = rtile;
           ++qc;
         }
-        bool ok = true;
-        for (int b = 0; b < kScoreSlices; ++b, ++kc) {
-          const int s = kc % kKSlots;
-          if (!tc::mbar_wait(&bars->k_empty[s], ((kc / kKSlots) & 1) ^ 1, abort, kWaitLimit)) {
-            ok = false;
-            break;
-          }
-          tc::mbar_expect_tx(&bars->k_full[s], L::kKSlot);
-          tc::tma_load_3d(smem + L::kOffK + s * L::kKSlot, &tmK, &bars->k_full[s], 0, j0, (int)(bh * kScoreSlices + b));
-        }
-        if (!ok) {
+        // the five K slices of the column tile under one barrier
+        if (!tc::mbar_wait(&bars->k_empty[s], kph ^ 1, abort, kWaitLimit)) {
           atomicCAS(&bars->abort, 0, 2);
           break;
+        }
+        tc::mbar_expect_tx(&bars->k_full[s], L::kKTile);
+        for (int b = 0; b < kScoreSlices; ++b)
+          tc::tma_load_3d(smem + L::kOffK + s * L::kKTile + b * L::kKSlot, &tmK, &bars->k_full[s], 0, j0,
+                          (int)(bh * kScoreSlices + b));
+        if (++s == kKTiles) {
+          s = 0;
+          kph ^= 1;
         }
       }
     }
@@ -175,98 +182,106 @@ __global__ void __launch_bounds__(kThreads, 1)
       // and every operand lies below 256 KB), so they are made once and offset by constants.
       const uint64_t qdesc0 = tc::smem_desc_sw128(tc::smem_u32(smem + L::kOffQ), 16, 1024);
       const uint64_t kdesc0 = tc::smem_desc_sw128(tc::smem_u32(smem + L::kOffK), 16, 1024);
-      uint32_t kc = 0, qc = 0;
-      int64_t cur = -1;
+      uint32_t qc = 0, kph = 0;
+      int s = 0;
       bool ok = true;
-      for (int64_t t = t_begin; ok && t < t_end; ++t) {
+      TileCursor tcur(t_begin, nrt, nct);
+      for (int64_t t = t_begin; ok && t < t_end; ++t, tcur.next()) {
         const uint32_t j = (uint32_t)(t - t_begin), buf = j & 1;
-        const int64_t rtile = row_tile(t);
-        if (rtile != cur) {
+        if (t == t_begin || tcur.ct == 0) {
           if (!tc::mbar_wait(&bars->q_full, qc & 1, abort, kWaitLimit)) { ok = false; break; }
-          cur = rtile;
           ++qc;
         }
-        if (!tc::mbar_wait(&bars->acc_empty[buf], ((j >> 1) & 1) ^ 1, abort, kWaitLimit)) { ok = false; break; }
+        // Two waits per tile: every mbarrier wait of this thread stalls the MMA stream for a
+        // few hundred cycles even when the phase is already complete.
+        if (!tc::mbar_wait(&bars->acc_empty[buf], ((j >> 1) & 1) ^ 1, abort, kWaitLimit) ||
+            !tc::mbar_wait(&bars->k_full[s], kph, abort, kWaitLimit)) {
+          ok = false;
+          break;
+        }
         tc::fence_after_sync();
         const uint32_t dbase = tbase + buf * kLevelCols;
+        const uint64_t kd0 = kdesc0 + (uint64_t)((s * L::kKTile) >> 4);
 #pragma unroll
-        for (int b = 0; b < kScoreSlices; ++b, ++kc) {
-          const int s = kc % kKSlots;
-          if (!tc::mbar_wait(&bars->k_full[s], (kc / kKSlots) & 1, abort, kWaitLimit)) { ok = false; break; }
-          tc::fence_after_sync();
-          const uint64_t kd = kdesc0 + (uint64_t)((s * L::kKSlot) >> 4);
+        for (int b = 0; b < kScoreSlices; ++b) {
 #pragma unroll
           for (int a = 0; a < kScoreSlices; ++a) {
             if (a + b >= kScoreSlices) continue;
 #pragma unroll
             for (int kk = 0; kk < L::kSteps; ++kk)
-              tc::mma_i8(dbase + (a + b) * kColsK, qdesc0 + ((a * L::kQSlice + kk * 32) >> 4), kd + ((kk * 32) >> 4),
-                         idesc, (b > 0 || kk > 0) ? 1u : 0u);
+              tc::mma_i8(dbase + (a + b) * kColsK, qdesc0 + ((a * L::kQSlice + kk * 32) >> 4),
+                         kd0 + ((b * L::kKSlot + kk * 32) >> 4), idesc, (b > 0 || kk > 0) ? 1u : 0u);
           }
-          tc::mma_commit(&bars->k_empty[s]);
         }
-        if (!ok) break;
+        tc::mma_commit(&bars->k_empty[s]);
+        if (++s == kKTiles) {
+          s = 0;
+          kph ^= 1;
+        }
         tc::mma_commit(&bars->acc_full[buf]);
-        if (t + 1 == t_end || row_tile(t + 1) != rtile) tc::mma_commit(&bars->q_empty);
+        if (t + 1 == t_end || tcur.ct + 1 == nct) tc::mma_commit(&bars->q_empty);
       }
       if (!ok) atomicCAS(&bars->abort, 0, 3);
       tc::mma_commit(&bars->drain);
       tc::mbar_wait(&bars->drain, 0, abort, kWaitLimit);
     }
   } else {
-    // ------------------------------------------------------------------ epilogue (warps 0-7)
-    const int quarter = warp & 3, half = warp >> 2;
+    // ------------------------------------------------------------------ epilogue (warps 0-15)
+    // A warp leaves on its own when a wait runs out or another role aborted: no barrier joins
+    // the epilogue warps inside the loop. The column exponents of the next tile are loaded one
+    // tile ahead.
+    const int quarter = warp & 3, part = warp >> 2;
     const int r = quarter * 32 + lane;                           // tile row == TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    int64_t cur = -1;
+    auto col_exp = [&](const TileCursor& c) -> int {             // exponent of column lane & 7
+      const int jl = c.ct * kColsK + part * kEpiCols + (lane & (kEpiCols - 1));
+      return jl < m.nb ? ek[c.bh * m.nb + jl] : 0;
+    };
     int ei = 0;
-    for (int64_t t = t_begin; t < t_end; ++t) {
+    TileCursor tcur(t_begin, nrt, nct), tnext = tcur;
+    int ej_next = t_begin < t_end ? col_exp(tcur) : 0;
+    for (int64_t t = t_begin; t < t_end; ++t, tcur.next()) {
       const uint32_t j = (uint32_t)(t - t_begin), buf = j & 1;
-      const int64_t rtile = row_tile(t);
-      const int64_t bh = rtile / nrt;
-      const int i0 = (int)(rtile - bh * nrt) * kRowsQ, j0 = (int)(t - rtile * nct) * kColsK;
-      if (rtile != cur) {
-        ei = i0 + r < m.nb ? eq[bh * m.nb + i0 + r] : 0;
-        cur = rtile;
-      }
-      // the 16 column exponents of this warp's half, one per lane 0-15
-      const int jl = j0 + half * 16 + (lane & 15);
-      const int ej_l = jl < m.nb ? ek[bh * m.nb + jl] : 0;
+      const int64_t bh = tcur.bh;
+      const int i0 = tcur.rt * kRowsQ, j0 = tcur.ct * kColsK;
+      if (t == t_begin || tcur.ct == 0) ei = i0 + r < m.nb ? eq[bh * m.nb + i0 + r] : 0;
+      const int ej_l = ej_next;
+      tnext.next();
+      if (t + 1 < t_end) ej_next = col_exp(tnext);
       const bool ready = tc::mbar_wait(&bars->acc_full[buf], (j >> 1) & 1, abort, kWaitLimit);
-      if (!epi_all(ready && !*abort)) break;                      // every epilogue warp leaves together
+      if (!ready || *abort) break;
       tc::fence_after_sync();
-      uint32_t acc[kScoreSlices][16];
+      uint32_t acc[kScoreSlices][kEpiCols];
 #pragma unroll
       for (int l = 0; l < kScoreSlices; ++l)
-        tc::tmem_ld16(tbase + lane_off + buf * kLevelCols + l * kColsK + half * 16, acc[l]);
+        tc::tmem_ld8(tbase + lane_off + buf * kLevelCols + l * kColsK + part * kEpiCols, acc[l]);
       tc::tmem_ld_wait();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&bars->acc_empty[buf]);     // the set can take the next tile
+      double out[kEpiCols];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
+      for (int e = 0; e < kEpiCols; ++e) {
         // levels combined from the finest: v = A_0 + 2^-8 (A_1 + 2^-8 (A_2 + ...))
-        double v = (double)(int32_t)acc[kScoreSlices - 1][e];
+        double v = i32_to_f64(acc[kScoreSlices - 1][e]);
 #pragma unroll
-        for (int l = kScoreSlices - 2; l >= 0; --l) v = fma(v, 0x1p-8, (double)(int32_t)acc[l][e]);
+        for (int l = kScoreSlices - 2; l >= 0; --l) v = fma(v, 0x1p-8, i32_to_f64(acc[l][e]));
         const int k = ei + __shfl_sync(0xffffffffu, ej_l, e) - 14;
-        const int col = half * 16 + e;
-        stage[r * kColsK + ((col + r) & (kColsK - 1))] = (v * scale) * pow2(max(-1000, min(1000, k)));
+        out[e] = (v * scale) * pow2(max(-1000, min(1000, k)));
       }
-      epi_sync();
-      // coalesced rows: 128 rows x 32 doubles, 256 threads, two consecutive doubles each
-      const int ncol = min(kColsK, m.nb - j0);
-      for (int x = threadIdx.x; x < kRowsQ * kColsK / 2; x += kEpiWarps * 32) {
-        const int rr = x / (kColsK / 2), cc = 2 * (x - rr * (kColsK / 2));
-        if (i0 + rr < m.nb) {
-          double* dst = logits + (bh * m.nb + i0 + rr) * (int64_t)ld + j0 + cc;
-          const double v0 = stage[rr * kColsK + ((cc + rr) & (kColsK - 1))];
-          const double v1 = stage[rr * kColsK + ((cc + 1 + rr) & (kColsK - 1))];
-          if (cc + 1 < ncol) *reinterpret_cast<double2*>(dst) = make_double2(v0, v1);
-          else if (cc < ncol) dst[0] = v0;
+      // the thread's 8 consecutive logits of row i0 + r (64 bytes, 64-byte aligned)
+      if (i0 + r < m.nb) {
+        const int c0 = j0 + part * kEpiCols;
+        double* dst = logits + (bh * m.nb + i0 + r) * (int64_t)ld + c0;
+        if (c0 + kEpiCols <= m.nb) {
+#pragma unroll
+          for (int e = 0; e < kEpiCols; e += 2) *reinterpret_cast<double2*>(dst + e) = make_double2(out[e], out[e + 1]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < kEpiCols; ++e)
+            if (c0 + e < m.nb) dst[e] = out[e];
         }
       }
-      epi_sync();
     }
   }
 
