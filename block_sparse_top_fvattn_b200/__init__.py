@@ -23,7 +23,8 @@ from . import _lib
 from ._lib import (FVATTN_BF16, FVATTN_F32, FVATTN_MODE_FRAME_TOPK, FVATTN_MODE_TOPP, FvattnError, check,
                    load, status_string)
 
-__all__ = ["RouteConfig", "CsrBuffers", "alloc_csr", "route", "sparse_attn", "block_means", "read_status",
+__all__ = ["RouteConfig", "CsrBuffers", "alloc_csr", "route", "sparse_attn", "block_means", "block_scores",
+           "read_status",
            "workspace_bytes", "shape_of", "load", "FvattnError", "status_string", "rlb_plan", "select_heads",
            "LazyRouter"]
 
@@ -187,6 +188,35 @@ def block_means(x: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> 
     check(load().fvattn_block_means(x.data_ptr(), ctypes.byref(shape_of(x)), out.data_ptr(), _stream(stream)),
           "fvattn_block_means")
     return out
+
+
+def block_scores(q: torch.Tensor, k: torch.Tensor, scale: float = 0.0,
+                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """fvattn_block_scores: the router's fp64 block scores <Qbar_i, Kbar_j> * scale of every head,
+    as a [B, H, nb, nb] view of the library's [B*H*nb, ld] output (scale 0: 1/sqrt(d)). Raises
+    FvattnError if a kernel reported an error."""
+    _check_tensor(q, "q")
+    _check_tensor(k, "k")
+    if k.shape != q.shape or k.dtype != q.dtype or k.device != q.device:
+        raise ValueError("q and k must have the same shape, dtype and device")
+    B, H, S, d = q.shape
+    shp = shape_of(q, scale)
+    lib = load()
+    nws = lib.fvattn_block_scores_workspace_bytes(ctypes.byref(shp))
+    ld = lib.fvattn_block_scores_ld(ctypes.byref(shp))
+    if nws == 0 or ld == 0:
+        raise FvattnError(_lib.FVATTN_ERR_INVALID, "fvattn_block_scores_workspace_bytes")
+    nb = -(-S // BLOCK)
+    ws = torch.empty(nws, dtype=torch.uint8, device=q.device)
+    out = torch.empty((B * H * nb, ld), dtype=torch.float64, device=q.device)
+    status = torch.zeros(4, dtype=torch.int32, device=q.device)
+    check(lib.fvattn_block_scores(q.data_ptr(), k.data_ptr(), ctypes.byref(shp), out.data_ptr(), ws.data_ptr(), nws,
+                                  status.data_ptr(), _stream(stream)), "fvattn_block_scores")
+    (stream if stream is not None else torch.cuda.current_stream(q.device)).synchronize()
+    code = int(status[0].item())
+    if code != 0:
+        raise FvattnError(code, "fvattn_block_scores (device status)")
+    return out.view(B, H, nb, ld)[..., :nb]
 
 
 def read_status(csr: CsrBuffers, stream: Optional[torch.cuda.Stream] = None) -> int:

@@ -75,6 +75,12 @@ def load() -> ctypes.CDLL:
     lib.fvattn_sparse_attn.argtypes = [vp, vp, vp, P(Shape), P(Csr), vp, vp, vp]
     lib.fvattn_block_means.restype = ctypes.c_int
     lib.fvattn_block_means.argtypes = [vp, P(Shape), vp, vp]
+    lib.fvattn_block_scores_workspace_bytes.restype = ctypes.c_size_t
+    lib.fvattn_block_scores_workspace_bytes.argtypes = [P(Shape)]
+    lib.fvattn_block_scores_ld.restype = ctypes.c_int64
+    lib.fvattn_block_scores_ld.argtypes = [P(Shape)]
+    lib.fvattn_block_scores.restype = ctypes.c_int
+    lib.fvattn_block_scores.argtypes = [vp, vp, P(Shape), vp, vp, ctypes.c_size_t, vp, vp]
     lib.fvattn_read_status.restype = ctypes.c_int
     lib.fvattn_read_status.argtypes = [P(Csr), vp]
     lib.fvattn_route_static_scratch.restype = ctypes.c_int

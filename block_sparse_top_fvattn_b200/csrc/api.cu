@@ -10,7 +10,7 @@ using namespace fv;
 
 namespace {
 
-constexpr int kVersion = (1 << 16) | 2;
+constexpr int kVersion = (1 << 16) | 3;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -252,6 +252,38 @@ int fvattn_block_means(const void* X, const fvattn_shape* shape, double* out, fv
   if (nsm <= 0) return FVATTN_ERR_CUDA;
   cudaError_t e = launch_pool(X, nullptr, 1, shape->dtype, m, 0, 0, out, nullptr, nullptr, nullptr, SliceOut{}, nsm,
                               reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
+size_t fvattn_block_scores_workspace_bytes(const fvattn_shape* shape) {
+  if (validate_shape(shape) != FVATTN_OK) return 0;
+  return ws_layout(make_dims(*shape, 0), FVATTN_MODE_TOPP).logits;   // the slices and exponents
+}
+
+int64_t fvattn_block_scores_ld(const fvattn_shape* shape) {
+  if (validate_shape(shape) != FVATTN_OK) return 0;
+  return means_ld(make_dims(*shape, 0).nb);
+}
+
+int fvattn_block_scores(const void* Q, const void* K, const fvattn_shape* shape, double* scores, void* workspace,
+                        size_t workspace_bytes, int32_t* status, fvattn_stream_t stream) {
+  const int st = validate_shape(shape);
+  if (st != FVATTN_OK) return st;
+  if (!Q || !K || !scores || !workspace || !status) return FVATTN_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(scores, 16) || !aligned(workspace, 256) || !aligned(status, 4))
+    return FVATTN_ERR_INVALID;
+  const Dims m = make_dims(*shape, 0);
+  const WsLayout L = ws_layout(m, FVATTN_MODE_TOPP);
+  if (workspace_bytes < L.logits) return FVATTN_ERR_CAPACITY;
+  const int nsm = num_sms();
+  if (nsm <= 0) return FVATTN_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  const SliceOut so{reinterpret_cast<int8_t*>(ws + L.qs), reinterpret_cast<int8_t*>(ws + L.ks),
+                    reinterpret_cast<int32_t*>(ws + L.eq), reinterpret_cast<int32_t*>(ws + L.ek)};
+  if (cudaMemsetAsync(status, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
+  cudaError_t e = launch_pool(Q, K, 2, shape->dtype, m, 1, 0, nullptr, nullptr, nullptr, nullptr, so, nsm, s);
+  if (e == cudaSuccess) e = launch_score_tc(so.qs, so.ks, so.eq, so.ek, m, softmax_scale(shape), scores, status, nsm, s);
   return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
 }
 

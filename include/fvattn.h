@@ -206,6 +206,26 @@ int fvattn_sparse_attn(const void* Q, const void* K, const void* V, const fvattn
 int fvattn_block_means(const void* X, const fvattn_shape* shape, double* out,
                        fvattn_stream_t stream);
 
+/*
+ * fvattn_block_scores -- the scores of step 2 of fvattn_route (Top-p and top-k modes) on
+ * their own: scores[bh*nb + i][j] = <Qbar_i, Kbar_j> * scale (FVAttn summary: the importance
+ * of key block j for query block i; notes §5.2: scaled dot products of block means), Qbar and
+ * Kbar the block means of step 1. The means are split into a power-of-two scale 2^e and five
+ * signed 8-bit integer slices, multiplied exactly on the tensor cores and combined in fp64;
+ * the terms left out are below 2^-30 * 2^(e_i + e_j).
+ * Q, K: device [B,H,S,d] as for fvattn_route, 16-byte aligned. scores: device fp64
+ * [B*H*nb][ld], ld = fvattn_block_scores_ld(shape) (nb rounded up to a multiple of 32),
+ * 16-byte aligned; columns >= nb are not written. workspace: device, 256-byte aligned, at least
+ * fvattn_block_scores_workspace_bytes(shape) bytes. status: device int32[4], zeroed on
+ * `stream` before the kernels; a kernel that times out writes FVATTN_ERR_TIMEOUT to status[0].
+ * Returns FVATTN_OK once everything is enqueued on `stream`; the caller owns every buffer.
+ */
+size_t fvattn_block_scores_workspace_bytes(const fvattn_shape* shape);
+int64_t fvattn_block_scores_ld(const fvattn_shape* shape);
+int fvattn_block_scores(const void* Q, const void* K, const fvattn_shape* shape, double* scores,
+                        void* workspace, size_t workspace_bytes, int32_t* status,
+                        fvattn_stream_t stream);
+
 /* Synchronises `stream`, then returns the device status word status[0] (FVATTN_OK or a
  * negative fvattn_status written by a kernel). FVATTN_ERR_CUDA if the copy fails. */
 int fvattn_read_status(const fvattn_csr* csr, fvattn_stream_t stream);

@@ -38,6 +38,22 @@ def test_version_and_status_strings(lib):
     assert _lib.status_string(12345) == "unknown status"
 
 
+def test_block_scores_sizes_and_host_checks(lib):
+    s = shape(B=1, H=2, S=1000)                 # nb = 16, ld = 32
+    assert lib.fvattn_block_scores_ld(ctypes.byref(s)) == 32
+    ws = lib.fvattn_block_scores_workspace_bytes(ctypes.byref(s))
+    assert ws >= 2 * (2 * 5 * 16 * 128) + 2 * (2 * 16 * 4)     # Q and K slices, exponents
+    bad = shape(d=96)
+    assert lib.fvattn_block_scores_ld(ctypes.byref(bad)) == 0
+    assert lib.fvattn_block_scores_workspace_bytes(ctypes.byref(bad)) == 0
+    buf = ctypes.create_string_buffer(4096)
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    st = lib.fvattn_block_scores(None, p, ctypes.byref(s), p, p, ws, p, None)
+    assert st == _lib.FVATTN_ERR_INVALID
+    st = lib.fvattn_block_scores(p, p, ctypes.byref(bad), p, p, ws, p, None)
+    assert st == _lib.FVATTN_ERR_UNSUPPORTED
+
+
 def shape(B=1, H=2, S=1000, d=128, block=64, dtype=0, scale=0.0):
     return _lib.Shape(B, H, S, d, block, dtype, scale)
 

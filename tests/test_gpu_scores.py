@@ -1,0 +1,61 @@
+"""fvattn_block_scores (the router's fp64 block scores from exact 8-bit integer slices on the
+tensor cores) against the oracle's scaled dot products of the fp64 block means, element by
+element, within a bound derived from the arithmetic: the pooling's fp32 partial sums of bf16
+rows (error <= 3 * 2^-24 * mean|x| per mean) plus the slices' dropped terms (below 2^-30 *
+2^(e_i + e_j), here bounded by 2^-24 * d * max|Qbar_i| * max|Kbar_j|). A wrong digit, level or
+exponent moves a score by at least 2^-8 of its size."""
+import importlib
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_top_fvattn_b200 as fv
+from workloads import get_workload, make_inputs
+
+oroute = importlib.import_module("oracle.route")
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    ("tiny", {}),                                   # fp32, d = 64, S = 1024
+    ("single", dict(H=2, S=3000)),                  # bf16, d = 128, ragged last block
+    ("single", dict(H=2, S=2000, d=64)),            # bf16, d = 64 (slice rows half zero)
+    ("dit", dict(H=2)),                             # bf16, S = 32760, peaked heads (large logits)
+]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    fv.load()
+
+
+@pytest.mark.parametrize("name,over", CASES)
+def test_block_scores_match_oracle(name, over):
+    w = get_workload(name).replace(**over) if over else get_workload(name)
+    d_ = make_inputs(w, device="cuda")
+    q, k = d_["q"], d_["k"]
+    B, H, S, d = q.shape
+    got = fv.block_scores(q, k).cpu().numpy().reshape(B * H, -1, -(-S // 64))
+    Q = q.reshape(B * H, S, d).cpu().double().numpy()
+    K = k.reshape(B * H, S, d).cpu().double().numpy()
+    scale = 1.0 / np.sqrt(d)
+    qm, km = oroute.pool_blocks(Q, 64), oroute.pool_blocks(K, 64)
+    want = oroute.block_scores(qm, km, scale)
+    qa, ka = oroute.pool_blocks(np.abs(Q), 64), oroute.pool_blocks(np.abs(K), 64)
+    pool_err = 3.0 * 2.0 ** -24 * (np.matmul(qa, np.abs(km).swapaxes(1, 2)) + np.matmul(np.abs(qm), ka.swapaxes(1, 2)))
+    slice_err = 2.0 ** -24 * d * np.abs(qm).max(axis=2)[:, :, None] * np.abs(km).max(axis=2)[:, None, :]
+    tol = scale * (1.01 * pool_err + slice_err) + 1e-300
+    err = np.abs(got - want)
+    worst = float((err / tol).max())
+    assert worst <= 1.0, f"max |gpu - oracle| / bound = {worst:.3g} (max abs error {err.max():.3g})"
+    # the bound is tight enough to mean something: far below the size of the scores
+    assert float(tol.max()) < 1e-5 * max(1.0, float(np.abs(want).max()))
+
+
+def test_block_scores_rejects_mismatched_inputs():
+    q = torch.zeros(1, 1, 128, 64, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fv.block_scores(q, torch.zeros(1, 1, 128, 64, device="cuda", dtype=torch.float32))
