@@ -410,6 +410,22 @@ def run_ours(args, w):
     router_gbs = rbytes / (route_avg * 1e-3) / 1e9
     traffic = traffic_from_profile(os.path.join(ROOT, "block_sparse_top_fvattn_b200", "csrc", "attn_tc.cu"))
 
+    # SM busy-time imbalance of the persistent attention grid (outside the timed region): one
+    # stamped launch on the router's longest-first order, one on ascending tile ids.
+    sm_busy = None
+    if q.dtype == torch.bfloat16 and not args.no_sm_busy:
+        fv.route(q, k, cfg, csr=csr, workspace=ws)
+        _, st_lpt = fv.sparse_attn_stamped(q, k, v, csr, out=out)
+        csr.tile_order.copy_(torch.arange(csr.tile_order.numel(), dtype=torch.int32, device=dev))
+        _, st_asc = fv.sparse_attn_stamped(q, k, v, csr, out=out)
+        torch.cuda.synchronize()
+        if fv.read_status(csr) != 0:
+            raise RuntimeError(f"device status {fv.read_status(csr)}")
+        a, b = fv.sm_busy_imbalance(st_lpt), fv.sm_busy_imbalance(st_asc)
+        sm_busy = {"longest_first": round(a["imbalance"], 4), "ascending": round(b["imbalance"], 4),
+                   "sms": a["sms"], "max_busy_ms": [round(a["max_ns"] / 1e6, 4), round(b["max_ns"] / 1e6, 4)],
+                   "definition": "per SM: last CTA end - first CTA start (globaltimer); max / mean over SMs"}
+
     # End to end through the public API with host buffers (pinned): every step copies its Q, K, V
     # in and its O out inside the timed region. As a serving loop would, the transfers of
     # neighbouring steps overlap the compute: the inputs of step s+1 go up and the output of step
@@ -508,6 +524,7 @@ def run_ours(args, w):
         "pct_bf16_peak_attn": 100.0 * attn_tflops / pk["bf16_tflops"],
         "density": density, "selected_flops_per_layer": flops, "padded_tile_flops_per_layer": flops_padded,
         "tile_mma_flops_per_layer": mma_flops, "tile_utilisation": flops / mma_flops if mma_flops else None,
+        "sm_busy_imbalance": sm_busy,
         "selected_kv_tokens_per_s": kv_tokens / (attn_avg * 1e-3),
         "query_tokens_per_s": BH * S / (ms_step * 1e-3),
         "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": attn_tflops, "peak": bf16_peak,
@@ -536,6 +553,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sm-busy", action="store_true", help="skip the stamped launches of the SM busy-time imbalance")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling case)")
     ap.add_argument("--p", type=float, default=0.0, help="override the Top-p threshold")
     ap.add_argument("--mode", default="topp", choices=["topp", "frame_topk"])

@@ -23,7 +23,8 @@ from . import _lib
 from ._lib import (FVATTN_BF16, FVATTN_F32, FVATTN_MODE_FRAME_TOPK, FVATTN_MODE_TOPP, FvattnError, check,
                    load, status_string)
 
-__all__ = ["RouteConfig", "CsrBuffers", "alloc_csr", "route", "sparse_attn", "block_means", "block_scores",
+__all__ = ["RouteConfig", "CsrBuffers", "alloc_csr", "route", "sparse_attn", "sparse_attn_stamped",
+           "sm_busy_imbalance", "block_means", "block_scores",
            "read_status",
            "workspace_bytes", "shape_of", "load", "FvattnError", "status_string", "rlb_plan", "select_heads",
            "LazyRouter"]
@@ -178,6 +179,43 @@ def sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, csr: CsrBuffe
                                     out.data_ptr(), lse.data_ptr() if lse is not None else None, _stream(stream)),
           "fvattn_sparse_attn")
     return out
+
+
+def sparse_attn_stamped(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, csr: CsrBuffers, *,
+                        out: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+                        scale: float = 0.0):
+    """fvattn_sparse_attn_stamped (bf16): the attention plus, per CTA of its persistent grid, the
+    SM id and the busy interval in ns. Returns (O, stamps [n_cta, 3] int64 on the device)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_tensor(t, n)
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k, v must have the same shape and dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    shp = shape_of(q, scale)
+    lib = load()
+    words = lib.fvattn_attn_stamp_words(ctypes.byref(shp))
+    if words <= 0:
+        raise FvattnError(_lib.FVATTN_ERR_UNSUPPORTED, "fvattn_attn_stamp_words")
+    stamps = torch.zeros(words, dtype=torch.int64, device=q.device)
+    check(lib.fvattn_sparse_attn_stamped(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(shp),
+                                         ctypes.byref(csr.to_c()), out.data_ptr(), None, stamps.data_ptr(), words,
+                                         _stream(stream)), "fvattn_sparse_attn_stamped")
+    return out, stamps.view(-1, 3)
+
+
+def sm_busy_imbalance(stamps: torch.Tensor) -> dict:
+    """From the [n_cta, 3] stamps of sparse_attn_stamped: each SM's busy time (last end minus
+    first start over its CTAs), and max / mean of those over the SMs."""
+    st = stamps.cpu().numpy().astype("int64")
+    busy = {}
+    for sm, t0, t1 in st:
+        lo, hi = busy.get(int(sm), (t0, t1))
+        busy[int(sm)] = (min(lo, t0), max(hi, t1))
+    times = [hi - lo for lo, hi in busy.values()]
+    mean = sum(times) / len(times)
+    return {"sms": len(times), "max_ns": int(max(times)), "mean_ns": float(mean),
+            "imbalance": float(max(times) / mean) if mean > 0 else 1.0}
 
 
 def block_means(x: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:

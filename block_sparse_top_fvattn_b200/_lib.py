@@ -81,6 +81,10 @@ def load() -> ctypes.CDLL:
     lib.fvattn_block_scores_ld.argtypes = [P(Shape)]
     lib.fvattn_block_scores.restype = ctypes.c_int
     lib.fvattn_block_scores.argtypes = [vp, vp, P(Shape), vp, vp, ctypes.c_size_t, vp, vp]
+    lib.fvattn_attn_stamp_words.restype = ctypes.c_int64
+    lib.fvattn_attn_stamp_words.argtypes = [P(Shape)]
+    lib.fvattn_sparse_attn_stamped.restype = ctypes.c_int
+    lib.fvattn_sparse_attn_stamped.argtypes = [vp, vp, vp, P(Shape), P(Csr), vp, vp, vp, ctypes.c_int64, vp]
     lib.fvattn_read_status.restype = ctypes.c_int
     lib.fvattn_read_status.argtypes = [P(Csr), vp]
     lib.fvattn_route_static_scratch.restype = ctypes.c_int

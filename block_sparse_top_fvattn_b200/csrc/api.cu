@@ -206,8 +206,12 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const 
   return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
 }
 
-int fvattn_sparse_attn(const void* Q, const void* K, const void* V, const fvattn_shape* shape,
-                       const fvattn_csr* csr, void* O, float* lse, fvattn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+int sparse_attn(const void* Q, const void* K, const void* V, const fvattn_shape* shape, const fvattn_csr* csr,
+                void* O, float* lse, uint64_t* stamps, fvattn_stream_t stream) {
   int st = validate_shape(shape);
   if (st != FVATTN_OK) return st;
   if (!Q || !K || !V || !O || !csr || !csr->row_ptr || !csr->col_idx || !csr->tile_order || !csr->status)
@@ -227,9 +231,38 @@ int fvattn_sparse_attn(const void* Q, const void* K, const void* V, const fvattn
     if (nsm <= 0) return FVATTN_ERR_CUDA;
     if (cudaMemsetAsync(csr->status + 2, 0, sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
     e = launch_attn_tc(Q, K, V, m, scale, csr->row_ptr, csr->col_idx, csr->col_code, csr->tile_order, csr->status, O,
-                       lse, nsm, s);
+                       lse, stamps, nsm, s);
   }
   return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fvattn_sparse_attn(const void* Q, const void* K, const void* V, const fvattn_shape* shape,
+                       const fvattn_csr* csr, void* O, float* lse, fvattn_stream_t stream) {
+  return sparse_attn(Q, K, V, shape, csr, O, lse, nullptr, stream);
+}
+
+int64_t fvattn_attn_stamp_words(const fvattn_shape* shape) {
+  if (validate_shape(shape) != FVATTN_OK || shape->dtype != FVATTN_BF16) return 0;
+  const int nsm = num_sms();
+  if (nsm <= 0) return 0;
+  return 3 * (int64_t)attn_tc_grid(make_dims(*shape, 0), nsm);
+}
+
+int fvattn_sparse_attn_stamped(const void* Q, const void* K, const void* V, const fvattn_shape* shape,
+                               const fvattn_csr* csr, void* O, float* lse, uint64_t* stamps, int64_t stamp_words,
+                               fvattn_stream_t stream) {
+  const int st = validate_shape(shape);
+  if (st != FVATTN_OK) return st;
+  if (shape->dtype != FVATTN_BF16) return FVATTN_ERR_UNSUPPORTED;
+  if (stamps == nullptr || !aligned(stamps, 8)) return FVATTN_ERR_INVALID;
+  const int64_t need = fvattn_attn_stamp_words(shape);
+  if (need <= 0) return FVATTN_ERR_CUDA;
+  if (stamp_words < need) return FVATTN_ERR_CAPACITY;
+  return sparse_attn(Q, K, V, shape, csr, O, lse, stamps, stream);
 }
 
 int fvattn_select_heads(const fvattn_shape* shape, const fvattn_csr* csr, const uint8_t* active,

@@ -170,7 +170,8 @@ __global__ void __launch_bounds__(192, 2)
                    const __grid_constant__ CUtensorMap tmV, Dims m, float scale_log2,
                    const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
                    const int32_t* __restrict__ col_code, const int32_t* __restrict__ tile_order,
-                   int32_t* __restrict__ control, __nv_bfloat16* __restrict__ O, float* __restrict__ lse) {
+                   int32_t* __restrict__ control, __nv_bfloat16* __restrict__ O, float* __restrict__ lse,
+                   uint64_t* __restrict__ stamps) {
   using L = TcLayout<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -215,6 +216,11 @@ __global__ void __launch_bounds__(192, 2)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tbase = bars->tmem_base;
+  if (stamps != nullptr && threadIdx.x == 0) {
+    uint64_t t_begin;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_begin));
+    stamps[3 * blockIdx.x + 1] = t_begin;
+  }
 
   if (warp == 0) {
     if (lane == 0) {
@@ -535,6 +541,15 @@ __global__ void __launch_bounds__(192, 2)
   tc::fence_after_sync();
   if (warp == 1) tc::tmem_dealloc(tbase, L::kTmemCols);
   if (threadIdx.x == 0 && bars->abort) report_error(control, FVATTN_ERR_TIMEOUT, bars->abort);
+  if (stamps != nullptr && threadIdx.x == 0) {
+    // this CTA's SM and its busy interval (ns), for the SM busy-time imbalance
+    uint64_t t_end;
+    uint32_t smid;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_end));
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    stamps[3 * blockIdx.x] = smid;
+    stamps[3 * blockIdx.x + 2] = t_end;
+  }
 }
 
 // [BH, S, d] bf16 viewed as a 3-D tensor (d innermost); 64 x 64 boxes with the 128-byte
@@ -546,29 +561,32 @@ bool make_map(CUtensorMap* map, const void* base, const Dims& m) {
 template <int D>
 cudaError_t launch_tc_d(const void* Q, const void* K, const void* V, const Dims& m, float scale,
                         const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
-                        const int32_t* tile_order, int32_t* control, void* O, float* lse, int nsm,
-                        cudaStream_t st) {
+                        const int32_t* tile_order, int32_t* control, void* O, float* lse, uint64_t* stamps,
+                        int nsm, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, Q, m) || !make_map(&mk, K, m) || !make_map(&mv, V, m)) return cudaErrorInvalidValue;
   const size_t smem = TcLayout<D>::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int64_t ntiles = m.BH * m.nt;
-  const int grid = (int)imin<int64_t>(ntiles, (int64_t)nsm * 2);
+  const int grid = attn_tc_grid(m, nsm);
   attn_tc_kernel<D><<<grid, 192, smem, st>>>(mq, mk, mv, m, scale * 1.4426950408889634f, row_ptr, col_idx,
-                                             col_code, tile_order, control, static_cast<__nv_bfloat16*>(O), lse);
+                                             col_code, tile_order, control, static_cast<__nv_bfloat16*>(O), lse,
+                                             stamps);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+int attn_tc_grid(const Dims& m, int nsm) { return (int)imin<int64_t>(m.BH * m.nt, (int64_t)nsm * 2); }
+
 cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const Dims& m, float scale,
                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
-                           const int32_t* tile_order, int32_t* control, void* O, float* lse, int nsm,
-                           cudaStream_t st) {
+                           const int32_t* tile_order, int32_t* control, void* O, float* lse, uint64_t* stamps,
+                           int nsm, cudaStream_t st) {
   if (m.d == 128)
-    return launch_tc_d<128>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O, lse, nsm, st);
-  return launch_tc_d<64>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O, lse, nsm, st);
+    return launch_tc_d<128>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O, lse, stamps, nsm,
+                            st);
+  return launch_tc_d<64>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O, lse, stamps, nsm, st);
 }
 
 }  // namespace fv

@@ -74,9 +74,12 @@ cudaError_t launch_attn_f32(const float* Q, const float* K, const float* V, cons
                             const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
                             const int32_t* tile_order, const int32_t* control, float* O, float* lse,
                             cudaStream_t st);
+// stamps: null, or 3 words per CTA of the launch (attn_tc_grid): the SM id and the CTA's busy
+// interval [start, end) in ns of %globaltimer.
+int attn_tc_grid(const Dims& m, int nsm);
 cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const Dims& m, float scale,
                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
-                           const int32_t* tile_order, int32_t* control, void* O, float* lse, int nsm,
-                           cudaStream_t st);
+                           const int32_t* tile_order, int32_t* control, void* O, float* lse, uint64_t* stamps,
+                           int nsm, cudaStream_t st);
 
 }  // namespace fv

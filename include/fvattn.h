@@ -200,6 +200,22 @@ int fvattn_sparse_attn(const void* Q, const void* K, const void* V, const fvattn
                        const fvattn_csr* csr, void* O, float* lse, fvattn_stream_t stream);
 
 /*
+ * fvattn_sparse_attn_stamped -- fvattn_sparse_attn (bf16 only) that also records, for every CTA
+ * of the persistent attention grid, the SM it ran on and its busy interval: stamps[3c] = SM id,
+ * stamps[3c+1] = start, stamps[3c+2] = end (ns of the GPU's global timer). The busy-time
+ * imbalance of the SMs (max / mean of max(end) - min(start) over each SM's CTAs) shows how well
+ * the tile order balances the work (the single-GPU analogue of the FVAttn summary's RLB
+ * imbalance factor). stamps: device uint64, at least fvattn_attn_stamp_words(shape) words
+ * (3 per CTA; the grid depends on the current device's SM count, so that call needs a GPU and
+ * returns 0 without one or for fp32). Errors as fvattn_sparse_attn, plus FVATTN_ERR_CAPACITY
+ * when stamp_words is too small.
+ */
+int64_t fvattn_attn_stamp_words(const fvattn_shape* shape);
+int fvattn_sparse_attn_stamped(const void* Q, const void* K, const void* V, const fvattn_shape* shape,
+                               const fvattn_csr* csr, void* O, float* lse, uint64_t* stamps,
+                               int64_t stamp_words, fvattn_stream_t stream);
+
+/*
  * fvattn_block_means -- step 1 of fvattn_route on its own: means of X [B,H,S,d] over the
  * valid tokens of each 64-token block, written as fp64 [B,H,nb,d] to `out` (device).
  */

@@ -3,7 +3,8 @@ tensor cores) against the oracle's scaled dot products of the fp64 block means, 
 element, within a bound derived from the arithmetic: the pooling's fp32 partial sums of bf16
 rows (error <= 3 * 2^-24 * mean|x| per mean) plus the slices' dropped terms (below 2^-30 *
 2^(e_i + e_j), here bounded by 2^-24 * d * max|Qbar_i| * max|Kbar_j|). A wrong digit, level or
-exponent moves a score by at least 2^-8 of its size."""
+exponent moves a score by at least 2^-8 of its size. Also the stamped attention entry point
+(per-CTA SM ids and busy intervals): same output as the plain call, valid stamps."""
 import importlib
 
 import numpy as np
@@ -59,3 +60,31 @@ def test_block_scores_rejects_mismatched_inputs():
     q = torch.zeros(1, 1, 128, 64, device="cuda", dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         fv.block_scores(q, torch.zeros(1, 1, 128, 64, device="cuda", dtype=torch.float32))
+
+
+def test_stamped_attention_equals_plain_and_stamps_are_valid():
+    """fvattn_sparse_attn_stamped runs the same kernel: its output equals fvattn_sparse_attn's
+    bit for bit, and every CTA reports an SM id below the device's SM count and start <= end."""
+    w = get_workload("single").replace(H=4, S=4000)
+    x = make_inputs(w, device="cuda")
+    q, k, v = x["q"], x["k"], x["v"]
+    csr = fv.route(q, k, fv.RouteConfig(p=0.9))
+    o_plain = fv.sparse_attn(q, k, v, csr)
+    o_st, stamps = fv.sparse_attn_stamped(q, k, v, csr)
+    torch.cuda.synchronize()
+    assert fv.read_status(csr) == 0
+    assert torch.equal(o_plain, o_st)
+    st = stamps.cpu().numpy()
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    assert st.shape[0] >= 1 and np.all(st[:, 0] >= 0) and np.all(st[:, 0] < nsm)
+    assert np.all(st[:, 1] > 0) and np.all(st[:, 2] >= st[:, 1])
+    imb = fv.sm_busy_imbalance(stamps)
+    assert imb["imbalance"] >= 1.0 and imb["sms"] <= nsm
+
+
+def test_stamped_attention_rejects_fp32():
+    w = get_workload("tiny")
+    x = make_inputs(w, device="cuda")
+    csr = fv.route(x["q"], x["k"], fv.RouteConfig(p=0.9))
+    with pytest.raises(fv.FvattnError):
+        fv.sparse_attn_stamped(x["q"], x["k"], x["v"], csr)
