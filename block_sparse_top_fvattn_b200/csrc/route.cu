@@ -48,7 +48,7 @@ __device__ __forceinline__ T warp_incl_scan(T v, int lane) {
 // summed in AccT (fp32 for bf16 input: exact unless the values' exponents are 16+ apart;
 // fp64 for fp32 input), the partial sums in fp64 in a fixed order, and the row groups of a
 // column are folded with shuffles. The next block's first batch is loaded before the current
-// block's epilogue. OUT selects what is written: means [row][d]; the means as exact bf16 integer
+// block's epilogue. OUT selects what is written: means [row][d]; the means as signed 8-bit integer
 // slices with power-of-two exponents (the operands of the score GEMM); or fp64 sums of the
 // tokens before / after the block's first frame boundary, [row][d].
 
