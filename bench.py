@@ -531,7 +531,12 @@ def run_ours(args, w):
                      "unit": "TFLOP/s", "frac": attn_tflops / bf16_peak, "traffic": traffic,
                      "peak_kind": peak_kind,
                      "frac_of_burst": attn_tflops / pk["bf16_tflops"],
-                     "frac_of_sustained": attn_tflops / pk["bf16_tflops_sustained"]},
+                     "frac_of_sustained": attn_tflops / pk["bf16_tflops_sustained"],
+                     # the MMA work the 128-row tiles execute (both query blocks of a tile over
+                     # the union of their key blocks), for context; `achieved` counts selected
+                     # pairs only
+                     "executed_tflops": mma_flops / (attn_avg * 1e-3) / 1e12,
+                     "frac_executed": mma_flops / (attn_avg * 1e-3) / 1e12 / bf16_peak},
         "roofline_router": {"bound": "hbm", "achieved": router_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                             "frac": router_gbs / pk["hbm_gbs"], "algorithmic_bytes": rbytes,
                             "peak_kind": f"hbm copy ({pk_src})"},
