@@ -23,7 +23,8 @@ from . import _lib
 from ._lib import (FVATTN_BF16, FVATTN_F32, FVATTN_MODE_FRAME_TOPK, FVATTN_MODE_TOPP, FvattnError, check,
                    load, status_string)
 
-__all__ = ["RouteConfig", "CsrBuffers", "alloc_csr", "route", "sparse_attn", "sparse_attn_stamped",
+__all__ = ["RouteConfig", "CsrBuffers", "alloc_csr", "route", "route_pool", "route_finish", "sparse_attn",
+           "sparse_attn_stamped",
            "sm_busy_imbalance", "block_means", "block_scores",
            "read_status",
            "workspace_bytes", "shape_of", "load", "FvattnError", "status_string", "rlb_plan", "select_heads",
@@ -160,6 +161,41 @@ def route(q: torch.Tensor, k: torch.Tensor, cfg: Optional[RouteConfig] = None, *
     check(load().fvattn_route(q.data_ptr(), k.data_ptr(), ctypes.byref(shp), ctypes.byref(c_cfg),
                               ctypes.byref(c_csr), workspace.data_ptr(), nws, _stream(stream)), "fvattn_route")
     csr._workspace = workspace      # keep the scratch alive until the kernels have run
+    return csr
+
+
+def route_pool(q: torch.Tensor, k: torch.Tensor, cfg: RouteConfig, block_begin: int, block_end: int,
+               workspace: torch.Tensor, *, stream: Optional[torch.cuda.Stream] = None, scale: float = 0.0) -> None:
+    """fvattn_route_pool: step 1 of the router for the 64-token blocks [block_begin, block_end)
+    of every head of q, k ([B, H, S, d]; only those blocks' tokens are read) into `workspace`
+    (uint8, at least workspace_bytes(q, cfg))."""
+    _check_tensor(q, "q")
+    _check_tensor(k, "k")
+    if k.shape != q.shape or k.dtype != q.dtype:
+        raise ValueError("q and k must have the same shape and dtype")
+    nws = workspace_bytes(q, cfg)
+    if workspace.numel() < nws or not workspace.is_cuda:
+        raise ValueError(f"workspace needs {nws} bytes on the device")
+    check(load().fvattn_route_pool(q.data_ptr(), k.data_ptr(), ctypes.byref(shape_of(q, scale)),
+                                   ctypes.byref(cfg.to_c()), int(block_begin), int(block_end), workspace.data_ptr(),
+                                   nws, _stream(stream)), "fvattn_route_pool")
+
+
+def route_finish(q: torch.Tensor, cfg: RouteConfig, workspace: torch.Tensor, *, csr: Optional[CsrBuffers] = None,
+                 stream: Optional[torch.cuda.Stream] = None, scale: float = 0.0) -> CsrBuffers:
+    """fvattn_route_finish: steps 2 and 3 of the router from a workspace in which route_pool has
+    pooled every block of every head (q gives the shape only). Returns the CSR buffers."""
+    _check_tensor(q, "q")
+    B, H, S, _ = q.shape
+    if csr is None:
+        csr = alloc_csr(B, H, S, q.device, codes=cfg.frame_exact)
+    nws = workspace_bytes(q, cfg)
+    if workspace.numel() < nws or not workspace.is_cuda:
+        raise ValueError(f"workspace needs {nws} bytes on the device")
+    check(load().fvattn_route_finish(ctypes.byref(shape_of(q, scale)), ctypes.byref(cfg.to_c()),
+                                     ctypes.byref(csr.to_c()), workspace.data_ptr(), nws, _stream(stream)),
+          "fvattn_route_finish")
+    csr._workspace = workspace
     return csr
 
 

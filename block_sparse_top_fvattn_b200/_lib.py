@@ -71,6 +71,11 @@ def load() -> ctypes.CDLL:
     lib.fvattn_route_workspace_bytes.argtypes = [P(Shape), P(RouteCfg)]
     lib.fvattn_route.restype = ctypes.c_int
     lib.fvattn_route.argtypes = [vp, vp, P(Shape), P(RouteCfg), P(Csr), vp, ctypes.c_size_t, vp]
+    lib.fvattn_route_pool.restype = ctypes.c_int
+    lib.fvattn_route_pool.argtypes = [vp, vp, P(Shape), P(RouteCfg), ctypes.c_int64, ctypes.c_int64, vp,
+                                      ctypes.c_size_t, vp]
+    lib.fvattn_route_finish.restype = ctypes.c_int
+    lib.fvattn_route_finish.argtypes = [P(Shape), P(RouteCfg), P(Csr), vp, ctypes.c_size_t, vp]
     lib.fvattn_sparse_attn.restype = ctypes.c_int
     lib.fvattn_sparse_attn.argtypes = [vp, vp, vp, P(Shape), P(Csr), vp, vp, vp]
     lib.fvattn_block_means.restype = ctypes.c_int

@@ -146,54 +146,45 @@ size_t fvattn_route_workspace_bytes(const fvattn_shape* shape, const fvattn_rout
   return ws_layout(m, cfg->mode).total;
 }
 
-int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const fvattn_route_cfg* cfg,
-                 const fvattn_csr* out, void* workspace, size_t workspace_bytes, fvattn_stream_t stream) {
-  int st = validate_shape(shape);
-  if (st != FVATTN_OK) return st;
-  st = validate_cfg(shape, cfg);
-  if (st != FVATTN_OK) return st;
-  if (Q == nullptr || K == nullptr || out == nullptr || workspace == nullptr) return FVATTN_ERR_INVALID;
-  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(workspace, 256)) return FVATTN_ERR_INVALID;
-  if (!out->row_ptr || !out->col_idx || !out->head_load || !out->tile_cost || !out->tile_order || !out->nnz ||
-      !out->status)
-    return FVATTN_ERR_INVALID;
-  if (cfg->frame_exact && out->col_code == nullptr) return FVATTN_ERR_INVALID;
-  const Dims m = make_dims(*shape, cfg->frame_len);
-  const WsLayout L = ws_layout(m, cfg->mode);
-  if (workspace_bytes < L.total) return FVATTN_ERR_CAPACITY;
-  if (out->col_capacity < m.BH * m.nb * m.nb) return FVATTN_ERR_CAPACITY;
-  const int nsm = num_sms();
-  if (nsm <= 0) return FVATTN_ERR_CUDA;
+}  // extern "C"
 
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  unsigned char* ws = static_cast<unsigned char*>(workspace);
-  double* qlo = reinterpret_cast<double*>(ws + L.qlo);
-  double* klo = reinterpret_cast<double*>(ws + L.klo);
+namespace {
+
+// Step 1 of the router for the blocks [b0, b1) of every head, into the workspace.
+cudaError_t route_pool(const void* Q, const void* K, const fvattn_shape* shape, const fvattn_route_cfg* cfg,
+                       const Dims& m, const WsLayout& L, unsigned char* ws, int b0, int b1, int nsm, cudaStream_t s) {
+  if (cfg->mode == FVATTN_MODE_TOPP || cfg->mode == FVATTN_MODE_TOPK_BLOCKS) {
+    const SliceOut so{reinterpret_cast<int8_t*>(ws + L.qs), reinterpret_cast<int8_t*>(ws + L.ks),
+                      reinterpret_cast<int32_t*>(ws + L.eq), reinterpret_cast<int32_t*>(ws + L.ek)};
+    return launch_pool(Q, K, 2, shape->dtype, m, b0, b1, 1, 0, nullptr, nullptr, nullptr, nullptr, so, nsm, s);
+  }
+  return launch_pool(Q, K, 2, shape->dtype, m, b0, b1, 2, cfg->frame_len, reinterpret_cast<double*>(ws + L.qlo),
+                     reinterpret_cast<double*>(ws + L.klo), reinterpret_cast<double*>(ws + L.qhi),
+                     reinterpret_cast<double*>(ws + L.khi), SliceOut{}, nsm, s);
+}
+
+// Steps 2 and 3 of the router from a workspace whose every block has been pooled.
+cudaError_t route_finish(const fvattn_shape* shape, const fvattn_route_cfg* cfg, const fvattn_csr* out, const Dims& m,
+                         const WsLayout& L, unsigned char* ws, int nsm, cudaStream_t s) {
   uint32_t* bits = reinterpret_cast<uint32_t*>(ws + L.bits);
   int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
   const double scale = softmax_scale(shape);
   ForceCfg fc{cfg->force_diag, cfg->local_window, cfg->frame_len, cfg->frame_window, cfg->force_first_frame};
-
-  if (cudaMemsetAsync(out->status, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
-  cudaError_t e;
+  cudaError_t e = cudaMemsetAsync(out->status, 0, 4 * sizeof(int32_t), s);
+  if (e != cudaSuccess) return e;
   if (cfg->mode == FVATTN_MODE_TOPP || cfg->mode == FVATTN_MODE_TOPK_BLOCKS) {
     const int kblocks = cfg->mode == FVATTN_MODE_TOPK_BLOCKS ? cfg->topk_blocks : 0;
     const SliceOut so{reinterpret_cast<int8_t*>(ws + L.qs), reinterpret_cast<int8_t*>(ws + L.ks),
                       reinterpret_cast<int32_t*>(ws + L.eq), reinterpret_cast<int32_t*>(ws + L.ek)};
-    e = launch_pool(Q, K, 2, shape->dtype, m, 1, 0, nullptr, nullptr, nullptr, nullptr, so, nsm, s);
-    if (e == cudaSuccess)
-      e = launch_topp(so, reinterpret_cast<double*>(ws + L.logits), m, cfg->p >= 1.f ? 1.0 : (double)cfg->p, kblocks,
-                      scale, fc, SasaCfg{cfg->sasa_coef, cfg->sasa_trigger}, bits, counts, out->tile_cost,
-                      out->status, nsm, s);
+    e = launch_topp(so, reinterpret_cast<double*>(ws + L.logits), m, cfg->p >= 1.f ? 1.0 : (double)cfg->p, kblocks,
+                    scale, fc, SasaCfg{cfg->sasa_coef, cfg->sasa_trigger}, bits, counts, out->tile_cost, out->status,
+                    nsm, s);
   } else {
-    double* qhi = reinterpret_cast<double*>(ws + L.qhi);
-    double* khi = reinterpret_cast<double*>(ws + L.khi);
-    double* qf = reinterpret_cast<double*>(ws + L.qf);
-    double* kf = reinterpret_cast<double*>(ws + L.kf);
-    e = launch_pool(Q, K, 2, shape->dtype, m, 2, cfg->frame_len, qlo, klo, qhi, khi, SliceOut{}, nsm, s);
-    if (e == cudaSuccess)
-      e = launch_frame(qlo, qhi, klo, khi, qf, kf, m, cfg->frame_len, cfg->topk_frames, scale, fc, bits, counts,
-                       out->tile_cost, reinterpret_cast<uint32_t*>(ws + L.fsel), s);
+    e = launch_frame(reinterpret_cast<double*>(ws + L.qlo), reinterpret_cast<double*>(ws + L.qhi),
+                     reinterpret_cast<double*>(ws + L.klo), reinterpret_cast<double*>(ws + L.khi),
+                     reinterpret_cast<double*>(ws + L.qf), reinterpret_cast<double*>(ws + L.kf), m, cfg->frame_len,
+                     cfg->topk_frames, scale, fc, bits, counts, out->tile_cost,
+                     reinterpret_cast<uint32_t*>(ws + L.fsel), s);
   }
   if (e == cudaSuccess)
     e = launch_schedule(counts, out->tile_cost, m, out->row_ptr, out->head_load, out->nnz, out->tile_order,
@@ -203,6 +194,79 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const 
     e = launch_codes(out->row_ptr, out->col_idx, m, cfg->frame_exact ? reinterpret_cast<const uint32_t*>(ws + L.fsel)
                                                                      : nullptr,
                      cfg->frame_len, fc, out->col_code, out->col_capacity, nsm, s);
+  return e;
+}
+
+int check_route_inputs(const fvattn_shape* shape, const fvattn_route_cfg* cfg, void* workspace,
+                       size_t workspace_bytes) {
+  int st = validate_shape(shape);
+  if (st != FVATTN_OK) return st;
+  st = validate_cfg(shape, cfg);
+  if (st != FVATTN_OK) return st;
+  if (workspace == nullptr || !aligned(workspace, 256)) return FVATTN_ERR_INVALID;
+  const Dims m = make_dims(*shape, cfg->frame_len);
+  if (workspace_bytes < ws_layout(m, cfg->mode).total) return FVATTN_ERR_CAPACITY;
+  return FVATTN_OK;
+}
+
+int check_csr_out(const fvattn_shape* shape, const fvattn_route_cfg* cfg, const fvattn_csr* out) {
+  if (out == nullptr || !out->row_ptr || !out->col_idx || !out->head_load || !out->tile_cost || !out->tile_order ||
+      !out->nnz || !out->status)
+    return FVATTN_ERR_INVALID;
+  if (cfg->frame_exact && out->col_code == nullptr) return FVATTN_ERR_INVALID;
+  const Dims m = make_dims(*shape, cfg->frame_len);
+  if (out->col_capacity < m.BH * m.nb * m.nb) return FVATTN_ERR_CAPACITY;
+  return FVATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const fvattn_route_cfg* cfg,
+                 const fvattn_csr* out, void* workspace, size_t workspace_bytes, fvattn_stream_t stream) {
+  int st = check_route_inputs(shape, cfg, workspace, workspace_bytes);
+  if (st != FVATTN_OK) return st;
+  if (Q == nullptr || K == nullptr || !aligned(Q, 16) || !aligned(K, 16)) return FVATTN_ERR_INVALID;
+  st = check_csr_out(shape, cfg, out);
+  if (st != FVATTN_OK) return st;
+  const Dims m = make_dims(*shape, cfg->frame_len);
+  const WsLayout L = ws_layout(m, cfg->mode);
+  const int nsm = num_sms();
+  if (nsm <= 0) return FVATTN_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  cudaError_t e = route_pool(Q, K, shape, cfg, m, L, ws, 0, m.nb, nsm, s);
+  if (e == cudaSuccess) e = route_finish(shape, cfg, out, m, L, ws, nsm, s);
+  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
+int fvattn_route_pool(const void* Q, const void* K, const fvattn_shape* shape, const fvattn_route_cfg* cfg,
+                      int64_t block_begin, int64_t block_end, void* workspace, size_t workspace_bytes,
+                      fvattn_stream_t stream) {
+  int st = check_route_inputs(shape, cfg, workspace, workspace_bytes);
+  if (st != FVATTN_OK) return st;
+  if (Q == nullptr || K == nullptr || !aligned(Q, 16) || !aligned(K, 16)) return FVATTN_ERR_INVALID;
+  const Dims m = make_dims(*shape, cfg->frame_len);
+  if (block_begin < 0 || block_end > m.nb || block_begin >= block_end) return FVATTN_ERR_INVALID;
+  const int nsm = num_sms();
+  if (nsm <= 0) return FVATTN_ERR_CUDA;
+  cudaError_t e = route_pool(Q, K, shape, cfg, m, ws_layout(m, cfg->mode), static_cast<unsigned char*>(workspace),
+                             (int)block_begin, (int)block_end, nsm, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
+int fvattn_route_finish(const fvattn_shape* shape, const fvattn_route_cfg* cfg, const fvattn_csr* out,
+                        void* workspace, size_t workspace_bytes, fvattn_stream_t stream) {
+  int st = check_route_inputs(shape, cfg, workspace, workspace_bytes);
+  if (st != FVATTN_OK) return st;
+  st = check_csr_out(shape, cfg, out);
+  if (st != FVATTN_OK) return st;
+  const Dims m = make_dims(*shape, cfg->frame_len);
+  const int nsm = num_sms();
+  if (nsm <= 0) return FVATTN_ERR_CUDA;
+  cudaError_t e = route_finish(shape, cfg, out, m, ws_layout(m, cfg->mode), static_cast<unsigned char*>(workspace),
+                               nsm, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
 }
 
@@ -283,7 +347,7 @@ int fvattn_block_means(const void* X, const fvattn_shape* shape, double* out, fv
   const Dims m = make_dims(*shape, 0);
   const int nsm = num_sms();
   if (nsm <= 0) return FVATTN_ERR_CUDA;
-  cudaError_t e = launch_pool(X, nullptr, 1, shape->dtype, m, 0, 0, out, nullptr, nullptr, nullptr, SliceOut{}, nsm,
+  cudaError_t e = launch_pool(X, nullptr, 1, shape->dtype, m, 0, m.nb, 0, 0, out, nullptr, nullptr, nullptr, SliceOut{}, nsm,
                               reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
 }
@@ -315,7 +379,7 @@ int fvattn_block_scores(const void* Q, const void* K, const fvattn_shape* shape,
   const SliceOut so{reinterpret_cast<int8_t*>(ws + L.qs), reinterpret_cast<int8_t*>(ws + L.ks),
                     reinterpret_cast<int32_t*>(ws + L.eq), reinterpret_cast<int32_t*>(ws + L.ek)};
   if (cudaMemsetAsync(status, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
-  cudaError_t e = launch_pool(Q, K, 2, shape->dtype, m, 1, 0, nullptr, nullptr, nullptr, nullptr, so, nsm, s);
+  cudaError_t e = launch_pool(Q, K, 2, shape->dtype, m, 0, m.nb, 1, 0, nullptr, nullptr, nullptr, nullptr, so, nsm, s);
   if (e == cudaSuccess) e = launch_score_tc(so.qs, so.ks, so.eq, so.ek, m, softmax_scale(shape), scores, status, nsm, s);
   return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
 }

@@ -76,7 +76,7 @@ enum PoolOut { kMeans = 0, kSliced = 1, kFrameSums = 2 };
 
 template <typename T, int D, int OUT>
 __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ Q, const T* __restrict__ K,
-                                                   int ntensors, Dims m, int frame_len,
+                                                   int ntensors, Dims m, int b0, int nbr, int frame_len,
                                                    double* __restrict__ qo, double* __restrict__ ko,
                                                    double* __restrict__ qhi, double* __restrict__ khi,
                                                    SliceOut so) {
@@ -89,7 +89,8 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ Q, cons
   constexpr bool FRAME = OUT == kFrameSums;
   const int lane = threadIdx.x & 31;
   const int c = lane % CPR, r0 = lane / CPR;
-  const int64_t per = m.BH * m.nb;
+  // units: (tensor, head, block) over the blocks [b0, b0 + nbr) of every head
+  const int64_t per = m.BH * nbr;
   const int64_t units = per * ntensors;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
   // Software-pipelined over units: the first batch of the next unit is loaded before the current
@@ -97,13 +98,13 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ Q, cons
   auto src_of = [&](int64_t uu) -> const T* {
     const bool k_ = uu >= per;
     const int64_t row_ = k_ ? uu - per : uu;
-    const int64_t bh_ = row_ / m.nb;
-    const int64_t t0_ = (row_ - bh_ * m.nb) * kBlock;
+    const int64_t bh_ = row_ / nbr;
+    const int64_t t0_ = (b0 + (row_ - bh_ * nbr)) * kBlock;
     return (k_ ? K : Q) + (bh_ * m.S + t0_) * D + c * VEC;
   };
   auto nvalid_of = [&](int64_t uu) -> int {
     const int64_t row_ = uu >= per ? uu - per : uu;
-    return (int)imin<int64_t>(kBlock, m.S - (row_ % m.nb) * kBlock);
+    return (int)imin<int64_t>(kBlock, m.S - (b0 + row_ % nbr) * kBlock);
   };
   uint4 v[BATCH];
   int64_t u = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -118,9 +119,10 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ Q, cons
   }
   for (; u < units; u += nwarps) {
     const bool isK = u >= per;
-    const int64_t row = isK ? u - per : u;       // bh * nb + blk
-    const int64_t bh = row / m.nb;
-    const int blk = (int)(row - bh * m.nb);
+    const int64_t unit = isK ? u - per : u;      // bh * nbr + (blk - b0)
+    const int64_t bh = unit / nbr;
+    const int blk = b0 + (int)(unit - bh * nbr);
+    const int64_t row = bh * m.nb + blk;
     const int64_t t0 = (int64_t)blk * kBlock;
     const int nvalid = (int)imin<int64_t>(kBlock, m.S - t0);
     const T* X = (isK ? K : Q) + (bh * m.S + t0) * D + c * VEC;
@@ -1055,33 +1057,39 @@ __global__ void __launch_bounds__(256) csr_kernel(const uint32_t* __restrict__ b
 // ------------------------------------------------------------------ launchers
 
 template <typename T, int D>
-static cudaError_t launch_pool_td(const void* Q, const void* K, int ntensors, const Dims& m, int out, int frame_len,
-                                  double* qo, double* ko, double* qhi, double* khi, const SliceOut& so, int nsm,
-                                  cudaStream_t st) {
-  const int64_t units = m.BH * m.nb * ntensors;
+static cudaError_t launch_pool_td(const void* Q, const void* K, int ntensors, const Dims& m, int b0, int b1, int out,
+                                  int frame_len, double* qo, double* ko, double* qhi, double* khi, const SliceOut& so,
+                                  int nsm, cudaStream_t st) {
+  const int nbr = b1 - b0;
+  if (nbr <= 0) return cudaSuccess;
+  const int64_t units = m.BH * nbr * ntensors;
   const int grid = (int)imin<int64_t>((units + 3) / 4, (int64_t)nsm * 16);
   const T* q = static_cast<const T*>(Q);
   const T* k = static_cast<const T*>(K);
   if (out == kSliced)
-    pool_kernel<T, D, kSliced><<<grid, 128, 0, st>>>(q, k, ntensors, m, 0, nullptr, nullptr, nullptr, nullptr, so);
+    pool_kernel<T, D, kSliced><<<grid, 128, 0, st>>>(q, k, ntensors, m, b0, nbr, 0, nullptr, nullptr, nullptr, nullptr,
+                                                      so);
   else if (out == kFrameSums)
-    pool_kernel<T, D, kFrameSums><<<grid, 128, 0, st>>>(q, k, ntensors, m, frame_len, qo, ko, qhi, khi, so);
+    pool_kernel<T, D, kFrameSums><<<grid, 128, 0, st>>>(q, k, ntensors, m, b0, nbr, frame_len, qo, ko, qhi, khi, so);
   else
-    pool_kernel<T, D, kMeans><<<grid, 128, 0, st>>>(q, k, ntensors, m, 0, qo, ko, nullptr, nullptr, so);
+    pool_kernel<T, D, kMeans><<<grid, 128, 0, st>>>(q, k, ntensors, m, b0, nbr, 0, qo, ko, nullptr, nullptr, so);
   return cudaGetLastError();
 }
 
-// out: 0 = means [row][d], 1 = score slices and exponents, 2 = frame segment sums.
-cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int out, int frame_len,
-                        double* qo, double* ko, double* qhi, double* khi, const SliceOut& so, int nsm,
+// out: 0 = means [row][d], 1 = score slices and exponents, 2 = frame segment sums; blocks
+// [b0, b1) of every head.
+cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int b0, int b1, int out,
+                        int frame_len, double* qo, double* ko, double* qhi, double* khi, const SliceOut& so, int nsm,
                         cudaStream_t st) {
   if (dtype == FVATTN_BF16) {
     if (m.d == 128)
-      return launch_pool_td<__nv_bfloat16, 128>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, so, nsm, st);
-    return launch_pool_td<__nv_bfloat16, 64>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, so, nsm, st);
+      return launch_pool_td<__nv_bfloat16, 128>(Q, K, ntensors, m, b0, b1, out, frame_len, qo, ko, qhi, khi, so, nsm,
+                                                st);
+    return launch_pool_td<__nv_bfloat16, 64>(Q, K, ntensors, m, b0, b1, out, frame_len, qo, ko, qhi, khi, so, nsm, st);
   }
-  if (m.d == 128) return launch_pool_td<float, 128>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, so, nsm, st);
-  return launch_pool_td<float, 64>(Q, K, ntensors, m, out, frame_len, qo, ko, qhi, khi, so, nsm, st);
+  if (m.d == 128)
+    return launch_pool_td<float, 128>(Q, K, ntensors, m, b0, b1, out, frame_len, qo, ko, qhi, khi, so, nsm, st);
+  return launch_pool_td<float, 64>(Q, K, ntensors, m, b0, b1, out, frame_len, qo, ko, qhi, khi, so, nsm, st);
 }
 
 

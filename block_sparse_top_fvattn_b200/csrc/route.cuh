@@ -33,9 +33,10 @@ struct SliceOut {
 cudaError_t launch_score_tc(const int8_t* qs, const int8_t* ks, const int32_t* eq, const int32_t* ek, const Dims& m,
                             double scale, double* logits, int32_t* status, int nsm, cudaStream_t st);
 
-// out: 0 = means [row][d] (qo, ko), 1 = score slices and exponents (so), 2 = frame segment sums.
-cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int out, int frame_len,
-                        double* qo, double* ko, double* qhi, double* khi, const SliceOut& so, int nsm,
+// out: 0 = means [row][d] (qo, ko), 1 = score slices and exponents (so), 2 = frame segment sums;
+// the blocks [b0, b1) of every head (outputs at their full-layout rows).
+cudaError_t launch_pool(const void* Q, const void* K, int ntensors, int dtype, const Dims& m, int b0, int b1, int out,
+                        int frame_len, double* qo, double* ko, double* qhi, double* khi, const SliceOut& so, int nsm,
                         cudaStream_t st);
 // Slack-aware augmentation of 128-row tiles (fvattn_route_cfg.sasa_coef / sasa_trigger).
 struct SasaCfg {

@@ -26,7 +26,8 @@ import numpy as np
 import torch
 import torch.distributed as dist
 
-from . import RouteConfig, alloc_csr, rlb_plan, route, select_heads, sparse_attn
+from . import (RouteConfig, alloc_csr, rlb_plan, route, route_finish, route_pool, select_heads, sparse_attn,
+               workspace_bytes)
 
 
 class Kernels:
@@ -38,6 +39,17 @@ class Kernels:
     def route(self, q: torch.Tensor, k: torch.Tensor):
         B, H, S, _ = q.shape
         return route(q, k, self.cfg, csr=alloc_csr(B, H, S, q.device, codes=self.cfg.frame_exact))
+
+    # The router in two stages (fvattn_route_pool / fvattn_route_finish), for pooling the blocks
+    # of each part of the sequence as it arrives.
+    def begin_route(self, q: torch.Tensor):
+        return torch.empty(workspace_bytes(q, self.cfg), dtype=torch.uint8, device=q.device)
+
+    def pool_blocks(self, handle, q: torch.Tensor, k: torch.Tensor, block_begin: int, block_end: int) -> None:
+        route_pool(q, k, self.cfg, block_begin, block_end, handle)
+
+    def finish_route(self, handle, q: torch.Tensor):
+        return route_finish(q, self.cfg, handle)
 
     @staticmethod
     def head_load(state) -> torch.Tensor:
@@ -91,9 +103,10 @@ def _exchange(ops) -> None:
 
 def balanced_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cfg: Optional[RouteConfig] = None, *,
                        group=None, target: float = 1.05, max_moves_per_rank: int = 1,
-                       kernels=None) -> Tuple[torch.Tensor, Plan]:
+                       kernels=None, state=None) -> Tuple[torch.Tensor, Plan]:
     """Block-sparse attention of this rank's heads with runtime head migration between ranks.
-    q, k, v: [1, Hl, S, d], the same Hl, S, d and dtype on every rank. Returns (O, plan)."""
+    q, k, v: [1, Hl, S, d], the same Hl, S, d and dtype on every rank; `state`: the routing of
+    these heads when the caller already has it. Returns (O, plan)."""
     if q.shape[0] != 1:
         raise ValueError("expected [1, Hl, S, d] per rank")
     kernels = kernels or Kernels(cfg or RouteConfig())
@@ -101,7 +114,8 @@ def balanced_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cfg: O
     peer = (lambda r: dist.get_global_rank(group, r)) if group is not None else (lambda r: r)
     _, Hl, S, d = q.shape
 
-    state = kernels.route(q, k)
+    if state is None:
+        state = kernels.route(q, k)
     plan = make_plan(gather_loads(kernels.head_load(state), group), target, max_moves_per_rank)
     out = torch.empty_like(q)
 

@@ -187,6 +187,27 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape,
                  void* workspace, size_t workspace_bytes, fvattn_stream_t stream);
 
 /*
+ * fvattn_route in two stages, so that step 1 can run on parts of the sequence as they arrive
+ * (sequence parallelism: the slices of a head come from different ranks):
+ *   fvattn_route_pool   -- step 1 (block means: score slices in Top-p / top-k modes, segment
+ *                          sums in frame mode) for the blocks [block_begin, block_end) of every
+ *                          head, into the workspace; reads only those blocks' tokens of Q and K.
+ *                          0 <= block_begin < block_end <= nb, else FVATTN_ERR_INVALID.
+ *   fvattn_route_finish -- steps 2 and 3 from a workspace in which every block of every head has
+ *                          been pooled (by one or more fvattn_route_pool calls on the same
+ *                          shape, cfg and workspace, ordered before it on `stream` or joined to
+ *                          it by the caller); writes `out` as fvattn_route does.
+ * fvattn_route(Q, K, ...) equals fvattn_route_pool over [0, nb) followed by
+ * fvattn_route_finish, bit for bit. Arguments, workspace size and errors as for fvattn_route.
+ */
+int fvattn_route_pool(const void* Q, const void* K, const fvattn_shape* shape,
+                      const fvattn_route_cfg* cfg, int64_t block_begin, int64_t block_end,
+                      void* workspace, size_t workspace_bytes, fvattn_stream_t stream);
+int fvattn_route_finish(const fvattn_shape* shape, const fvattn_route_cfg* cfg,
+                        const fvattn_csr* out, void* workspace, size_t workspace_bytes,
+                        fvattn_stream_t stream);
+
+/*
  * fvattn_sparse_attn -- exact softmax attention over the selected key blocks:
  *   O[t] = sum_u softmax_u(Q[t].K[u] * scale) V[u],  u over the tokens (< S) of the key
  *   blocks listed in the CSR row of t's query block.

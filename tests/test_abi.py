@@ -144,6 +144,23 @@ def test_route_rejects_on_host_before_any_launch(lib):
                             None) == -2
 
 
+def test_two_stage_route_rejects_on_host_before_any_launch(lib):
+    s, c = shape(), cfg()                       # S = 1000: nb = 16
+    ws = lib.fvattn_route_workspace_bytes(ctypes.byref(s), ctypes.byref(c))
+    csr = _fake_csr(lib.fvattn_csr_max_nnz(ctypes.byref(s)))
+    P = 4096
+    pool = lib.fvattn_route_pool
+    assert pool(None, P, ctypes.byref(s), ctypes.byref(c), 0, 16, P, ws, None) == -1
+    assert pool(P, P, ctypes.byref(s), ctypes.byref(c), 0, 16, P, ws - 1, None) == -3
+    for b0, b1 in ((-1, 4), (4, 4), (10, 17), (5, 3)):
+        assert pool(P, P, ctypes.byref(s), ctypes.byref(c), b0, b1, P, ws, None) == -1
+    assert pool(P, P, ctypes.byref(shape(d=96)), ctypes.byref(c), 0, 16, P, ws, None) == -2
+    fin = lib.fvattn_route_finish
+    assert fin(ctypes.byref(s), ctypes.byref(c), None, P, ws, None) == -1
+    assert fin(ctypes.byref(s), ctypes.byref(c), ctypes.byref(csr), None, ws, None) == -1
+    assert fin(ctypes.byref(s), ctypes.byref(c), ctypes.byref(_fake_csr(10)), P, ws, None) == -3
+
+
 def test_attention_and_status_reject_on_host(lib):
     s = shape()
     csr = _fake_csr(1)

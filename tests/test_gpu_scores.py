@@ -4,7 +4,8 @@ element, within a bound derived from the arithmetic: the pooling's fp32 partial 
 rows (error <= 3 * 2^-24 * mean|x| per mean) plus the slices' dropped terms (below 2^-30 *
 2^(e_i + e_j), here bounded by 2^-24 * d * max|Qbar_i| * max|Kbar_j|). A wrong digit, level or
 exponent moves a score by at least 2^-8 of its size. Also the stamped attention entry point
-(per-CTA SM ids and busy intervals): same output as the plain call, valid stamps."""
+(per-CTA SM ids and busy intervals: same output as the plain call, valid stamps) and the
+two-stage router (pooling by block ranges, then the rest: the same CSR as fvattn_route)."""
 import importlib
 
 import numpy as np
@@ -88,3 +89,42 @@ def test_stamped_attention_rejects_fp32():
     csr = fv.route(x["q"], x["k"], fv.RouteConfig(p=0.9))
     with pytest.raises(fv.FvattnError):
         fv.sparse_attn_stamped(x["q"], x["k"], x["v"], csr)
+
+
+SPLIT_CASES = [
+    ("single", dict(H=3, S=3000), fv.RouteConfig(p=0.9), [(20, 47), (0, 20)]),                  # ragged tail last
+    ("single", dict(H=2, S=4096), fv.RouteConfig(p=0.8, local_window=1), [(32, 64), (0, 8), (8, 32)]),
+    ("single", dict(H=2, S=3120, frame_len=1560), fv.RouteConfig(mode="frame_topk", topk_frames=1, frame_len=1560,
+                                                                   frame_window=0, force_first_frame=True),
+     [(25, 49), (0, 25)]),
+]
+
+
+@pytest.mark.parametrize("name,over,cfg,ranges", SPLIT_CASES)
+def test_split_route_equals_route(name, over, cfg, ranges):
+    """fvattn_route_pool over block ranges in any order, then fvattn_route_finish, gives the CSR
+    of fvattn_route bit for bit (the same kernels on the same blocks)."""
+    w = get_workload(name).replace(**over)
+    x = make_inputs(w, device="cuda")
+    q, k = x["q"], x["k"]
+    a = fv.route(q, k, cfg)
+    ws = torch.empty(fv.workspace_bytes(q, cfg), dtype=torch.uint8, device="cuda")
+    for b0, b1 in ranges:
+        fv.route_pool(q, k, cfg, b0, b1, ws)
+    b = fv.route_finish(q, cfg, ws)
+    torch.cuda.synchronize()
+    assert fv.read_status(a) == 0 and fv.read_status(b) == 0
+    for f in ("row_ptr", "head_load", "tile_cost", "tile_order", "nnz"):
+        assert torch.equal(getattr(a, f), getattr(b, f)), f
+    n = int(a.nnz.item())
+    assert torch.equal(a.col_idx[:n], b.col_idx[:n])
+
+
+def test_route_pool_rejects_bad_ranges():
+    w = get_workload("single").replace(H=1, S=1000)
+    x = make_inputs(w, device="cuda")
+    cfg = fv.RouteConfig(p=0.9)
+    ws = torch.empty(fv.workspace_bytes(x["q"], cfg), dtype=torch.uint8, device="cuda")
+    for b0, b1 in ((-1, 4), (4, 4), (10, 17), (5, 3)):
+        with pytest.raises(fv.FvattnError):
+            fv.route_pool(x["q"], x["k"], cfg, b0, b1, ws)

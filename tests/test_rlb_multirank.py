@@ -32,6 +32,22 @@ class OracleKernels:
     def route(self, q, k):
         return self.o.route(q[0], k[0], self.cfg)
 
+    # the router in two stages: record the pooled block ranges, route on the full heads at the end
+    def begin_route(self, q):
+        return {"ranges": []}
+
+    def pool_blocks(self, handle, q, k, b0, b1):
+        handle["ranges"].append((b0, b1))
+        handle["q"], handle["k"] = q, k          # the full heads, filled slice by slice
+
+    def finish_route(self, handle, q):
+        nb = -(-q.shape[2] // 64)
+        covered = sorted(handle["ranges"])
+        assert covered[0][0] == 0 and covered[-1][1] == nb
+        assert all(a[1] == b[0] for a, b in zip(covered, covered[1:])), covered
+        assert handle["q"] is q
+        return self.route(handle["q"], handle["k"])
+
     def head_load(self, state):
         return torch.from_numpy(self.o.head_loads(state["mask"]))
 
@@ -82,7 +98,7 @@ def test_balanced_attention_gloo(world):
     assert out[0][3] < out[0][2]                  # the imbalance went down
 
 
-def _ulysses_worker(rank, world, port, balance, out):
+def _ulysses_worker(rank, world, port, balance, overlap, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -94,7 +110,7 @@ def _ulysses_worker(rank, world, port, balance, out):
         Sl = w.S // world
         shard = [t[:, :, rank * Sl:(rank + 1) * Sl].contiguous() for t in (x["q"], x["k"], x["v"])]
         kern = OracleKernels(0.9)
-        o, plan = ulysses.ulysses_attention(*shard, group=None, balance=balance, target=1.0,
+        o, plan = ulysses.ulysses_attention(*shard, group=None, balance=balance, target=1.0, overlap_pool=overlap,
                                             max_moves_per_rank=1, kernels=kern)
         ref = torch.empty_like(x["q"])
         kern.attend(x["q"], x["k"], x["v"], kern.route(x["q"], x["k"]), None, ref)
@@ -104,14 +120,15 @@ def _ulysses_worker(rank, world, port, balance, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,balance", [(2, False), (2, True), (3, True)])
-def test_ulysses_attention_gloo(world, balance):
+@pytest.mark.parametrize("world,balance,overlap", [(2, False, False), (2, True, False), (3, True, False),
+                                                   (2, False, True), (3, True, True)])
+def test_ulysses_attention_gloo(world, balance, overlap):
     # sequence -> heads all-to-all, routing and attention of the local heads (with head migration
     # when balance), heads -> sequence: each rank's output slice equals the single-process
     # oracle attention of the whole layer
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.start_processes(_ulysses_worker, args=(world, _free_port(), balance, out), nprocs=world,
+    mp.start_processes(_ulysses_worker, args=(world, _free_port(), balance, overlap, out), nprocs=world,
                        start_method="spawn", join=True)
     for r in range(world):
         assert out[r] == 0.0, (r, out[r])
