@@ -25,6 +25,20 @@ def test_header_declares_the_boundary():
         assert n in names
 
 
+def test_header_is_plain_c(tmp_path):
+    # the boundary has no C++ or torch types: the header compiles as C99 with warnings as errors
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text('#include "fvattn.h"\nint main(void) { return fvattn_version() > 0 ? 0 : 1; }\n')
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.dirname(HEADER),
+                        "-c", str(src), "-o", str(tmp_path / "use.o")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
 def test_library_exports_every_declared_symbol(lib):
     for n in declared_functions():
         assert hasattr(lib, n), n
