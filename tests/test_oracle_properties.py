@@ -69,3 +69,13 @@ def test_topk_keeps_the_k_largest_scores(logits, k):
     for a in kept:
         for b in dropped:
             assert sc[a] > sc[b] or (sc[a] == sc[b] and a < b)
+
+
+@given(st.sampled_from([2, 4, 8, 16, 32]), st.data())
+def test_topp_cut_reaching_p_exactly_keeps_that_prefix(n, data):
+    # uniform rows of a power-of-two length: every prefix mass m/n is exact in binary, so a cut
+    # at p = m/n must keep exactly m blocks ("reaches p": >=, not >), the lowest indices first
+    m = data.draw(st.integers(min_value=1, max_value=n - 1))
+    pi = R.row_softmax(np.zeros((1, n)))[0]
+    order, k, csum = R.topp_row(pi, m / n)
+    assert k == m and list(order[:k]) == list(range(m))
