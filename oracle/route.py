@@ -6,6 +6,7 @@ Test infrastructure only (see the package docstring); never used by the product 
 from __future__ import annotations
 
 import dataclasses
+import itertools
 import math
 from typing import Optional
 
@@ -367,8 +368,10 @@ def valid_sasa_row(key_row: np.ndarray, base_row: np.ndarray, partner_row: np.nd
 def near_tie_rows(r: dict, S: int, cfg: RouteCfg) -> np.ndarray:
     """Rows whose selection is decided by a difference below the stated resolution:
     a cumulative mass within EPS_MASS of p at the cut (k* or k*-1 blocks), or a probability
-    gap under EPS_GAP between the last block kept and the first block left out. In frame
-    mode: a score gap under EPS_GAP at the top-k boundary of any frame the row touches."""
+    gap under EPS_GAP between the last block kept and the first block left out. Top-k mode: a
+    gap under EPS_GAP * max(1, |s|) between the k-th and the (k+1)-th score s (the scores are
+    unnormalised logits, whose rounding grows with their magnitude). Frame mode: a frame-score
+    gap under EPS_GAP at the top-k boundary of any frame the row touches."""
     mask = r["mask"]
     BH, nb, _ = mask.shape
     near = np.zeros((BH, nb), dtype=bool)
@@ -379,7 +382,7 @@ def near_tie_rows(r: dict, S: int, cfg: RouteCfg) -> np.ndarray:
         for bh in range(BH):
             for i in range(nb):
                 srt = np.sort(r["scores"][bh, i])[::-1]
-                near[bh, i] = (srt[k - 1] - srt[k]) < EPS_GAP * max(1.0, abs(srt[k - 1]))
+                near[bh, i] = (srt[k - 1] - srt[k]) < _gap_eps(srt[k - 1], "topk")
         return near
     if cfg.mode == "topp":
         if cfg.p >= 1.0:
@@ -411,11 +414,37 @@ def near_tie_rows(r: dict, S: int, cfg: RouteCfg) -> np.ndarray:
     return near
 
 
+def _kept_sets(scores: np.ndarray, k: int, eps: float):
+    """Every set of k indices that the top-k rule can keep when scores closer than `eps` are
+    taken as tied. With hi the k-th and lo the (k+1)-th highest score, an index is ranked
+    clearly inside when its score is at least lo + eps (no tie with anything left out) and
+    clearly outside when it is at most hi - eps; the set is the clearly-inside indices plus any
+    choice of the rest. When hi - lo >= eps this is the top-k set alone. Yields boolean masks."""
+    n = scores.shape[0]
+    k = min(k, n)
+    srt = np.sort(scores)[::-1]
+    hi_cut = srt[k - 1]
+    lo_cut = srt[k] if k < n else -np.inf
+    must = (scores - lo_cut) >= eps
+    band = ~must & ((hi_cut - scores) < eps)
+    need = k - int(must.sum())
+    for pick in itertools.combinations(np.nonzero(band)[0].tolist(), need):
+        m = must.copy()
+        m[list(pick)] = True
+        yield m
+
+
 def valid_near_tie_set(r: dict, bh: int, i: int, gpu_row: np.ndarray, S: int, cfg: RouteCfg) -> bool:
     """Is `gpu_row` (boolean [nb]) an acceptable selection for a near-tie row?
 
-    It must hold every forced block and every block clearly above the cut, hold nothing
-    clearly below it, and (Top-p) reach mass p - EPS_MASS."""
+    A near-tie row's selection may differ from the oracle's only by the order of scores closer
+    than the stated resolution (a gap under EPS_GAP, in probability units for Top-p, relative
+    to the score in top-k mode, absolute for frame scores). So `gpu_row` must hold every forced
+    block and be the forced set united with a selection the rule could make under such a
+    reordering. Top-p: every block ranked clearly above the cut kept, none clearly below, and
+    a kept mass of at least p - EPS_MASS. Top-k: exactly k routed blocks, chosen as in
+    _kept_sets. Frame mode: per touched query frame exactly k key frames, chosen as in
+    _kept_sets, united over the frames the query block touches and expanded to key blocks."""
     forced = r["forced"][i]
     gpu_row = np.asarray(gpu_row, dtype=bool)
     if np.any(forced & ~gpu_row):
@@ -423,39 +452,32 @@ def valid_near_tie_set(r: dict, bh: int, i: int, gpu_row: np.ndarray, S: int, cf
     if cfg.mode == "topk":
         sc = r["scores"][bh, i]
         k = min(cfg.topk_blocks, sc.shape[0])
-        srt = np.sort(sc)[::-1]
-        eps = EPS_GAP * max(1.0, abs(srt[k - 1]))
-        lo_cut = srt[k] if k < sc.shape[0] else -np.inf
-        must = (sc > srt[k - 1] + eps) | forced
-        may = (sc >= lo_cut - eps) | forced
-        return bool(np.all(gpu_row[must]) and not np.any(gpu_row & ~may))
+        eps = _gap_eps(np.sort(sc)[::-1][k - 1], "topk")
+        return any(np.array_equal(m | forced, gpu_row) for m in _kept_sets(sc, k, eps))
     if cfg.mode == "topp":
         pi = r["pi"][bh, i]
         order, ks, csum = topp_row(pi, cfg.p)
         srt = pi[order]
         hi_cut = srt[ks - 1]
         lo_cut = srt[ks] if ks < pi.shape[0] else -np.inf
-        must = (pi > hi_cut + EPS_GAP) | forced
-        may = (pi >= lo_cut - EPS_GAP) | forced
+        must = ((pi - hi_cut) >= EPS_GAP) | forced
+        may = ((lo_cut - pi) < EPS_GAP) | forced
         if pi[gpu_row].sum() < cfg.p - EPS_MASS:
             return False
-    else:
-        fs = r["frame_scores"][bh]
-        F = fs.shape[0]
-        k = min(cfg.topk_frames, F)
-        f0, f1 = _frames_of_block(i, S, cfg.block, cfg.frame_len)
-        fm = np.zeros(F, dtype=bool)
-        fy = np.zeros(F, dtype=bool)
-        for f in range(f0, f1 + 1):
-            srt = np.sort(fs[f])[::-1]
-            hi_cut = srt[k - 1]
-            lo_cut = srt[k] if k < F else -np.inf
-            fm |= fs[f] > hi_cut + EPS_GAP
-            fy |= fs[f] >= lo_cut - EPS_GAP
-        inc = frame_incidence(S, cfg.block, cfg.frame_len)
-        must = _blocks_touching_frames(fm, inc) | forced
-        may = _blocks_touching_frames(fy, inc) | forced
-    return bool(np.all(gpu_row[must]) and not np.any(gpu_row & ~may))
+        return bool(np.all(gpu_row[must]) and not np.any(gpu_row & ~may))
+    fs = r["frame_scores"][bh]
+    F = fs.shape[0]
+    k = min(cfg.topk_frames, F)
+    f0, f1 = _frames_of_block(i, S, cfg.block, cfg.frame_len)
+    inc = frame_incidence(S, cfg.block, cfg.frame_len)
+    options = [list(_kept_sets(fs[f], k, EPS_GAP)) for f in range(f0, f1 + 1)]
+    if math.prod(len(o) for o in options) > 200_000:
+        raise ValueError("too many tied frame choices to enumerate")
+    for combo in itertools.product(*options):
+        sel = np.logical_or.reduce(combo)
+        if np.array_equal(_blocks_touching_frames(sel, inc) | forced, gpu_row):
+            return True
+    return False
 
 
 # ---------------------------------------------------------------- token-exact frame selection
