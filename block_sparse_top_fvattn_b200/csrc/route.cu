@@ -335,8 +335,12 @@ __device__ void topp_select(double* E, int n, double p, uint32_t* w, int lane) {
   const double P = p * z;
   __syncwarp();
 
-  // Max extraction. Each lane keeps the best (key, slot) of its unselected elements.
-  uint64_t taken = 0;                       // bit e: element lane + 32 e is selected
+  // Max extraction. Each lane keeps the best (key, slot) of its unselected elements. The
+  // selected elements are marked in the row's bitmask words themselves (element lane + 32 e is
+  // bit `lane` of w[e]), so rows of any length are covered; only the lane that owns an element
+  // ever sets its bit.
+  for (int q = lane; q < nw; q += 32) w[q] = 0u;
+  __syncwarp();
   uint32_t bkey = 0;
   int bslot = -1;
   auto rescan = [&]() {
@@ -344,7 +348,7 @@ __device__ void topp_select(double* E, int n, double p, uint32_t* w, int lane) {
     bslot = -1;
     for (int e = 0; e < nw; ++e) {
       const int j = lane + 32 * e;
-      if (j < n && !((taken >> e) & 1ull)) {
+      if (j < n && !((w[e] >> lane) & 1u)) {
         const uint32_t k = wkey(E[j]);
         if (bslot < 0 || k > bkey) { bkey = k; bslot = e; }
       }
@@ -360,19 +364,13 @@ __device__ void topp_select(double* E, int n, double p, uint32_t* w, int lane) {
     if (gj == 0xffffffffu) break;
     acc += E[gj];
     if ((int)(gj & 31) == lane) {
-      taken |= 1ull << (gj >> 5);
+      atomicOr(&w[gj >> 5], 1u << lane);
       rescan();
     }
+    __syncwarp();
     done = acc >= P;
   }
-  if (done) {
-    for (int e = 0; e < nw; ++e) {
-      const uint32_t word = __ballot_sync(0xffffffffu, (taken >> e) & 1ull);
-      if (lane == 0) w[e] = word;
-    }
-    __syncwarp();
-    return;
-  }
+  if (done) return;                          // w holds exactly the extracted elements
   // Bisection: largest T with mass{key >= T} >= P. M(0) = z >= P; keys are below 2^31.
   uint32_t lo = 0, hi = 0x7f800001u;
   while (hi - lo > 1) {

@@ -389,12 +389,14 @@ def test_full_length_long_frame_mode_sampled_heads():
 
 
 # The three register/shared-memory variants of the per-row cut: rows of <= 512 blocks, of
-# 513..1280 blocks (the long layer's 1182) and of more than 1280 blocks (shared-memory cut),
-# each with the full block lists checked and attention on a sample of query blocks.
+# 513..1280 blocks (the long layer's 1182) and of more than 1280 blocks (shared-memory cut, also
+# past 2048 blocks, where a row's bitmask has more than 64 words), each with the full block
+# lists checked and attention on a sample of query blocks.
 @pytest.mark.slow
 @pytest.mark.parametrize("S,extra", [
     (75600, {}),                                                        # nb = 1182
     (1290 * 64 + 17, {}),                                               # nb = 1291: shared-memory cut
+    (2100 * 64, {}),                                                    # nb = 2100: 66 mask words per row
     (700 * 64, {"mode": "topk", "topk_blocks": 40}),                    # nb = 700, top-k
     (700 * 64 + 5, {"sasa_coef": 0.5, "sasa_trigger": 2}),               # nb = 701, tile augmentation
 ])
