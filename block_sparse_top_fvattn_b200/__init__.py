@@ -25,7 +25,8 @@ from ._lib import (FVATTN_BF16, FVATTN_F32, FVATTN_MODE_FRAME_TOPK, FVATTN_MODE_
 
 __all__ = ["RouteConfig", "CsrBuffers", "alloc_csr", "route", "route_pool", "route_finish", "sparse_attn",
            "sparse_attn_stamped",
-           "sm_busy_imbalance", "block_means", "block_scores",
+           "sm_busy_imbalance", "block_means", "block_scores", "sparse_attn_timeout_check",
+           "block_scores_timeout_check",
            "read_status",
            "workspace_bytes", "shape_of", "load", "FvattnError", "status_string", "rlb_plan", "select_heads",
            "LazyRouter"]
@@ -291,6 +292,42 @@ def block_scores(q: torch.Tensor, k: torch.Tensor, scale: float = 0.0,
     if code != 0:
         raise FvattnError(code, "fvattn_block_scores (device status)")
     return out.view(B, H, nb, ld)[..., :nb]
+
+
+def sparse_attn_timeout_check(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, csr: CsrBuffers, out: torch.Tensor,
+                              polls: int = 64, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """fvattn_sparse_attn_timeout_check: the attention kernel with a first bounded wait on a
+    barrier that nothing completes, so that it times out before any copy or MMA. Returns the
+    device status word afterwards (FVATTN_ERR_TIMEOUT expected); `out` is left unwritten."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _check_tensor(t, n)
+    lib = load()
+    check(lib.fvattn_sparse_attn_timeout_check(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(shape_of(q)),
+                                               ctypes.byref(csr.to_c()), out.data_ptr(), int(polls), _stream(stream)),
+          "fvattn_sparse_attn_timeout_check")
+    return read_status(csr, stream)
+
+
+def block_scores_timeout_check(q: torch.Tensor, k: torch.Tensor, polls: int = 64,
+                               stream: Optional[torch.cuda.Stream] = None) -> Tuple[int, torch.Tensor]:
+    """fvattn_block_scores_timeout_check: the block-score kernel with a first bounded wait on a
+    barrier that nothing completes. Returns (device status word, the score buffer, filled with NaN
+    before the call and left unwritten by the kernel)."""
+    _check_tensor(q, "q")
+    _check_tensor(k, "k")
+    B, H, S, d = q.shape
+    shp = shape_of(q)
+    lib = load()
+    nws = lib.fvattn_block_scores_workspace_bytes(ctypes.byref(shp))
+    ld = lib.fvattn_block_scores_ld(ctypes.byref(shp))
+    ws = torch.empty(nws, dtype=torch.uint8, device=q.device)
+    out = torch.full((B * H * -(-S // BLOCK), ld), float("nan"), dtype=torch.float64, device=q.device)
+    status = torch.zeros(4, dtype=torch.int32, device=q.device)
+    check(lib.fvattn_block_scores_timeout_check(q.data_ptr(), k.data_ptr(), ctypes.byref(shp), out.data_ptr(),
+                                                ws.data_ptr(), nws, status.data_ptr(), int(polls), _stream(stream)),
+          "fvattn_block_scores_timeout_check")
+    (stream if stream is not None else torch.cuda.current_stream(q.device)).synchronize()
+    return int(status[0].item()), out
 
 
 def read_status(csr: CsrBuffers, stream: Optional[torch.cuda.Stream] = None) -> int:

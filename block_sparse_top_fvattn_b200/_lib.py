@@ -90,6 +90,11 @@ def load() -> ctypes.CDLL:
     lib.fvattn_attn_stamp_words.argtypes = [P(Shape)]
     lib.fvattn_sparse_attn_stamped.restype = ctypes.c_int
     lib.fvattn_sparse_attn_stamped.argtypes = [vp, vp, vp, P(Shape), P(Csr), vp, vp, vp, ctypes.c_int64, vp]
+    lib.fvattn_sparse_attn_timeout_check.restype = ctypes.c_int
+    lib.fvattn_sparse_attn_timeout_check.argtypes = [vp, vp, vp, P(Shape), P(Csr), vp, ctypes.c_uint32, vp]
+    lib.fvattn_block_scores_timeout_check.restype = ctypes.c_int
+    lib.fvattn_block_scores_timeout_check.argtypes = [vp, vp, P(Shape), vp, vp, ctypes.c_size_t, vp, ctypes.c_uint32,
+                                                      vp]
     lib.fvattn_read_status.restype = ctypes.c_int
     lib.fvattn_read_status.argtypes = [P(Csr), vp]
     lib.fvattn_route_static_scratch.restype = ctypes.c_int

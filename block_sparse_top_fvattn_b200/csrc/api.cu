@@ -275,7 +275,7 @@ int fvattn_route_finish(const fvattn_shape* shape, const fvattn_route_cfg* cfg, 
 namespace {
 
 int sparse_attn(const void* Q, const void* K, const void* V, const fvattn_shape* shape, const fvattn_csr* csr,
-                void* O, float* lse, uint64_t* stamps, fvattn_stream_t stream) {
+                void* O, float* lse, uint64_t* stamps, fvattn_stream_t stream, uint32_t hold_polls = 0) {
   int st = validate_shape(shape);
   if (st != FVATTN_OK) return st;
   if (!Q || !K || !V || !O || !csr || !csr->row_ptr || !csr->col_idx || !csr->tile_order || !csr->status)
@@ -295,7 +295,7 @@ int sparse_attn(const void* Q, const void* K, const void* V, const fvattn_shape*
     if (nsm <= 0) return FVATTN_ERR_CUDA;
     if (cudaMemsetAsync(csr->status + 2, 0, sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
     e = launch_attn_tc(Q, K, V, m, scale, csr->row_ptr, csr->col_idx, csr->col_code, csr->tile_order, csr->status, O,
-                       lse, stamps, nsm, s);
+                       lse, stamps, hold_polls, nsm, s);
   }
   return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
 }
@@ -381,6 +381,39 @@ int fvattn_block_scores(const void* Q, const void* K, const fvattn_shape* shape,
   if (cudaMemsetAsync(status, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
   cudaError_t e = launch_pool(Q, K, 2, shape->dtype, m, 0, m.nb, 1, 0, nullptr, nullptr, nullptr, nullptr, so, nsm, s);
   if (e == cudaSuccess) e = launch_score_tc(so.qs, so.ks, so.eq, so.ek, m, softmax_scale(shape), scores, status, nsm, s);
+  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
+int fvattn_sparse_attn_timeout_check(const void* Q, const void* K, const void* V, const fvattn_shape* shape,
+                                     const fvattn_csr* csr, void* O, uint32_t polls, fvattn_stream_t stream) {
+  const int st = validate_shape(shape);
+  if (st != FVATTN_OK) return st;
+  if (shape->dtype != FVATTN_BF16) return FVATTN_ERR_UNSUPPORTED;
+  if (polls == 0) return FVATTN_ERR_INVALID;
+  return sparse_attn(Q, K, V, shape, csr, O, nullptr, nullptr, stream, polls);
+}
+
+int fvattn_block_scores_timeout_check(const void* Q, const void* K, const fvattn_shape* shape, double* scores,
+                                      void* workspace, size_t workspace_bytes, int32_t* status, uint32_t polls,
+                                      fvattn_stream_t stream) {
+  const int st = validate_shape(shape);
+  if (st != FVATTN_OK) return st;
+  if (!Q || !K || !scores || !workspace || !status || polls == 0) return FVATTN_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(scores, 16) || !aligned(workspace, 256) || !aligned(status, 4))
+    return FVATTN_ERR_INVALID;
+  const Dims m = make_dims(*shape, 0);
+  const WsLayout L = ws_layout(m, FVATTN_MODE_TOPP);
+  if (workspace_bytes < L.logits) return FVATTN_ERR_CAPACITY;
+  const int nsm = num_sms();
+  if (nsm <= 0) return FVATTN_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  const SliceOut so{reinterpret_cast<int8_t*>(ws + L.qs), reinterpret_cast<int8_t*>(ws + L.ks),
+                    reinterpret_cast<int32_t*>(ws + L.eq), reinterpret_cast<int32_t*>(ws + L.ek)};
+  if (cudaMemsetAsync(status, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
+  cudaError_t e = launch_pool(Q, K, 2, shape->dtype, m, 0, m.nb, 1, 0, nullptr, nullptr, nullptr, nullptr, so, nsm, s);
+  if (e == cudaSuccess)
+    e = launch_score_tc(so.qs, so.ks, so.eq, so.ek, m, softmax_scale(shape), scores, status, nsm, s, polls);
   return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
 }
 

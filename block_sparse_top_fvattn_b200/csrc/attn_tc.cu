@@ -23,8 +23,10 @@
 // even when the phase is already complete (measured), so that thread waits only twice per step:
 // once for K_j (whose barrier also publishes the step record) and once for P_j together with
 // V_j (one barrier); coincident events share one barrier and one commit.
-// Every mbarrier wait is bounded; a wait that runs out sets an abort flag, every role
-// unwinds, TMEM is freed and FVATTN_ERR_TIMEOUT is written to the device status word.
+// Every mbarrier wait is bounded; a wait that runs out sets an abort flag and every role
+// unwinds: the loaders wait (bounded) for the copies they issued, the MMA thread for its MMAs,
+// TMEM is freed and FVATTN_ERR_TIMEOUT is written to the device status word. With hold_polls > 0
+// (failure-path check only) the scheduler first waits on a barrier that nothing completes.
 #include <cuda.h>
 #include <math.h>
 
@@ -74,6 +76,10 @@ struct TcBars {
   uint64_t o_full, o_empty;
   uint64_t sched_full[2], sched_empty[2];
   uint64_t info_full[NI];
+  uint64_t hold;              // completed by nothing: the failure-path check waits on it
+  uint64_t drain;             // MMA drain: every MMA of the CTA has completed
+  int p_arrived[4];           // per softmax warp: the last step whose P it published
+  int v_armed;                // the last step whose V load was issued
   int sched_tile[2];
   int step_info[NI];          // key block j | membership mask << 28 | last step of tile << 30
   int step_code[NI];          // token mask of the step: allow bits of block 2t (0-3) and 2t+1 (4-7),
@@ -171,7 +177,7 @@ __global__ void __launch_bounds__(192, 2)
                    const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
                    const int32_t* __restrict__ col_code, const int32_t* __restrict__ tile_order,
                    int32_t* __restrict__ control, __nv_bfloat16* __restrict__ O, float* __restrict__ lse,
-                   uint64_t* __restrict__ stamps) {
+                   uint64_t* __restrict__ stamps, uint32_t hold_polls) {
   using L = TcLayout<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -200,6 +206,10 @@ __global__ void __launch_bounds__(192, 2)
     for (int s = 0; s < NI; ++s) tc::mbar_init(&bars->info_full[s], 1);
     tc::mbar_init(&bars->o_full, 1);
     tc::mbar_init(&bars->o_empty, 4);
+    tc::mbar_init(&bars->hold, 1);
+    tc::mbar_init(&bars->drain, 1);
+    for (int w = 0; w < 4; ++w) bars->p_arrived[w] = -1;
+    bars->v_armed = -1;
     bars->abort = 0;
     tc::fence_mbar_init();
   }
@@ -235,7 +245,12 @@ __global__ void __launch_bounds__(192, 2)
       // fvattn_select_heads (control[3]).
       const int64_t count = imin<int64_t>(ntiles, imax<int64_t>(0, *reinterpret_cast<volatile int32_t*>(&control[3])));
       uint32_t g = 0;
-      for (uint32_t n = 0;; ++n) {
+      // parities of the last phases this thread armed (-1: none), waited for before it leaves,
+      // so that no copy is still writing shared memory when the CTA exits
+      int q_par = -1, k_par[NS] = {-1, -1};
+      // failure-path check: a bounded wait on a barrier nothing completes, before any copy
+      if (hold_polls > 0 && !tc::mbar_wait(&bars->hold, 0, abort, hold_polls)) fail(bars, 20);
+      for (uint32_t n = 0; !*abort; ++n) {
         const int s = n & 1;
         if (!tc::mbar_wait(&bars->sched_empty[s], ((n >> 1) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 1); break; }
         const int k = atomicAdd(&control[2], 1);
@@ -251,6 +266,7 @@ __global__ void __launch_bounds__(192, 2)
         const int t = (int)(tile - bh * m.nt);
         if (!tc::mbar_wait(&bars->q_empty, (n & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 2); break; }
         tc::mbar_expect_tx(&bars->q_full, L::kQBytes);
+        q_par = n & 1;
         for (int c = 0; c < D / 64; ++c)
           for (int h = 0; h < 2; ++h)
             tc::tma_load_3d(sQ + c * L::kQChunk + h * L::kKVChunk, &tmQ, &bars->q_full, c * 64,
@@ -272,12 +288,16 @@ __global__ void __launch_bounds__(192, 2)
           const int st = g % NS;
           if (!tc::mbar_wait(&bars->s_full[st], ((g / NS) & 1) ^ 1, abort, kWaitLimit)) { fail(bars, 3); ok = false; break; }
           tc::mbar_expect_tx(&bars->k_full[st], L::kKBytes);
+          k_par[st] = (g / NS) & 1;
           for (int c = 0; c < D / 64; ++c)
             tc::tma_load_3d(sK + st * L::kKBytes + c * L::kKVChunk, &tmK, &bars->k_full[st], c * 64, j * kBlock, (int)bh);
           ++g;
         }
         if (!ok) break;
       }
+      if (q_par >= 0) tc::mbar_wait_drain(&bars->q_full, (uint32_t)q_par, kWaitLimit);
+      for (int st = 0; st < NS; ++st)
+        if (k_par[st] >= 0) tc::mbar_wait_drain(&bars->k_full[st], (uint32_t)k_par[st], kWaitLimit);
     } else if (lane == 1) {
       // ---------------------------------------------------------- V loader
       // Loads V_j for the same steps; a V stage is refilled once the P.V that read it is done.
@@ -299,6 +319,7 @@ __global__ void __launch_bounds__(192, 2)
           tc::mbar_expect_tx(&bars->p_full[st], L::kKBytes);
           for (int c = 0; c < D / 64; ++c)
             tc::tma_load_3d(sV + st * L::kKBytes + c * L::kKVChunk, &tmV, &bars->p_full[st], c * 64, j * kBlock, (int)bh);
+          *reinterpret_cast<volatile int*>(&bars->v_armed) = (int)g;
           ++g;
         }
         if (!ok) break;
@@ -368,8 +389,9 @@ __global__ void __launch_bounds__(192, 2)
         tc::mma_commit(&bars->o_full);
         g += i;
       }
-      // Drain: every MMA issued so far has completed before TMEM can be released.
-      if (ok && n > 0) tc::mbar_wait(&bars->o_full, (n - 1) & 1, abort, kWaitLimit);
+      // Drain, on every path: every MMA issued so far has completed before TMEM is released.
+      tc::mma_commit(&bars->drain);
+      tc::mbar_wait_drain(&bars->drain, 0, kWaitLimit);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -497,7 +519,10 @@ __global__ void __launch_bounds__(192, 2)
         tc::tmem_st_wait();
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&bars->p_full[sb]);
+        if (lane == 0) {
+          tc::mbar_arrive(&bars->p_full[sb]);
+          *reinterpret_cast<volatile int*>(&bars->p_arrived[q]) = (int)gi;
+        }
         ++i;
       }
       if (__any_sync(0xffffffffu, !ok || *abort)) break;
@@ -540,7 +565,22 @@ __global__ void __launch_bounds__(192, 2)
   __syncthreads();
   tc::fence_after_sync();
   if (warp == 1) tc::tmem_dealloc(tbase, L::kTmemCols);
-  if (threadIdx.x == 0 && bars->abort) report_error(control, FVATTN_ERR_TIMEOUT, bars->abort);
+  if (threadIdx.x == 0 && bars->abort) {
+    // Every role has stopped. A V copy completes the P barrier of its step only together with
+    // the four softmax arrivals; after an abort some of them may never have come, so the missing
+    // ones are made here and the copies of the (at most two) V stages in use are waited for.
+    const int va = bars->v_armed;
+    for (int gg = va - 1; gg <= va; ++gg) {
+      if (gg < 0) continue;
+      uint64_t* pb = &bars->p_full[gg & 1];
+      const uint32_t par = ((uint32_t)gg >> 1) & 1;
+      if (tc::mbar_try_wait(pb, par)) continue;
+      for (int w = 0; w < 4; ++w)
+        if (bars->p_arrived[w] < gg) tc::mbar_arrive(pb);
+      tc::mbar_wait_drain(pb, par, kWaitLimit);
+    }
+    report_error(control, FVATTN_ERR_TIMEOUT, bars->abort);
+  }
   if (stamps != nullptr && threadIdx.x == 0) {
     // this CTA's SM and its busy interval (ns), for the SM busy-time imbalance
     uint64_t t_end;
@@ -562,7 +602,7 @@ template <int D>
 cudaError_t launch_tc_d(const void* Q, const void* K, const void* V, const Dims& m, float scale,
                         const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
                         const int32_t* tile_order, int32_t* control, void* O, float* lse, uint64_t* stamps,
-                        int nsm, cudaStream_t st) {
+                        uint32_t hold_polls, int nsm, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, Q, m) || !make_map(&mk, K, m) || !make_map(&mv, V, m)) return cudaErrorInvalidValue;
   const size_t smem = TcLayout<D>::kBytes + 1024;
@@ -571,7 +611,7 @@ cudaError_t launch_tc_d(const void* Q, const void* K, const void* V, const Dims&
   const int grid = attn_tc_grid(m, nsm);
   attn_tc_kernel<D><<<grid, 192, smem, st>>>(mq, mk, mv, m, scale * 1.4426950408889634f, row_ptr, col_idx,
                                              col_code, tile_order, control, static_cast<__nv_bfloat16*>(O), lse,
-                                             stamps);
+                                             stamps, hold_polls);
   return cudaGetLastError();
 }
 
@@ -582,11 +622,12 @@ int attn_tc_grid(const Dims& m, int nsm) { return (int)imin<int64_t>(m.BH * m.nt
 cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const Dims& m, float scale,
                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
                            const int32_t* tile_order, int32_t* control, void* O, float* lse, uint64_t* stamps,
-                           int nsm, cudaStream_t st) {
+                           uint32_t hold_polls, int nsm, cudaStream_t st) {
   if (m.d == 128)
-    return launch_tc_d<128>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O, lse, stamps, nsm,
-                            st);
-  return launch_tc_d<64>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O, lse, stamps, nsm, st);
+    return launch_tc_d<128>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O, lse, stamps,
+                            hold_polls, nsm, st);
+  return launch_tc_d<64>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O, lse, stamps,
+                         hold_polls, nsm, st);
 }
 
 }  // namespace fv

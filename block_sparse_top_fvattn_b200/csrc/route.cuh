@@ -31,7 +31,8 @@ struct SliceOut {
   int32_t* ek;
 };
 cudaError_t launch_score_tc(const int8_t* qs, const int8_t* ks, const int32_t* eq, const int32_t* ek, const Dims& m,
-                            double scale, double* logits, int32_t* status, int nsm, cudaStream_t st);
+                            double scale, double* logits, int32_t* status, int nsm, cudaStream_t st,
+                            uint32_t hold_polls = 0);
 
 // out: 0 = means [row][d] (qo, ko), 1 = score slices and exponents (so), 2 = frame segment sums;
 // the blocks [b0, b1) of every head (outputs at their full-layout rows).
@@ -76,11 +77,12 @@ cudaError_t launch_attn_f32(const float* Q, const float* K, const float* V, cons
                             const int32_t* tile_order, const int32_t* control, float* O, float* lse,
                             cudaStream_t st);
 // stamps: null, or 3 words per CTA of the launch (attn_tc_grid): the SM id and the CTA's busy
-// interval [start, end) in ns of %globaltimer.
+// interval [start, end) in ns of %globaltimer. hold_polls: 0, or (failure-path check) the poll
+// limit of a first wait on a barrier that nothing completes, so that the kernel times out.
 int attn_tc_grid(const Dims& m, int nsm);
 cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const Dims& m, float scale,
                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
                            const int32_t* tile_order, int32_t* control, void* O, float* lse, uint64_t* stamps,
-                           int nsm, cudaStream_t st);
+                           uint32_t hold_polls, int nsm, cudaStream_t st);
 
 }  // namespace fv

@@ -59,6 +59,7 @@ struct ScBars {
   uint64_t k_full[kKTiles], k_empty[kKTiles];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
+  uint64_t hold;            // completed by nothing: the failure-path check waits on it
   uint32_t tmem_base;
   int abort;
 };
@@ -97,7 +98,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const int32_t* __restrict__ eq, const int32_t* __restrict__ ek, Dims m, double scale, int ld,
-                    double* __restrict__ logits, int32_t* __restrict__ status) {
+                    double* __restrict__ logits, int32_t* __restrict__ status, uint32_t hold_polls) {
   using L = ScLayout<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -123,6 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&bars->acc_empty[s], kEpiWarps);
     }
     tc::mbar_init(&bars->drain, 1);
+    tc::mbar_init(&bars->hold, 1);
     bars->abort = 0;
     tc::fence_mbar_init();
   }
@@ -140,8 +142,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------------- loads
       uint32_t qc = 0, kph = 0;
       int s = 0;
+      // parities of the last phases this thread armed (-1: none), waited for before it leaves,
+      // so that no copy is still writing shared memory when the CTA exits
+      int q_par = -1, k_par[kKTiles];
+      for (int x = 0; x < kKTiles; ++x) k_par[x] = -1;
+      // failure-path check: a bounded wait on a barrier nothing completes, before any copy
+      if (hold_polls > 0 && !tc::mbar_wait(&bars->hold, 0, abort, hold_polls)) atomicCAS(&bars->abort, 0, 4);
       TileCursor tcur(t_begin, nrt, nct);
-      for (int64_t t = t_begin; t < t_end; ++t, tcur.next()) {
+      for (int64_t t = t_begin; t < t_end && !*abort; ++t, tcur.next()) {
         const int64_t bh = tcur.bh;
         const int i0 = tcur.rt * kRowsQ, j0 = tcur.ct * kColsK;
         if (t == t_begin || tcur.ct == 0) {
@@ -151,6 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc::mbar_expect_tx(&bars->q_full, kScoreSlices * L::kQSlice);
+          q_par = (int)(qc & 1);
           for (int a = 0; a < kScoreSlices; ++a)
             tc::tma_load_3d(smem + L::kOffQ + a * L::kQSlice, &tmQ, &bars->q_full, 0, i0, (int)(bh * kScoreSlices + a));
           ++qc;
@@ -161,6 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc::mbar_expect_tx(&bars->k_full[s], L::kKTile);
+        k_par[s] = (int)kph;
         for (int b = 0; b < kScoreSlices; ++b)
           tc::tma_load_3d(smem + L::kOffK + s * L::kKTile + b * L::kKSlot, &tmK, &bars->k_full[s], 0, j0,
                           (int)(bh * kScoreSlices + b));
@@ -169,6 +179,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           kph ^= 1;
         }
       }
+      if (q_par >= 0) tc::mbar_wait_drain(&bars->q_full, (uint32_t)q_par, kWaitLimit);
+      for (int x = 0; x < kKTiles; ++x)
+        if (k_par[x] >= 0) tc::mbar_wait_drain(&bars->k_full[x], (uint32_t)k_par[x], kWaitLimit);
     }
   } else if (warp == kEpiWarps + 1) {
     if (lane == 0) {
@@ -223,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) atomicCAS(&bars->abort, 0, 3);
       tc::mma_commit(&bars->drain);
-      tc::mbar_wait(&bars->drain, 0, abort, kWaitLimit);
+      tc::mbar_wait_drain(&bars->drain, 0, kWaitLimit);
     }
   } else {
     // ------------------------------------------------------------------ epilogue (warps 0-15)
@@ -294,7 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D>
 cudaError_t launch_score_tc_d(const int8_t* qs, const int8_t* ks, const int32_t* eq, const int32_t* ek, const Dims& m,
-                              double scale, double* logits, int32_t* status, int nsm, cudaStream_t st) {
+                              double scale, double* logits, int32_t* status, int nsm, cudaStream_t st,
+                              uint32_t hold_polls) {
   CUtensorMap mq, mk;
   const uint64_t planes = (uint64_t)m.BH * kScoreSlices;
   if (!make_map_i8_3d(&mq, qs, (uint64_t)kSliceRow, (uint64_t)m.nb, planes, kRowsQ) ||
@@ -305,16 +319,18 @@ cudaError_t launch_score_tc_d(const int8_t* qs, const int8_t* ks, const int32_t*
   if (e != cudaSuccess) return e;
   const int64_t tiles = m.BH * ((m.nb + kRowsQ - 1) / kRowsQ) * ((m.nb + kColsK - 1) / kColsK);
   const int grid = (int)imin<int64_t>(tiles, nsm);
-  score_tc_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, eq, ek, m, scale, means_ld(m.nb), logits, status);
+  score_tc_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, eq, ek, m, scale, means_ld(m.nb), logits, status,
+                                                   hold_polls);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_score_tc(const int8_t* qs, const int8_t* ks, const int32_t* eq, const int32_t* ek, const Dims& m,
-                            double scale, double* logits, int32_t* status, int nsm, cudaStream_t st) {
-  if (m.d == 128) return launch_score_tc_d<128>(qs, ks, eq, ek, m, scale, logits, status, nsm, st);
-  return launch_score_tc_d<64>(qs, ks, eq, ek, m, scale, logits, status, nsm, st);
+                            double scale, double* logits, int32_t* status, int nsm, cudaStream_t st,
+                            uint32_t hold_polls) {
+  if (m.d == 128) return launch_score_tc_d<128>(qs, ks, eq, ek, m, scale, logits, status, nsm, st, hold_polls);
+  return launch_score_tc_d<64>(qs, ks, eq, ek, m, scale, logits, status, nsm, st, hold_polls);
 }
 
 }  // namespace fv

@@ -263,6 +263,25 @@ int fvattn_block_scores(const void* Q, const void* K, const fvattn_shape* shape,
                         void* workspace, size_t workspace_bytes, int32_t* status,
                         fvattn_stream_t stream);
 
+/*
+ * Failure-path checks of the bounded device waits; the pages have no counterpart. Every wait
+ * of the tensor-core kernels on a barrier is bounded: when one runs out, the kernel stops
+ * issuing work, waits (bounded) for the copies and MMAs it has in flight, frees its tensor
+ * memory, writes FVATTN_ERR_TIMEOUT to the status word and returns, so that the context and
+ * the stream stay usable. These two calls make that path run on purpose: they launch the
+ * kernels of fvattn_sparse_attn (bf16) and of fvattn_block_scores with one extra wait at the
+ * start of every CTA on a barrier that nothing completes, bounded by `polls` (>= 1) polls and
+ * taken before any copy or MMA is issued. The wait runs out, the kernel returns without
+ * writing O (resp. scores), and FVATTN_ERR_TIMEOUT is left in csr->status[0] (resp.
+ * status[0]); read it with fvattn_read_status. Arguments otherwise as for the calls they
+ * mirror. Returns FVATTN_ERR_INVALID for polls == 0.
+ */
+int fvattn_sparse_attn_timeout_check(const void* Q, const void* K, const void* V, const fvattn_shape* shape,
+                                     const fvattn_csr* csr, void* O, uint32_t polls, fvattn_stream_t stream);
+int fvattn_block_scores_timeout_check(const void* Q, const void* K, const fvattn_shape* shape, double* scores,
+                                      void* workspace, size_t workspace_bytes, int32_t* status, uint32_t polls,
+                                      fvattn_stream_t stream);
+
 /* Synchronises `stream`, then returns the device status word status[0] (FVATTN_OK or a
  * negative fvattn_status written by a kernel). FVATTN_ERR_CUDA if the copy fails. */
 int fvattn_read_status(const fvattn_csr* csr, fvattn_stream_t stream);
@@ -315,7 +334,9 @@ int fvattn_select_heads(const fvattn_shape* shape, const fvattn_csr* csr, const 
  * Sizes whose fvattn_route_workspace_bytes exceeds it return FVATTN_ERR_CAPACITY (8 MiB
  * covers, e.g., B*H = 12 heads at S = 8192, d = 128 in Top-p mode). The first call on each
  * device looks up the array's device address (cudaGetSymbolAddress, device current); make
- * that first call before any stream capture. All calls share the one array: calls that
+ * that first call before any stream capture. The cached address assumes the device is not
+ * reset: after cudaDeviceReset the array may be reloaded elsewhere, so a process that resets a
+ * device must not call this entry point on it again. All calls share the one array: calls that
  * overlap on the GPU (other streams, other threads) race and must be serialised by the
  * caller. Q, K, shape, cfg, out and stream are as for fvattn_route.
  */

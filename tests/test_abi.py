@@ -68,6 +68,27 @@ def test_block_scores_sizes_and_host_checks(lib):
     assert st == _lib.FVATTN_ERR_UNSUPPORTED
 
 
+def test_timeout_checks_reject_bad_arguments_on_the_host(lib):
+    s = shape(B=1, H=2, S=1000)
+    buf = ctypes.create_string_buffer(4096)
+    p = ctypes.cast(ctypes.addressof(buf) + (-ctypes.addressof(buf)) % 256, ctypes.c_void_p)
+    csr = _fake_csr(16 * 16 * 2)
+    assert lib.fvattn_sparse_attn_timeout_check(p, p, p, ctypes.byref(s), ctypes.byref(csr), p, 0, None) == \
+        _lib.FVATTN_ERR_INVALID
+    f32 = shape(dtype=1)
+    assert lib.fvattn_sparse_attn_timeout_check(p, p, p, ctypes.byref(f32), ctypes.byref(csr), p, 4, None) == \
+        _lib.FVATTN_ERR_UNSUPPORTED
+    assert lib.fvattn_sparse_attn_timeout_check(p, p, p, ctypes.byref(shape(d=96)), ctypes.byref(csr), p, 4,
+                                                None) == _lib.FVATTN_ERR_UNSUPPORTED
+    ws = lib.fvattn_block_scores_workspace_bytes(ctypes.byref(s))
+    assert lib.fvattn_block_scores_timeout_check(p, p, ctypes.byref(s), p, p, ws, p, 0, None) == \
+        _lib.FVATTN_ERR_INVALID
+    assert lib.fvattn_block_scores_timeout_check(None, p, ctypes.byref(s), p, p, ws, p, 4, None) == \
+        _lib.FVATTN_ERR_INVALID
+    assert lib.fvattn_block_scores_timeout_check(p, p, ctypes.byref(s), p, p, ws - 1, p, 4, None) == \
+        _lib.FVATTN_ERR_CAPACITY
+
+
 def shape(B=1, H=2, S=1000, d=128, block=64, dtype=0, scale=0.0):
     return _lib.Shape(B, H, S, d, block, dtype, scale)
 

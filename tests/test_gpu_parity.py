@@ -76,8 +76,14 @@ def check_route(q, k, cfg: fv.RouteConfig, csr=None, r=None):
     Rows may differ only where the oracle flags a near-tie, and there the GPU's set must be a
     valid selection; the bookkeeping equals the oracle's when no row differs, and satisfies its
     invariants on the GPU's own selection in every case."""
-    B, H, S, d = q.shape
     csr = fv.route(q, k, cfg, csr=csr)
+    return compare_csr(csr, q, k, cfg, r)
+
+
+def compare_csr(csr, q, k, cfg: fv.RouteConfig, r=None):
+    """The checks of check_route on a CSR the GPU router has already written. In token-exact
+    frame mode the per-entry codes must also equal the oracle's."""
+    B, H, S, d = q.shape
     assert fv.read_status(csr) == 0
     gm = gpu_mask(csr)
     oc = to_oracle_cfg(cfg)
@@ -99,6 +105,12 @@ def check_route(q, k, cfg: fv.RouteConfig, csr=None, r=None):
         costs = oracle.tile_costs(om)
         np.testing.assert_array_equal(csr.tile_cost.cpu().numpy(), costs.reshape(-1))
         np.testing.assert_array_equal(csr.tile_order.cpu().numpy(), oracle.lpt_order(costs))
+        if cfg.frame_exact:
+            nb = -(-S // 64)
+            bf = oracle.block_forced(S, oc)
+            want = np.array([oracle.frame_entry_code(r["frame_sets"][row // nb], bf, row % nb, int(ci[e]), S, oc)
+                             for row in range(B * H * nb) for e in range(rp[row], rp[row + 1])], dtype=np.int64)
+            np.testing.assert_array_equal(csr.col_code[: len(ci)].cpu().numpy().astype(np.int64), want)
     check_bookkeeping_properties(csr, gm)
     return csr, gm, r
 
@@ -107,9 +119,16 @@ def check_attention(q, k, v, csr, r, gm, scale, items=None, max_abs=MAX_ABS_BF16
     """The library's attention against the oracle's attention under the oracle's selection
     (r["mask"]). Query blocks whose GPU selection differs from the oracle's (near-tie rows,
     validated by check_route) are left out of the element-wise comparison."""
-    B, H, S, d = q.shape
     o = fv.sparse_attn(q, k, v, csr)
     assert fv.read_status(csr) == 0
+    return compare_attention(o, q, k, v, r, gm, scale, items, max_abs, mean_abs)
+
+
+def compare_attention(o, q, k, v, r, gm, scale, items=None, max_abs=MAX_ABS_BF16, mean_abs=MEAN_ABS_BF16):
+    """The checks of check_attention on an output the GPU has already written: the rows of
+    `items` ((head, query block) pairs) against the oracle's attention under its own selection,
+    leaving out query blocks whose GPU selection differs (validated near-ties)."""
+    B, H, S, d = q.shape
     nb = -(-S // 64)
     ref_mask = r["mask"]
     differs = np.any(gm != ref_mask, axis=2)

@@ -13,6 +13,7 @@ import pytest
 import torch
 
 import block_sparse_top_fvattn_b200 as fv
+from test_gpu_parity import compare_csr
 from workloads import get_workload, make_inputs
 
 oroute = importlib.import_module("oracle.route")
@@ -97,13 +98,22 @@ SPLIT_CASES = [
     ("single", dict(H=2, S=3120, frame_len=1560), fv.RouteConfig(mode="frame_topk", topk_frames=1, frame_len=1560,
                                                                    frame_window=0, force_first_frame=True),
      [(25, 49), (0, 25)]),
+    # range ends inside frames (blocks 10 and 30 start at tokens 640 and 1920, inside frames 0
+    # and 2 of 900 tokens) and a ragged last block (tokens 2944-2999)
+    ("single", dict(H=2, S=3000, frame_len=900, region_len=128),
+     fv.RouteConfig(mode="frame_topk", topk_frames=2, frame_len=900, frame_window=-1), [(30, 47), (0, 10), (10, 30)]),
+    ("single", dict(H=2, S=3000, frame_len=900, region_len=128),
+     fv.RouteConfig(mode="frame_topk", topk_frames=1, frame_len=900, frame_window=0, force_first_frame=True,
+                    frame_exact=True), [(10, 30), (30, 47), (0, 10)]),
+    ("single", dict(H=3, S=2500), fv.RouteConfig(mode="topk", topk_blocks=6), [(0, 13), (13, 40)]),
 ]
 
 
 @pytest.mark.parametrize("name,over,cfg,ranges", SPLIT_CASES)
 def test_split_route_equals_route(name, over, cfg, ranges):
-    """fvattn_route_pool over block ranges in any order, then fvattn_route_finish, gives the CSR
-    of fvattn_route bit for bit (the same kernels on the same blocks)."""
+    """fvattn_route_pool over block ranges in any order, then fvattn_route_finish: the CSR (and in
+    token-exact frame mode the entry codes) against the oracle's router on the same inputs, and
+    bit for bit equal to fvattn_route's (the same kernels on the same blocks)."""
     w = get_workload(name).replace(**over)
     x = make_inputs(w, device="cuda")
     q, k = x["q"], x["k"]
@@ -114,10 +124,13 @@ def test_split_route_equals_route(name, over, cfg, ranges):
     b = fv.route_finish(q, cfg, ws)
     torch.cuda.synchronize()
     assert fv.read_status(a) == 0 and fv.read_status(b) == 0
+    compare_csr(b, q, k, cfg)
     for f in ("row_ptr", "head_load", "tile_cost", "tile_order", "nnz"):
         assert torch.equal(getattr(a, f), getattr(b, f)), f
     n = int(a.nnz.item())
     assert torch.equal(a.col_idx[:n], b.col_idx[:n])
+    if cfg.frame_exact:
+        assert torch.equal(a.col_code[:n], b.col_code[:n])
 
 
 def test_route_pool_rejects_bad_ranges():

@@ -62,6 +62,22 @@ def test_static_scratch_matches_route_on_two_calls_in_a_row():
         _same(got, ref)
 
 
+def test_static_scratch_other_modes_on_a_dirty_array():
+    # Frame top-k and fixed top-k use other parts of the scratch than Top-p (segment sums, frame
+    # means, kept-frame bits); after a Top-p call has left its contents there, each must still
+    # give exactly what fvattn_route gives.
+    q, k = _inputs(14, H=4, S=3000, frame_len=900, region_len=128)
+    cfgs = (fv.RouteConfig(p=0.8),
+            fv.RouteConfig(mode="frame_topk", topk_frames=2, frame_len=900, frame_window=0, force_first_frame=True),
+            fv.RouteConfig(mode="topk", topk_blocks=5, local_window=1),
+            fv.RouteConfig(mode="frame_topk", topk_frames=1, frame_len=900, frame_window=-1))
+    for cfg in cfgs:
+        st, got = _static_route(q, k, cfg)
+        assert st == 0, _lib.status_string(st)
+        assert fv.read_status(got) == 0
+        _same(got, fv.route(q, k, cfg))
+
+
 def test_static_scratch_rejects_sizes_beyond_its_array():
     q, k = _inputs(13, H=40, S=8192)          # needs about 10 MiB of router scratch
     st, _ = _static_route(q, k, fv.RouteConfig(p=0.9))
