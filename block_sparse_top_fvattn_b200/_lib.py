@@ -42,7 +42,12 @@ class Csr(ctypes.Structure):
 
 class FvattnError(RuntimeError):
     def __init__(self, code: int, what: str):
-        super().__init__(f"{what}: {status_string(code)} ({code})")
+        msg = f"{what}: {status_string(code)} ({code})"
+        if code == FVATTN_ERR_CUDA:
+            lib = load()
+            err = lib.fvattn_last_cuda_error()
+            msg += f" [{lib.fvattn_cuda_error_name(err).decode()} ({err})]"
+        super().__init__(msg)
         self.code = code
 
 
@@ -63,6 +68,10 @@ def load() -> ctypes.CDLL:
     lib.fvattn_version.argtypes = []
     lib.fvattn_status_string.restype = ctypes.c_char_p
     lib.fvattn_status_string.argtypes = [ctypes.c_int]
+    lib.fvattn_last_cuda_error.restype = ctypes.c_int
+    lib.fvattn_last_cuda_error.argtypes = []
+    lib.fvattn_cuda_error_name.restype = ctypes.c_char_p
+    lib.fvattn_cuda_error_name.argtypes = [ctypes.c_int]
     lib.fvattn_csr_max_nnz.restype = ctypes.c_int64
     lib.fvattn_csr_max_nnz.argtypes = [P(Shape)]
     lib.fvattn_num_tiles.restype = ctypes.c_int64

@@ -21,7 +21,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfvattn.so")
 
 SOURCES = ["api.cu", "route.cu", "attn_f32.cu", "attn_tc.cu", "route_static.cu", "balance.cu", "score_tc.cu"]
-HEADERS = ["common.cuh", "route.cuh", "tc_ptx.cuh", "tmap.cuh"]
+HEADERS = ["common.cuh", "route.cuh", "route_dev.cuh", "tc_ptx.cuh", "tmap.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -14,6 +14,16 @@ constexpr int kVersion = (1 << 16) | 3;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// The CUDA error behind the last FVATTN_ERR_CUDA this thread got (fvattn_last_cuda_error).
+thread_local int g_last_cuda_error = 0;
+
+// FVATTN_OK, or FVATTN_ERR_CUDA with the CUDA error recorded for this thread.
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return FVATTN_OK;
+  g_last_cuda_error = (int)e;
+  return FVATTN_ERR_CUDA;
+}
+
 int validate_shape(const fvattn_shape* s) {
   if (s == nullptr) return FVATTN_ERR_INVALID;
   if (s->B < 1 || s->H < 1 || s->S < 1 || s->d < 1) return FVATTN_ERR_INVALID;
@@ -113,6 +123,10 @@ double softmax_scale(const fvattn_shape* s) {
 extern "C" {
 
 int fvattn_version(void) { return kVersion; }
+
+int fvattn_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* fvattn_cuda_error_name(int code) { return cudaGetErrorName((cudaError_t)code); }
 
 const char* fvattn_status_string(int status) {
   switch (status) {
@@ -238,7 +252,7 @@ int fvattn_route(const void* Q, const void* K, const fvattn_shape* shape, const 
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   cudaError_t e = route_pool(Q, K, shape, cfg, m, L, ws, 0, m.nb, nsm, s);
   if (e == cudaSuccess) e = route_finish(shape, cfg, out, m, L, ws, nsm, s);
-  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+  return cuda_status(e);
 }
 
 int fvattn_route_pool(const void* Q, const void* K, const fvattn_shape* shape, const fvattn_route_cfg* cfg,
@@ -253,7 +267,7 @@ int fvattn_route_pool(const void* Q, const void* K, const fvattn_shape* shape, c
   if (nsm <= 0) return FVATTN_ERR_CUDA;
   cudaError_t e = route_pool(Q, K, shape, cfg, m, ws_layout(m, cfg->mode), static_cast<unsigned char*>(workspace),
                              (int)block_begin, (int)block_end, nsm, reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+  return cuda_status(e);
 }
 
 int fvattn_route_finish(const fvattn_shape* shape, const fvattn_route_cfg* cfg, const fvattn_csr* out,
@@ -267,7 +281,7 @@ int fvattn_route_finish(const fvattn_shape* shape, const fvattn_route_cfg* cfg, 
   if (nsm <= 0) return FVATTN_ERR_CUDA;
   cudaError_t e = route_finish(shape, cfg, out, m, ws_layout(m, cfg->mode), static_cast<unsigned char*>(workspace),
                                nsm, reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+  return cuda_status(e);
 }
 
 }  // extern "C"
@@ -293,11 +307,11 @@ int sparse_attn(const void* Q, const void* K, const void* V, const fvattn_shape*
   } else {
     const int nsm = num_sms();
     if (nsm <= 0) return FVATTN_ERR_CUDA;
-    if (cudaMemsetAsync(csr->status + 2, 0, sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
+    if (const cudaError_t me = cudaMemsetAsync(csr->status + 2, 0, sizeof(int32_t), s)) return cuda_status(me);
     e = launch_attn_tc(Q, K, V, m, scale, csr->row_ptr, csr->col_idx, csr->col_code, csr->tile_order, csr->status, O,
                        lse, stamps, hold_polls, nsm, s);
   }
-  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+  return cuda_status(e);
 }
 
 }  // namespace
@@ -337,7 +351,7 @@ int fvattn_select_heads(const fvattn_shape* shape, const fvattn_csr* csr, const 
   const Dims m = make_dims(*shape, 0);
   if (m.BH * m.nt > 0x7fffffff) return FVATTN_ERR_UNSUPPORTED;
   cudaError_t e = launch_select_heads(csr->tile_order, m, active, csr->status, reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+  return cuda_status(e);
 }
 
 int fvattn_block_means(const void* X, const fvattn_shape* shape, double* out, fvattn_stream_t stream) {
@@ -349,7 +363,7 @@ int fvattn_block_means(const void* X, const fvattn_shape* shape, double* out, fv
   if (nsm <= 0) return FVATTN_ERR_CUDA;
   cudaError_t e = launch_pool(X, nullptr, 1, shape->dtype, m, 0, m.nb, 0, 0, out, nullptr, nullptr, nullptr, SliceOut{}, nsm,
                               reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+  return cuda_status(e);
 }
 
 size_t fvattn_block_scores_workspace_bytes(const fvattn_shape* shape) {
@@ -378,10 +392,10 @@ int fvattn_block_scores(const void* Q, const void* K, const fvattn_shape* shape,
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   const SliceOut so{reinterpret_cast<int8_t*>(ws + L.qs), reinterpret_cast<int8_t*>(ws + L.ks),
                     reinterpret_cast<int32_t*>(ws + L.eq), reinterpret_cast<int32_t*>(ws + L.ek)};
-  if (cudaMemsetAsync(status, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
+  if (const cudaError_t me = cudaMemsetAsync(status, 0, 4 * sizeof(int32_t), s)) return cuda_status(me);
   cudaError_t e = launch_pool(Q, K, 2, shape->dtype, m, 0, m.nb, 1, 0, nullptr, nullptr, nullptr, nullptr, so, nsm, s);
   if (e == cudaSuccess) e = launch_score_tc(so.qs, so.ks, so.eq, so.ek, m, softmax_scale(shape), scores, status, nsm, s);
-  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+  return cuda_status(e);
 }
 
 int fvattn_sparse_attn_timeout_check(const void* Q, const void* K, const void* V, const fvattn_shape* shape,
@@ -410,19 +424,19 @@ int fvattn_block_scores_timeout_check(const void* Q, const void* K, const fvattn
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   const SliceOut so{reinterpret_cast<int8_t*>(ws + L.qs), reinterpret_cast<int8_t*>(ws + L.ks),
                     reinterpret_cast<int32_t*>(ws + L.eq), reinterpret_cast<int32_t*>(ws + L.ek)};
-  if (cudaMemsetAsync(status, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
+  if (const cudaError_t me = cudaMemsetAsync(status, 0, 4 * sizeof(int32_t), s)) return cuda_status(me);
   cudaError_t e = launch_pool(Q, K, 2, shape->dtype, m, 0, m.nb, 1, 0, nullptr, nullptr, nullptr, nullptr, so, nsm, s);
   if (e == cudaSuccess)
     e = launch_score_tc(so.qs, so.ks, so.eq, so.ek, m, softmax_scale(shape), scores, status, nsm, s, polls);
-  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+  return cuda_status(e);
 }
 
 int fvattn_read_status(const fvattn_csr* csr, fvattn_stream_t stream) {
   if (csr == nullptr || csr->status == nullptr) return FVATTN_ERR_INVALID;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(s) != cudaSuccess) return FVATTN_ERR_CUDA;
+  if (const cudaError_t se = cudaStreamSynchronize(s)) return cuda_status(se);
   int32_t v = 0;
-  if (cudaMemcpy(&v, csr->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return FVATTN_ERR_CUDA;
+  if (const cudaError_t ce = cudaMemcpy(&v, csr->status, sizeof(v), cudaMemcpyDeviceToHost)) return cuda_status(ce);
   return v;
 }
 

@@ -151,6 +151,12 @@ typedef struct {
 /* Library version, (major << 16) | minor. */
 int fvattn_version(void);
 
+/* The cudaError_t code behind the most recent FVATTN_ERR_CUDA returned to the calling thread
+ * (0 if none), and the CUDA runtime's name for a code ("cudaErrorInvalidValue", ...). Host only;
+ * the name works without a GPU. */
+int fvattn_last_cuda_error(void);
+const char* fvattn_cuda_error_name(int code);
+
 /* Static text for a status code. Never NULL. */
 const char* fvattn_status_string(int status);
 
