@@ -8,10 +8,17 @@ fvattn_sparse_attn. The layer is B=1, H=40, S=32760 (21 frames x 1560 tokens), d
 block 64, p=0.9 with the diagonal forced; inputs (1 GB of Q, K, V) are larger than L2.
 
 `value` is the effective TFLOPS of the step: attention FLOPs of the selected blocks only
-(4*d per selected query/key token pair) divided by the step time. With N GPUs every rank runs
-its own layer (weak scaling, no collective on the data path); the time is the max over ranks.
+(4*d per selected query/key token pair) divided by the step time.
 
---impl reference times the CPU oracle (fp64 NumPy) on a bounded sample of the same layer.
+With N > 1 GPUs (torchrun, one rank per GPU) the one layer is split as sequence parallelism holds
+it: every rank has all heads of its S/N-token slice; ulysses_attention exchanges them (NCCL
+all-to-all) for H/N heads over the whole sequence, routes and attends them with runtime head
+migration between ranks (rlb.balanced_attention) and returns the outputs to the sequence layout.
+Strong scaling: the layer is fixed, the time is the max over ranks. --sharded runs this path on
+one GPU too; --replicas gives every rank its own independent layer instead (weak scaling).
+
+--impl reference times the CPU oracle (fp64 NumPy) on a bounded sample of the same layer (the same
+input draw as the GPU arm, copied to the host).
 """
 from __future__ import annotations
 
@@ -31,6 +38,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "block-sparse attn effective TFLOPS & ms per layer at S=32760,H=40,p=0.9; % bf16 peak"
 UNIT = "TFLOPS"
+NOMINAL_BF16_TFLOPS = 2250.0    # B200 datasheet dense bf16 (context: the roofline uses the measured peak)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -59,7 +67,7 @@ def workload_desc(w, mode: str = "topp", topk_frames: int = 4, sasa_coef: float 
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -72,9 +80,13 @@ class ClockSampler:
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200", "-i", str(self.gpu)], stdout=self.f, stderr=subprocess.DEVNULL)
+                                          "-lms", "50", "-i", str(self.gpu)], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+
+    def mark(self, which: str):
+        """Host time of the start / end of the timed region: only samples between the two count."""
+        setattr(self, "t_" + which, time.time())
 
     def stop(self):
         if self.proc is None:
@@ -87,16 +99,23 @@ class ClockSampler:
         self.f.close()
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        import datetime
+        t0, t1 = getattr(self, "t_start", None), getattr(self, "t_end", None)
+        rows = []
         for line in open(self.path):
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+        inside = [r for r in rows if t0 is not None and t1 is not None and t0 <= r[0] <= t1]
+        for _, c, m, rs in (inside or rows):          # a region shorter than the interval: every sample
+            sm.append(c)
+            mx.append(m)
+            for n, v in zip(names, rs):
                 if v.lower() == "active":
                     reasons.add(n)
         os.unlink(self.path)
@@ -190,65 +209,98 @@ def reduce_over_ranks(ms: float, flops: float, device):
 
 # ------------------------------------------------------------------ CPU oracle baseline
 
-def cpu_oracle_run(w, q_cpu, k_cpu, v_cpu, n_items: int, seed: int = 0, heads_sample=None):
-    """Time the oracle (as it stands) on a bounded sample of the layer: the full router on
-    `heads` heads and exact attention for `n_items` query blocks of those heads. Returns
-    (estimated seconds for the whole layer, sample description, threads used, sample FLOPs)."""
-    import numpy as np
-    import oracle
+def oracle_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
-        threads = os.cpu_count() or 1
+        return os.cpu_count() or 1
+
+
+def oracle_layer(w, q_cpu, k_cpu):
+    """The oracle's routing of the whole layer (its masks and selected FLOPs), the scale of every
+    sample below. Not timed by the reference arm; timed in full by the GPU arm's cpu_baseline."""
+    import oracle
     BH = w.B * w.H
-    heads = BH if heads_sample is None else min(BH, heads_sample)
-    Q = q_cpu.reshape(BH, w.S, w.d)[:heads]
-    K = k_cpu.reshape(BH, w.S, w.d)[:heads]
-    V = v_cpu.reshape(BH, w.S, w.d)[:heads]
-    cfg = oracle.RouteCfg(p=w.p, force_diag=True)
+    Q = q_cpu.reshape(BH, w.S, w.d)
+    K = k_cpu.reshape(BH, w.S, w.d)
     t0 = time.perf_counter()
-    r = oracle.route(Q, K, cfg)
+    r = oracle.route(Q, K, oracle.RouteCfg(p=w.p, force_diag=True))
     t_route = time.perf_counter() - t0
+    return r, oracle.selected_flops(r["mask"], w.S, 64, w.d), t_route
+
+
+def oracle_sample(w, q_cpu, k_cpu, v_cpu, r, layer_flops, n_items: int, route_heads: int, seed: int,
+                  t_route_all=None):
+    """Time the oracle (as it stands) on a bounded sample of the layer and scale it to the layer:
+    the router on `route_heads` heads (time x heads of the layer; or the measured whole-layer
+    router time t_route_all) plus exact attention of `n_items` seeded query blocks (time x the
+    layer's selected FLOPs / the sample's). Returns (estimated layer seconds, description)."""
+    import numpy as np
+    import oracle
+    BH = w.B * w.H
+    Q = q_cpu.reshape(BH, w.S, w.d)
+    K = k_cpu.reshape(BH, w.S, w.d)
+    V = v_cpu.reshape(BH, w.S, w.d)
     rng = np.random.default_rng(seed)
-    items = [(int(b), int(i)) for b, i in zip(rng.integers(0, heads, n_items), rng.integers(0, w.nb, n_items))]
+    if t_route_all is None:
+        heads = rng.choice(BH, size=route_heads, replace=False)
+        t0 = time.perf_counter()
+        oracle.route(Q[heads], K[heads], oracle.RouteCfg(p=w.p, force_diag=True))
+        t_route = (time.perf_counter() - t0) * BH / route_heads
+        rdesc = f"router on {route_heads}/{BH} heads scaled by heads"
+    else:
+        t_route = t_route_all
+        rdesc = f"router on all {BH} heads"
+    # query blocks drawn in proportion to their selected FLOPs, so that the sample's time per FLOP
+    # is that of the layer
+    nrow = np.array([min(w.S, (i + 1) * 64) - i * 64 for i in range(w.nb)])
+    wts = (r["mask"] * nrow[None, None, :]).sum(axis=2) * nrow[None, :]
+    flat = rng.choice(wts.size, size=n_items, replace=False, p=(wts / wts.sum()).reshape(-1))
+    items = [(int(f // w.nb), int(f % w.nb)) for f in flat]
     t0 = time.perf_counter()
     oracle.attention_rows(Q, K, V, r["mask"], 1.0 / math.sqrt(w.d), items)
     t_attn = time.perf_counter() - t0
-    # scale: router time per head x BH; attention time per sampled block x all blocks of the layer,
-    # weighted by the selected-FLOP share of the sample
-    flops_heads = oracle.selected_flops(r["mask"], w.S, 64, w.d)
-    nrow = np.array([min(w.S, (i + 1) * 64) - i * 64 for i in range(w.nb)])
     f_items = sum(4 * w.d * int(nrow[i]) * int(nrow[r["mask"][b, i]].sum()) for b, i in items)
-    est_layer_flops = flops_heads * BH / heads
-    t_layer = t_route * BH / heads + t_attn * (est_layer_flops / max(f_items, 1))
-    desc = (f"oracle router on {heads}/{BH} heads ({t_route:.1f} s) + exact attention of {n_items} sampled query "
-            f"blocks ({t_attn:.1f} s), scaled to the whole layer by heads and by selected-FLOP share")
-    return t_layer, desc, threads, est_layer_flops
+    t_layer = t_route + t_attn * (layer_flops / max(f_items, 1))
+    desc = (f"fp64 NumPy oracle: {rdesc} ({t_route:.1f} s for the layer) + exact attention of {n_items} query "
+            f"blocks drawn by selected-FLOP weight ({t_attn:.2f} s), scaled by the layer's selected FLOPs")
+    return t_layer, desc
+
+
+def layer_inputs_host(w):
+    """The layer's Q, K, V as the GPU arm draws them (on the GPU when there is one), on the host."""
+    import torch
+    from workloads import make_inputs
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = make_inputs(w, device=dev)
+    return x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), dev
 
 
 def run_reference(args, w):
     rank, world, _ = env_rank()
     if rank != 0:
         return 0
-    import torch
-    from workloads import make_inputs
-    x = make_inputs(w.replace(H=4), device="cpu")      # the sample's heads (same per-head generator)
-    times = []
-    flops = None
-    desc = threads = None
+    q, k, v, drawn_on = layer_inputs_host(w)
+    r, layer_flops, _ = oracle_layer(w, q, k)
+    threads = oracle_threads()
+    times, wall = [], []
+    desc = None
     for s in range(args.warmup + args.steps):
-        t_layer, desc, threads, flops = cpu_oracle_run(w.replace(H=4), x["q"], x["k"], x["v"], n_items=24, seed=s)
-        t_layer *= w.H / 4
+        t0 = time.perf_counter()
+        t_layer, desc = oracle_sample(w, q, k, v, r, layer_flops, n_items=4, route_heads=1, seed=s)
         if s >= args.warmup:
             times.append(t_layer)
-    flops = flops * w.H / 4
+            wall.append(time.perf_counter() - t0)
     t = statistics.median(times)
-    value = flops / t / 1e12
+    value = layer_flops / t / 1e12
+    desc += f"; inputs drawn on the {drawn_on} as the GPU arm's; median over {args.steps} samples"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": workload_desc(w), "l2": "n/a (CPU)"},
+            # ms_per_step is the layer time the sample extrapolates to; the samples themselves took:
+            "measured_sample_ms_per_step": statistics.mean(wall) * 1e3,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -317,6 +369,162 @@ def emulate_ranks(fv, q, k, v, cfg, csr, out, stream, R: int, target: float, bud
     }
 
 
+def run_sharded(args, w):
+    """The layer split over the ranks (see the module docstring): Ulysses sequence parallelism
+    with runtime head migration. Strong scaling; the time of a step is the slowest rank's."""
+    import datetime
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_top_fvattn_b200 as fv
+    from block_sparse_top_fvattn_b200 import rlb, ulysses
+    from workloads import make_inputs
+
+    rank, world, local = env_rank()
+    if "MASTER_ADDR" in os.environ:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:                                        # one process without torchrun (--sharded)
+        dist.init_process_group("nccl", init_method=f"file://{tempfile.mktemp(prefix='fvattn_pg_')}", rank=0,
+                                world_size=1, timeout=datetime.timedelta(seconds=120))
+    R = dist.get_world_size()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    fv.load()
+    pk, pk_src = peaks()
+    B, H, S, d = w.B, w.H, w.S, w.d
+    if B != 1 or H % R or S % R:
+        raise SystemExit(f"the sharded layer needs B = 1 and H, S divisible by {R} ranks")
+    x = make_inputs(w, device=dev)              # the one layer, drawn identically on every rank
+    Sl = S // R
+    ql, kl, vl = (x[n][:, :, rank * Sl:(rank + 1) * Sl].contiguous() for n in ("q", "k", "v"))
+    cfg = fv.RouteConfig(p=w.p, force_diag=True)
+    kernels = rlb.Kernels(cfg)
+    # the layer's selected FLOPs (the routing does not depend on how the layer is split)
+    csr_full = fv.route(x["q"], x["k"], cfg)
+    flops, nnz, _, _ = selected_flops_from_csr(csr_full, S, d)
+    density = nnz / (B * H * csr_full.nb * csr_full.nb)
+    # this rank's heads over the whole sequence, for the attention kernel's own roofline figure
+    Hl = H // R
+    qh, kh, vh = (x[n][:, rank * Hl:(rank + 1) * Hl].contiguous() for n in ("q", "k", "v"))
+    del x, csr_full
+    torch.cuda.empty_cache()
+
+    def step(balance):
+        return ulysses.ulysses_attention(ql, kl, vl, cfg, balance=balance, target=args.rlb_target,
+                                         max_moves_per_rank=args.rlb_budget, kernels=kernels, overlap_pool=True)
+
+    def timed(n, balance):
+        dist.barrier()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        plan = None
+        for _ in range(n):
+            _, plan = step(balance)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / n
+        per_rank = [torch.zeros(1, dtype=torch.float64, device=dev) for _ in range(R)]
+        dist.all_gather(per_rank, torch.tensor([ms], dtype=torch.float64, device=dev))
+        dist.barrier()
+        return [float(t.item()) for t in per_rank], plan
+
+    for _ in range(max(args.warmup, 3)):
+        step(True)
+    torch.cuda.synchronize()
+    n_cmp = min(args.steps, 20)
+    unbalanced, _ = timed(n_cmp, False)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    sampler.mark("start")
+    balanced, plan = timed(args.steps, True)
+    sampler.mark("end")
+    clocks = sampler.stop()
+    ms_step = max(balanced)
+    value = flops / (ms_step * 1e-3) / 1e12
+
+    # end to end: this rank's slice of Q, K, V from pinned host memory in, its slice of O out
+    hq, hk, hv = (t.cpu().pin_memory() for t in (ql, kl, vl))
+    ho = torch.empty(ql.shape, dtype=ql.dtype, pin_memory=True)
+    n_e2e = max(3, min(6, args.steps))
+    dist.barrier()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(n_e2e):
+        ql.copy_(hq, non_blocking=True)
+        kl.copy_(hk, non_blocking=True)
+        vl.copy_(hv, non_blocking=True)
+        o, _ = step(True)
+        ho.copy_(o, non_blocking=True)
+    b.record()
+    torch.cuda.synchronize()
+    e_ms = torch.tensor([a.elapsed_time(b) / n_e2e], dtype=torch.float64, device=dev)
+    dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+    e_ms = float(e_ms.item())
+
+    # the attention kernel alone on this rank's own heads (outside the timed region)
+    csr_l = fv.route(qh, kh, cfg)
+    out_l = torch.empty_like(qh)
+    f_local, _, _, _ = selected_flops_from_csr(csr_l, S, d)
+    ts = []
+    for i in range(8):
+        ea = torch.cuda.Event(enable_timing=True)
+        eb = torch.cuda.Event(enable_timing=True)
+        ea.record()
+        fv.sparse_attn(qh, kh, vh, csr_l, out=out_l)
+        eb.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ts.append(ea.elapsed_time(eb))
+    attn_local_tflops = f_local / (statistics.median(ts) * 1e-3) / 1e12
+    if fv.read_status(csr_l) != 0:
+        raise RuntimeError("device status after the attention of the local heads")
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    esize = ql.element_size()
+    loads = plan.loads if plan is not None else None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": R, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "parallelism": f"sequence parallel x{R} (Ulysses all-to-all over "
+                   f"NCCL) + runtime head migration", "l2": "inputs larger than L2"},
+        "density": density, "selected_flops_per_layer": flops,
+        "rlb": {"heads_per_rank": Hl, "rank_head_loads": loads.tolist() if loads is not None else None,
+                "moves": len(plan.moves) if plan is not None else 0,
+                "load_imbalance_before": plan.imbalance_before if plan is not None else None,
+                "load_imbalance_after": plan.imbalance_after if plan is not None else None,
+                "rank_ms_unbalanced": unbalanced, "rank_ms_balanced": balanced,
+                "time_imbalance_unbalanced": max(unbalanced) / (sum(unbalanced) / R),
+                "time_imbalance_balanced": max(balanced) / (sum(balanced) / R),
+                "migrated_bytes_per_step": (len(plan.moves) if plan is not None else 0) * 4 * S * d * esize},
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (rank 0's heads, timed alone)",
+                     "achieved": attn_local_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": attn_local_tflops / pk["bf16_tflops"], "traffic": None,
+                     "peak_kind": f"bf16 burst ({pk_src})"},
+        "e2e": {"value": flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+                "h2d_bytes_per_step": 3 * ql.numel() * esize * R, "d2h_bytes_per_step": ql.numel() * esize * R,
+                "pipeline": "per rank: its slice in, the layer, its slice out (no overlap)"},
+        "cpu_baseline": None,
+        # rank 0's launches of this library's kernels in the timed region: the router (pooling per
+        # arriving slice + 4 kernels, or 5), the attention, and with head migration fvattn_select_heads
+        # on a sender and the router + attention of the received heads on a receiver
+        "gpu_launches": args.steps * (((R + 4) if Sl % 64 == 0 else 5) + 1 +
+                                      (1 if plan is not None and any(m[0] == 0 for m in plan.moves) else 0) +
+                                      (6 if plan is not None and any(m[2] == 0 for m in plan.moves) else 0)),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ours(args, w):
     import numpy as np
     import torch
@@ -326,6 +534,8 @@ def run_ours(args, w):
     from workloads import make_inputs
 
     rank, world, local = env_rank()
+    if args.sharded or (world > 1 and not args.replicas):
+        return run_sharded(args, w)
     if world > 1:
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     torch.cuda.set_device(local)
@@ -382,6 +592,7 @@ def run_ours(args, w):
     time.sleep(0.3)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    sampler.mark("start")
     t_start.record(stream)
     routed_steps = 0
     for s in range(args.steps):
@@ -394,6 +605,7 @@ def run_ours(args, w):
         ev[s][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
+    sampler.mark("end")
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
@@ -494,8 +706,12 @@ def run_ours(args, w):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t_layer, desc, threads, _ = cpu_oracle_run(w, q.cpu(), k.cpu(), v.cpu(), n_items=160)
-        cpu = {"value": flops / t_layer / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+        qh, kh, vh = q.cpu(), k.cpu(), v.cpu()
+        r, layer_flops_oracle, t_route_all = oracle_layer(w, qh, kh)
+        t_layer, desc = oracle_sample(w, qh, kh, vh, r, layer_flops_oracle, n_items=48, route_heads=BH, seed=0,
+                                      t_route_all=t_route_all)
+        cpu = {"value": layer_flops_oracle / t_layer / 1e12, "unit": UNIT, "cores": oracle_threads(),
+               "kind": "oracle", "sample": desc + "; the GPU arm's input draw"}
 
     if world > 1:
         dist.barrier()
@@ -509,6 +725,11 @@ def run_ours(args, w):
         clocks.get("sm_mhz") and clocks.get("sm_max_mhz") and clocks["sm_mhz"] < 0.95 * clocks["sm_max_mhz"])
     bf16_peak = pk["bf16_tflops_sustained"] if capped else pk["bf16_tflops"]
     peak_kind = ("bf16 sustained, power-capped clocks" if capped else "bf16 burst, maximum clocks") + f" ({pk_src})"
+    # The attention time scaled to the maximum SM clock by the median clock sampled under load
+    # (the kernel is compute bound, so its time scales with the clock): the burst fraction
+    # that does not depend on where the clock sat during the timed region.
+    clock_ratio = (clocks["sm_mhz"] / clocks["sm_max_mhz"]) if clocks.get("sm_mhz") and clocks.get("sm_max_mhz") else None
+    attn_at_max = attn_avg * clock_ratio if clock_ratio else None
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -536,7 +757,11 @@ def run_ours(args, w):
                      # the union of their key blocks), for context; `achieved` counts selected
                      # pairs only
                      "executed_tflops": mma_flops / (attn_avg * 1e-3) / 1e12,
-                     "frac_executed": mma_flops / (attn_avg * 1e-3) / 1e12 / bf16_peak},
+                     "frac_executed": mma_flops / (attn_avg * 1e-3) / 1e12 / bf16_peak,
+                     "frac_of_datasheet": attn_tflops / NOMINAL_BF16_TFLOPS,
+                     "attn_ms_at_max_clock": attn_at_max,
+                     "frac_of_burst_at_max_clock": (flops / (attn_at_max * 1e-3) / 1e12 / pk["bf16_tflops"])
+                     if attn_at_max else None},
         "roofline_router": {"bound": "hbm", "achieved": router_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                             "frac": router_gbs / pk["hbm_gbs"], "algorithmic_bytes": rbytes,
                             "peak_kind": f"hbm copy ({pk_src})"},
@@ -552,8 +777,8 @@ def run_ours(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="dit")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -574,6 +799,10 @@ def main():
                     help="emulate runtime load balancing over this many ranks on one GPU (0: off)")
     ap.add_argument("--rlb-target", type=float, default=1.05)
     ap.add_argument("--rlb-budget", type=int, default=1, help="heads a rank may send")
+    ap.add_argument("--sharded", action="store_true",
+                    help="the sequence-parallel layer with head migration also on one process")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with N > 1: an independent layer per rank (weak scaling) instead of the sharded layer")
     args = ap.parse_args()
     if args.refresh_every < 1:
         ap.error("--refresh-every must be >= 1")
