@@ -167,7 +167,7 @@ size_t select_smem_bytes_t(const Dims& m) {
 // warps 2w and 2w+1 hold the two rows of a 128-row tile and write its cost, then (register
 // path, sasa.coef > 0) augment each other's slack.
 template <int NE>
-__global__ void __launch_bounds__(SEL_WARPS * 32) select_kernel(const double* __restrict__ logits, Dims m, double p,
+__global__ void __launch_bounds__(SEL_WARPS * 32, NE == 16 ? 8 : 1) select_kernel(const double* __restrict__ logits, Dims m, double p,
                                                      int kblocks, ForceCfg fc, SasaCfg sasa,
                                                      uint32_t* __restrict__ bits, int32_t* __restrict__ counts,
                                                      int32_t* __restrict__ tile_cost) {
