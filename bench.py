@@ -382,14 +382,14 @@ def run_sharded(args, w):
     from workloads import make_inputs
 
     rank, world, local = env_rank()
+    torch.cuda.set_device(local)                 # before the process group: NCCL binds this device
+    dev = torch.device("cuda", local)
     if "MASTER_ADDR" in os.environ:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     else:                                        # one process without torchrun (--sharded)
         dist.init_process_group("nccl", init_method=f"file://{tempfile.mktemp(prefix='fvattn_pg_')}", rank=0,
-                                world_size=1, timeout=datetime.timedelta(seconds=120))
+                                world_size=1, timeout=datetime.timedelta(seconds=120), device_id=dev)
     R = dist.get_world_size()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
     fv.load()
     pk, pk_src = peaks()
     B, H, S, d = w.B, w.H, w.S, w.d
@@ -536,10 +536,10 @@ def run_ours(args, w):
     rank, world, local = env_rank()
     if args.sharded or (world > 1 and not args.replicas):
         return run_sharded(args, w)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
-    torch.cuda.set_device(local)
+    torch.cuda.set_device(local)                 # before the process group: NCCL binds this device
     dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120), device_id=dev)
     fv.load()
     pk, pk_src = peaks()
 
