@@ -10,12 +10,15 @@ block 64, p=0.9 with the diagonal forced; inputs (1 GB of Q, K, V) are larger th
 `value` is the effective TFLOPS of the step: attention FLOPs of the selected blocks only
 (4*d per selected query/key token pair) divided by the step time.
 
-With N > 1 GPUs (torchrun, one rank per GPU) the one layer is split as sequence parallelism holds
-it: every rank has all heads of its S/N-token slice; ulysses_attention exchanges them (NCCL
-all-to-all) for H/N heads over the whole sequence, routes and attends them with runtime head
-migration between ranks (rlb.balanced_attention) and returns the outputs to the sequence layout.
-Strong scaling: the layer is fixed, the time is the max over ranks. --sharded runs this path on
-one GPU too; --replicas gives every rank its own independent layer instead (weak scaling).
+With N > 1 GPUs (torchrun, one rank per GPU) the one layer is split over the ranks by head: each
+rank holds H/N heads over the whole sequence (the layout sequence parallelism reaches after its
+all-to-all), routes them, and runtime head migration between ranks (rlb.balanced_attention:
+all-gather of per-head loads, the plan, point-to-point moves of Q, K, V and O) evens out the
+ranks' loads before and during the attention. --ulysses starts instead from sequence-sharded
+inputs (every rank has all heads of its S/N-token slice) and adds the sequence-to-head and
+head-to-sequence all-to-alls (ulysses_attention). Strong scaling: the layer is fixed, the time is
+the max over ranks. --sharded runs this path on one GPU too; --replicas gives every rank its own
+independent layer instead (weak scaling).
 
 --impl reference times the CPU oracle (fp64 NumPy) on a bounded sample of the same layer (the same
 input draw as the GPU arm, copied to the host).
@@ -410,9 +413,20 @@ def run_sharded(args, w):
     del x, csr_full
     torch.cuda.empty_cache()
 
-    def step(balance):
-        return ulysses.ulysses_attention(ql, kl, vl, cfg, balance=balance, target=args.rlb_target,
-                                         max_moves_per_rank=args.rlb_budget, kernels=kernels, overlap_pool=True)
+    if args.ulysses:
+        def step(balance):
+            return ulysses.ulysses_attention(ql, kl, vl, cfg, balance=balance, target=args.rlb_target,
+                                             max_moves_per_rank=args.rlb_budget, kernels=kernels, overlap_pool=True)
+    else:
+        ql, kl, vl = qh, kh, vh                  # this rank's heads over the whole sequence
+        out_h = torch.empty_like(qh)
+
+        def step(balance):
+            if balance:
+                return rlb.balanced_attention(ql, kl, vl, cfg, target=args.rlb_target,
+                                              max_moves_per_rank=args.rlb_budget, kernels=kernels)
+            kernels.attend(ql, kl, vl, kernels.route(ql, kl), None, out_h)
+            return out_h, None
 
     def timed(n, balance):
         dist.barrier()
@@ -494,8 +508,10 @@ def run_sharded(args, w):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": R, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": workload_desc(w), "parallelism": f"sequence parallel x{R} (Ulysses all-to-all over "
-                   f"NCCL) + runtime head migration", "l2": "inputs larger than L2"},
+        "config": {"workload": workload_desc(w),
+                   "parallelism": (f"sequence parallel x{R} (Ulysses all-to-all over NCCL) + runtime head migration"
+                                   if args.ulysses else f"heads split over {R} ranks + runtime head migration (NCCL)"),
+                   "l2": "inputs larger than L2"},
         "density": density, "selected_flops_per_layer": flops,
         "rlb": {"heads_per_rank": Hl, "rank_head_loads": loads.tolist() if loads is not None else None,
                 "moves": len(plan.moves) if plan is not None else 0,
@@ -511,12 +527,12 @@ def run_sharded(args, w):
                      "peak_kind": f"bf16 burst ({pk_src})"},
         "e2e": {"value": flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
                 "h2d_bytes_per_step": 3 * ql.numel() * esize * R, "d2h_bytes_per_step": ql.numel() * esize * R,
-                "pipeline": "per rank: its slice in, the layer, its slice out (no overlap)"},
+                "pipeline": "per rank: its part of Q, K, V in, the layer, its part of O out (no overlap)"},
         "cpu_baseline": None,
         # rank 0's launches of this library's kernels in the timed region: the router (pooling per
         # arriving slice + 4 kernels, or 5), the attention, and with head migration fvattn_select_heads
         # on a sender and the router + attention of the received heads on a receiver
-        "gpu_launches": args.steps * (((R + 4) if Sl % 64 == 0 else 5) + 1 +
+        "gpu_launches": args.steps * (((R + 4) if (args.ulysses and Sl % 64 == 0) else 5) + 1 +
                                       (1 if plan is not None and any(m[0] == 0 for m in plan.moves) else 0) +
                                       (6 if plan is not None and any(m[2] == 0 for m in plan.moves) else 0)),
         "clocks": clocks,
@@ -801,6 +817,8 @@ def main():
     ap.add_argument("--rlb-budget", type=int, default=1, help="heads a rank may send")
     ap.add_argument("--sharded", action="store_true",
                     help="the sequence-parallel layer with head migration also on one process")
+    ap.add_argument("--ulysses", action="store_true",
+                    help="the sharded layer from sequence-sharded inputs, with the Ulysses all-to-alls")
     ap.add_argument("--replicas", action="store_true",
                     help="with N > 1: an independent layer per rank (weak scaling) instead of the sharded layer")
     args = ap.parse_args()
