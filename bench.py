@@ -259,6 +259,7 @@ def oracle_sample(w, q_cpu, k_cpu, v_cpu, r, layer_flops, n_items: int, route_he
     # is that of the layer
     nrow = np.array([min(w.S, (i + 1) * 64) - i * 64 for i in range(w.nb)])
     wts = (r["mask"] * nrow[None, None, :]).sum(axis=2) * nrow[None, :]
+    n_items = min(n_items, int((wts > 0).sum()))
     flat = rng.choice(wts.size, size=n_items, replace=False, p=(wts / wts.sum()).reshape(-1))
     items = [(int(f // w.nb), int(f % w.nb)) for f in flat]
     t0 = time.perf_counter()

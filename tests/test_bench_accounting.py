@@ -62,3 +62,21 @@ def test_router_bytes():
     nt = BH * 256
     want = 2 * BH * S * d * 2 + 4 * (BH * nb + 1) + 4 * nnz + 8 * BH + 8 * nt + 8
     assert bench.router_bytes(BH, S, d, 2, nb, nnz) == want
+
+
+def test_oracle_baseline_sample_scaling():
+    # The oracle baselines scale a timed sample to the layer: the router time by heads and the
+    # attention time by selected FLOPs. With every head routed and every query block sampled the
+    # scale is 1, so the estimate is the sample's own time; a small layer with fewer query blocks
+    # than asked for samples all of them.
+    from workloads import get_workload, make_inputs
+    w = get_workload("tiny")
+    x = make_inputs(w)
+    r, layer_flops, t_route = bench.oracle_layer(w, x["q"], x["k"])
+    BH = w.B * w.H
+    assert layer_flops == oracle.selected_flops(r["mask"], w.S, 64, w.d) > 0
+    t_layer, desc = bench.oracle_sample(w, x["q"], x["k"], x["v"], r, layer_flops, n_items=10 ** 6,
+                                        route_heads=BH, seed=0, t_route_all=t_route)
+    assert t_layer > t_route and f"{BH * w.nb} query blocks" in desc
+    t1, d1 = bench.oracle_sample(w, x["q"], x["k"], x["v"], r, layer_flops, n_items=4, route_heads=1, seed=1)
+    assert t1 > 0 and "router on 1/2 heads" in d1
