@@ -220,6 +220,52 @@ __global__ void __launch_bounds__(SEL_WARPS * 32, NE == 16 ? 8 : 1) select_kerne
   }
 }
 
+// Rows of at most 32 NE blocks: one warp per 128-row tile (query blocks 2t and 2t+1 of one
+// head): the cut of both rows in registers, forced blocks, bitmask rows and counts, the tile's
+// cost, then (sasa.coef > 0) each row augmented from the other's slack. A warp needs no other
+// warp's rows, so the CTA has no barrier and a tile's rows never wait for a slower row of
+// another tile.
+template <int NE>
+__global__ void __launch_bounds__(SEL_WARPS * 32, NE == 16 ? 8 : 1)
+    select_tile_kernel(const double* __restrict__ logits, Dims m, double p, int kblocks, ForceCfg fc, SasaCfg sasa,
+                       uint32_t* __restrict__ bits, int32_t* __restrict__ counts, int32_t* __restrict__ tile_cost) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* sw = reinterpret_cast<uint32_t*>(smem_raw) + (size_t)warp * 4 * m.nw;   // rows 2t, 2t+1, wc, wo
+  const int64_t bh = blockIdx.y;
+  const int t = blockIdx.x * SEL_WARPS + warp;
+  if (t >= m.nt) return;
+  const int ld = means_ld(m.nb);
+  uint32_t* w[2] = {sw, sw + m.nw};
+  for (int rr = 0; rr < 2; ++rr) {
+    const int i = 2 * t + rr;
+    if (i >= m.nb) {
+      for (int q = lane; q < m.nw; q += 32) w[rr][q] = 0u;
+      __syncwarp();
+      continue;
+    }
+    const double* src = logits + (bh * m.nb + i) * (int64_t)ld;
+    if (kblocks > 0) topk_select_reg<NE>(src, m.nb, kblocks, w[rr], lane);
+    else topp_select_reg<NE>(src, m.nb, p, w[rr], lane);
+    const int64_t grow = bh * m.nb + i;
+    finalize_row(w[rr], i, m, fc, lane, bits + grow * m.nw, counts + grow);
+  }
+  int c = 0;
+  for (int q = lane; q < m.nw; q += 32) c += __popc(w[0][q] | w[1][q]);
+  c = warp_sum(c);
+  if (lane == 0) tile_cost[bh * m.nt + t] = c;
+  if (sasa.coef > 0.f && 2 * t + 1 < m.nb) {
+    uint32_t* wc = sw + 2 * m.nw;
+    uint32_t* wo = sw + 3 * m.nw;
+    for (int rr = 0; rr < 2; ++rr) {
+      const int64_t grow = bh * m.nb + 2 * t + rr;
+      sasa_row<NE>(logits + grow * (int64_t)ld, m, sasa, w[rr], w[rr ^ 1], wc, wo, lane, bits + grow * m.nw,
+                   counts + grow);
+      __syncwarp();
+    }
+  }
+}
+
 template <int NE>
 static cudaError_t launch_select_t(const double* logits, const Dims& m, double p, int kblocks, const ForceCfg& fc,
                                    const SasaCfg& sasa, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
@@ -229,6 +275,19 @@ static cudaError_t launch_select_t(const double* logits, const Dims& m, double p
   if (e != cudaSuccess) return e;
   dim3 g((m.nb + SEL_WARPS - 1) / SEL_WARPS, (unsigned)m.BH);
   select_kernel<NE><<<g, SEL_WARPS * 32, smem, st>>>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost);
+  return cudaGetLastError();
+}
+
+template <int NE>
+static cudaError_t launch_select_tile_t(const double* logits, const Dims& m, double p, int kblocks, const ForceCfg& fc,
+                                        const SasaCfg& sasa, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
+                                        cudaStream_t st) {
+  const size_t smem = (size_t)SEL_WARPS * 4 * m.nw * 4;
+  cudaError_t e =
+      cudaFuncSetAttribute(select_tile_kernel<NE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 g((m.nt + SEL_WARPS - 1) / SEL_WARPS, (unsigned)m.BH);
+  select_tile_kernel<NE><<<g, SEL_WARPS * 32, smem, st>>>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost);
   return cudaGetLastError();
 }
 
@@ -608,8 +667,8 @@ cudaError_t launch_topp(const SliceOut& so, double* logits, const Dims& m, doubl
                         int32_t* status, int nsm, cudaStream_t st) {
   cudaError_t e = launch_score_tc(so.qs, so.ks, so.eq, so.ek, m, scale, logits, status, nsm, st);
   if (e != cudaSuccess) return e;
-  if (m.nb <= 32 * 16) return launch_select_t<16>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost, st);
-  if (m.nb <= 32 * 40) return launch_select_t<40>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost, st);
+  if (m.nb <= 32 * 16) return launch_select_tile_t<16>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost, st);
+  if (m.nb <= 32 * 40) return launch_select_tile_t<40>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost, st);
   return launch_select_t<0>(logits, m, p, 0, fc, SasaCfg{0.f, 0}, bits, counts, tile_cost, st);
 }
 
