@@ -156,21 +156,18 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ Q, cons
 
 size_t logits_elems(const Dims& m) { return (size_t)m.BH * m.nb * means_ld(m.nb); }
 
-template <int NE>
-size_t select_smem_bytes_t(const Dims& m) {
-  return NE > 0 ? (size_t)3 * SEL_WARPS * m.nw * 4
-                : (size_t)SEL_WARPS * m.nw * 32 * 8 + (size_t)SEL_WARPS * m.nw * 4;
+size_t select_smem_bytes(const Dims& m) {
+  return (size_t)SEL_WARPS * m.nw * 4 + 16 + (size_t)SEL_WARPS * m.nw * 32 * 8;
 }
 
-// One warp per query block: the Top-p cut of its fp64 logit row (in registers when the row
-// has at most 32 NE blocks, else through shared memory), forced blocks, bitmask row and count;
-// warps 2w and 2w+1 hold the two rows of a 128-row tile and write its cost, then (register
-// path, sasa.coef > 0) augment each other's slack.
-template <int NE>
-__global__ void __launch_bounds__(SEL_WARPS * 32, NE == 16 ? 8 : 1) select_kernel(const double* __restrict__ logits, Dims m, double p,
-                                                     int kblocks, ForceCfg fc, SasaCfg sasa,
-                                                     uint32_t* __restrict__ bits, int32_t* __restrict__ counts,
-                                                     int32_t* __restrict__ tile_cost) {
+// Rows of more than 40 * 32 blocks: one warp per query block, the row's logits staged in shared
+// memory for the Top-p cut; forced blocks, bitmask row and count; warps 2w and 2w+1 hold the two
+// rows of a 128-row tile and write its cost (no top-k and no slack augmentation at this size:
+// the host rejects both).
+__global__ void __launch_bounds__(SEL_WARPS * 32) select_smem_kernel(const double* __restrict__ logits, Dims m,
+                                                                   double p, ForceCfg fc, uint32_t* __restrict__ bits,
+                                                                   int32_t* __restrict__ counts,
+                                                                   int32_t* __restrict__ tile_cost) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int nbp = m.nw * 32;
   uint32_t* sW = reinterpret_cast<uint32_t*>(smem_raw);                          // [warp][nw]
@@ -182,15 +179,10 @@ __global__ void __launch_bounds__(SEL_WARPS * 32, NE == 16 ? 8 : 1) select_kerne
   uint32_t* w = sW + warp * m.nw;
   if (i < m.nb) {
     const double* src = logits + (bh * m.nb + i) * (int64_t)ld;
-    if (NE > 0) {
-      if (kblocks > 0) topk_select_reg<(NE > 0 ? NE : 1)>(src, m.nb, kblocks, w, lane);
-      else topp_select_reg<(NE > 0 ? NE : 1)>(src, m.nb, p, w, lane);
-    } else {
-      double* E = sE + (size_t)warp * nbp;
-      for (int j = lane; j < m.nb; j += 32) E[j] = src[j];
-      __syncwarp();
-      topp_select(E, m.nb, p, w, lane);
-    }
+    double* E = sE + (size_t)warp * nbp;
+    for (int j = lane; j < m.nb; j += 32) E[j] = src[j];
+    __syncwarp();
+    topp_select(E, m.nb, p, w, lane);
     const int64_t grow = bh * m.nb + i;
     finalize_row(w, i, m, fc, lane, bits + grow * m.nw, counts + grow);
   } else {
@@ -206,16 +198,6 @@ __global__ void __launch_bounds__(SEL_WARPS * 32, NE == 16 ? 8 : 1) select_kerne
       for (int q = lane; q < m.nw; q += 32) c += __popc(wa[q] | wb[q]);
       c = warp_sum(c);
       if (lane == 0) tile_cost[bh * m.nt + t] = c;
-    }
-  }
-  if constexpr (NE > 0) {
-    if (sasa.coef > 0.f && i < m.nb && (i ^ 1) < m.nb) {
-      // the rows of this CTA's tiles are final in sW; augmentation writes only wc/wo and global
-      uint32_t* wc = sW + (size_t)SEL_WARPS * m.nw + (size_t)warp * m.nw;
-      uint32_t* wo = sW + (size_t)2 * SEL_WARPS * m.nw + (size_t)warp * m.nw;
-      const int64_t grow = bh * m.nb + i;
-      sasa_row<NE>(logits + grow * (int64_t)ld, m, sasa, w, sW + (warp ^ 1) * m.nw, wc, wo, lane,
-                   bits + grow * m.nw, counts + grow);
     }
   }
 }
@@ -266,15 +248,13 @@ __global__ void __launch_bounds__(SEL_WARPS * 32, NE == 16 ? 8 : 1)
   }
 }
 
-template <int NE>
-static cudaError_t launch_select_t(const double* logits, const Dims& m, double p, int kblocks, const ForceCfg& fc,
-                                   const SasaCfg& sasa, uint32_t* bits, int32_t* counts, int32_t* tile_cost,
-                                   cudaStream_t st) {
-  const size_t smem = select_smem_bytes_t<NE>(m) + 16;
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<NE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+static cudaError_t launch_select_smem(const double* logits, const Dims& m, double p, const ForceCfg& fc,
+                                      uint32_t* bits, int32_t* counts, int32_t* tile_cost, cudaStream_t st) {
+  const size_t smem = select_smem_bytes(m);
+  cudaError_t e = cudaFuncSetAttribute(select_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 g((m.nb + SEL_WARPS - 1) / SEL_WARPS, (unsigned)m.BH);
-  select_kernel<NE><<<g, SEL_WARPS * 32, smem, st>>>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost);
+  select_smem_kernel<<<g, SEL_WARPS * 32, smem, st>>>(logits, m, p, fc, bits, counts, tile_cost);
   return cudaGetLastError();
 }
 
@@ -669,7 +649,7 @@ cudaError_t launch_topp(const SliceOut& so, double* logits, const Dims& m, doubl
   if (e != cudaSuccess) return e;
   if (m.nb <= 32 * 16) return launch_select_tile_t<16>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost, st);
   if (m.nb <= 32 * 40) return launch_select_tile_t<40>(logits, m, p, kblocks, fc, sasa, bits, counts, tile_cost, st);
-  return launch_select_t<0>(logits, m, p, 0, fc, SasaCfg{0.f, 0}, bits, counts, tile_cost, st);
+  return launch_select_smem(logits, m, p, fc, bits, counts, tile_cost, st);
 }
 
 cudaError_t launch_frame(const double* qlo, const double* qhi, const double* klo, const double* khi,
