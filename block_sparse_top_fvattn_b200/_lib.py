@@ -6,6 +6,11 @@ import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfvattn.so")
+# The checked build (-DFVATTN_DEBUG): the same entry points; its kernels check every CSR list
+# before reading it and report a failed check as FVATTN_ERR_INVALID (status[1] = 101: row
+# offsets, 102: a key block out of range, 103: a list not ascending).
+DEBUG_LIB_PATH = os.path.join(_HERE, "libfvattn_debug.so")
+DEBUG_OFFSETS, DEBUG_COLUMN, DEBUG_ORDER = 101, 102, 103
 
 FVATTN_OK = 0
 FVATTN_ERR_INVALID = -1
@@ -52,6 +57,14 @@ class FvattnError(RuntimeError):
 
 
 _lib = None
+
+
+def use_debug_build() -> None:
+    """Make this process load the checked build. Must come before the first load()."""
+    global LIB_PATH
+    if _lib is not None and LIB_PATH != DEBUG_LIB_PATH:
+        raise RuntimeError("the library is already loaded; select the checked build before the first call")
+    LIB_PATH = DEBUG_LIB_PATH
 
 
 def load() -> ctypes.CDLL:

@@ -302,14 +302,14 @@ int sparse_attn(const void* Q, const void* K, const void* V, const fvattn_shape*
   cudaError_t e;
   if (shape->dtype == FVATTN_F32) {
     e = launch_attn_f32(static_cast<const float*>(Q), static_cast<const float*>(K), static_cast<const float*>(V), m,
-                        scale, csr->row_ptr, csr->col_idx, csr->col_code, csr->tile_order, csr->status,
-                        static_cast<float*>(O), lse, s);
+                        scale, csr->row_ptr, csr->col_idx, csr->col_capacity, csr->col_code, csr->tile_order,
+                        csr->status, static_cast<float*>(O), lse, s);
   } else {
     const int nsm = num_sms();
     if (nsm <= 0) return FVATTN_ERR_CUDA;
     if (const cudaError_t me = cudaMemsetAsync(csr->status + 2, 0, sizeof(int32_t), s)) return cuda_status(me);
-    e = launch_attn_tc(Q, K, V, m, scale, csr->row_ptr, csr->col_idx, csr->col_code, csr->tile_order, csr->status, O,
-                       lse, stamps, hold_polls, nsm, s);
+    e = launch_attn_tc(Q, K, V, m, scale, csr->row_ptr, csr->col_idx, csr->col_capacity, csr->col_code,
+                       csr->tile_order, csr->status, O, lse, stamps, hold_polls, nsm, s);
   }
   return cuda_status(e);
 }

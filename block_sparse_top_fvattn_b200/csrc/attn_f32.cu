@@ -18,10 +18,10 @@ template <int D>
 __global__ void __launch_bounds__(256) attn_f32_kernel(const float* __restrict__ Q, const float* __restrict__ K,
                                                        const float* __restrict__ V, Dims m, float scale,
                                                        const int32_t* __restrict__ row_ptr,
-                                                       const int32_t* __restrict__ col_idx,
+                                                       const int32_t* __restrict__ col_idx, int64_t col_cap,
                                                        const int32_t* __restrict__ col_code,
                                                        const int32_t* __restrict__ tile_order,
-                                                       const int32_t* __restrict__ control,
+                                                       int32_t* __restrict__ control,
                                                        float* __restrict__ O, float* __restrict__ lse) {
   constexpr int DQ = D / 4;
   constexpr int KCH = D == 128 ? 32 : 64;     // keys staged per step (shared memory <= 48 KB)
@@ -49,6 +49,12 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float* __restrict__
   }
   float mx = -INFINITY, l = 0.f;
   const int64_t row = bh * m.nb + i;
+#ifdef FVATTN_DEBUG
+  if (const int bad = debug_row_check(row_ptr, col_idx, col_cap, row, m.nb)) {   // uniform over the CTA
+    if (tid == 0) report_error(control, FVATTN_ERR_INVALID, bad);
+    return;
+  }
+#endif
   const int e0 = row_ptr[row], e1 = row_ptr[row + 1];
   for (int e = e0; e < e1; ++e) {
     const int j = col_idx[e];
@@ -96,18 +102,17 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float* __restrict__
 }
 
 cudaError_t launch_attn_f32(const float* Q, const float* K, const float* V, const Dims& m, float scale,
-                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
-                            const int32_t* tile_order, const int32_t* control, float* O, float* lse,
-                            cudaStream_t st) {
+                            const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap, const int32_t* col_code,
+                            const int32_t* tile_order, int32_t* control, float* O, float* lse, cudaStream_t st) {
   const int64_t ntiles = m.BH * m.nt;
   if (ntiles > 0x7fffffff) return cudaErrorInvalidValue;
   dim3 grid((unsigned)ntiles, 2);
   if (m.d == 128)
-    attn_f32_kernel<128><<<grid, 256, 0, st>>>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O,
-                                               lse);
+    attn_f32_kernel<128><<<grid, 256, 0, st>>>(Q, K, V, m, scale, row_ptr, col_idx, col_cap, col_code, tile_order,
+                                               control, O, lse);
   else
-    attn_f32_kernel<64><<<grid, 256, 0, st>>>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O,
-                                              lse);
+    attn_f32_kernel<64><<<grid, 256, 0, st>>>(Q, K, V, m, scale, row_ptr, col_idx, col_cap, col_code, tile_order,
+                                              control, O, lse);
   return cudaGetLastError();
 }
 

@@ -174,7 +174,7 @@ template <int D>
 __global__ void __launch_bounds__(192, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, Dims m, float scale_log2,
-                   const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                   const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx, int64_t col_cap,
                    const int32_t* __restrict__ col_code, const int32_t* __restrict__ tile_order,
                    int32_t* __restrict__ control, __nv_bfloat16* __restrict__ O, float* __restrict__ lse,
                    uint64_t* __restrict__ stamps, uint32_t hold_polls) {
@@ -258,6 +258,16 @@ __global__ void __launch_bounds__(192, 2)
         if (k < count) {
           tile = tile_order[k];
           if (tile < 0 || tile >= ntiles) { fail(bars, 11); tile = -1; }
+#ifdef FVATTN_DEBUG
+          // debug build: both block lists of the tile are checked before any role reads them
+          if (tile >= 0) {
+            const int64_t tb = tile / m.nt;
+            const int tt = (int)(tile - tb * m.nt);
+            int bad = debug_row_check(row_ptr, col_idx, col_cap, tb * m.nb + 2 * tt, m.nb);
+            if (!bad && 2 * tt + 1 < m.nb) bad = debug_row_check(row_ptr, col_idx, col_cap, tb * m.nb + 2 * tt + 1, m.nb);
+            if (bad) { fail(bars, bad); tile = -1; }
+          }
+#endif
         }
         bars->sched_tile[s] = tile;
         tc::mbar_arrive(&bars->sched_full[s]);
@@ -579,7 +589,10 @@ __global__ void __launch_bounds__(192, 2)
         if (bars->p_arrived[w] < gg) tc::mbar_arrive(pb);
       tc::mbar_wait_drain(pb, par, kWaitLimit);
     }
-    report_error(control, FVATTN_ERR_TIMEOUT, bars->abort);
+    // a tile index out of range (11) or a failed list check of the debug build (>= 100) is a
+    // bad argument; every other code is a wait that ran out
+    const int ab = bars->abort;
+    report_error(control, (ab == 11 || ab >= 100) ? FVATTN_ERR_INVALID : FVATTN_ERR_TIMEOUT, ab);
   }
   if (stamps != nullptr && threadIdx.x == 0) {
     // this CTA's SM and its busy interval (ns), for the SM busy-time imbalance
@@ -600,7 +613,7 @@ bool make_map(CUtensorMap* map, const void* base, const Dims& m) {
 
 template <int D>
 cudaError_t launch_tc_d(const void* Q, const void* K, const void* V, const Dims& m, float scale,
-                        const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
+                        const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap, const int32_t* col_code,
                         const int32_t* tile_order, int32_t* control, void* O, float* lse, uint64_t* stamps,
                         uint32_t hold_polls, int nsm, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
@@ -610,8 +623,8 @@ cudaError_t launch_tc_d(const void* Q, const void* K, const void* V, const Dims&
   if (e != cudaSuccess) return e;
   const int grid = attn_tc_grid(m, nsm);
   attn_tc_kernel<D><<<grid, 192, smem, st>>>(mq, mk, mv, m, scale * 1.4426950408889634f, row_ptr, col_idx,
-                                             col_code, tile_order, control, static_cast<__nv_bfloat16*>(O), lse,
-                                             stamps, hold_polls);
+                                             col_cap, col_code, tile_order, control,
+                                             static_cast<__nv_bfloat16*>(O), lse, stamps, hold_polls);
   return cudaGetLastError();
 }
 
@@ -620,13 +633,13 @@ cudaError_t launch_tc_d(const void* Q, const void* K, const void* V, const Dims&
 int attn_tc_grid(const Dims& m, int nsm) { return (int)imin<int64_t>(m.BH * m.nt, (int64_t)nsm * 2); }
 
 cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const Dims& m, float scale,
-                           const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
+                           const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap, const int32_t* col_code,
                            const int32_t* tile_order, int32_t* control, void* O, float* lse, uint64_t* stamps,
                            uint32_t hold_polls, int nsm, cudaStream_t st) {
   if (m.d == 128)
-    return launch_tc_d<128>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O, lse, stamps,
-                            hold_polls, nsm, st);
-  return launch_tc_d<64>(Q, K, V, m, scale, row_ptr, col_idx, col_code, tile_order, control, O, lse, stamps,
+    return launch_tc_d<128>(Q, K, V, m, scale, row_ptr, col_idx, col_cap, col_code, tile_order, control, O, lse,
+                            stamps, hold_polls, nsm, st);
+  return launch_tc_d<64>(Q, K, V, m, scale, row_ptr, col_idx, col_cap, col_code, tile_order, control, O, lse, stamps,
                          hold_polls, nsm, st);
 }
 

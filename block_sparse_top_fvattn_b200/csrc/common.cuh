@@ -45,6 +45,28 @@ __device__ __forceinline__ void report_error(int32_t* status, int code, int deta
   if (atomicCAS(status, 0, code) == 0) status[1] = detail;
 }
 
+#ifdef FVATTN_DEBUG
+// Debug build (-DFVATTN_DEBUG) only: checks the CSR list of one row before a kernel reads it.
+// Returns 0, or the failed check: kDbgOffsets (row offsets decreasing, negative or beyond the
+// column array's capacity), kDbgColumn (a key block outside [0, nb)), kDbgOrder (the list not
+// strictly ascending). Kernels report it as FVATTN_ERR_INVALID with the check in status[1]
+// and skip the row; nothing outside the arrays is read.
+constexpr int kDbgOffsets = 101, kDbgColumn = 102, kDbgOrder = 103;
+__device__ inline int debug_row_check(const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap, int64_t row,
+                                      int nb) {
+  const int64_t a = row_ptr[row], b = row_ptr[row + 1];
+  if (a < 0 || b < a || b > col_cap) return kDbgOffsets;
+  int prev = -1;
+  for (int64_t e = a; e < b; ++e) {
+    const int j = col_idx[e];
+    if (j < 0 || j >= nb) return kDbgColumn;
+    if (j <= prev) return kDbgOrder;
+    prev = j;
+  }
+  return 0;
+}
+#endif
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(m));

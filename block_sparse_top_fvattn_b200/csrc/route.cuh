@@ -72,16 +72,16 @@ cudaError_t launch_select_heads(int32_t* tile_order, const Dims& m, const uint8_
 
 // Attention (attn_f32.cu, attn_tc.cu).
 // col_code may be null (every entry allows its whole key block).
+// col_cap: the capacity of col_idx (read only by the debug build's list checks).
 cudaError_t launch_attn_f32(const float* Q, const float* K, const float* V, const Dims& m, float scale,
-                            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
-                            const int32_t* tile_order, const int32_t* control, float* O, float* lse,
-                            cudaStream_t st);
+                            const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap, const int32_t* col_code,
+                            const int32_t* tile_order, int32_t* control, float* O, float* lse, cudaStream_t st);
 // stamps: null, or 3 words per CTA of the launch (attn_tc_grid): the SM id and the CTA's busy
 // interval [start, end) in ns of %globaltimer. hold_polls: 0, or (failure-path check) the poll
 // limit of a first wait on a barrier that nothing completes, so that the kernel times out.
 int attn_tc_grid(const Dims& m, int nsm);
 cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const Dims& m, float scale,
-                           const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_code,
+                           const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap, const int32_t* col_code,
                            const int32_t* tile_order, int32_t* control, void* O, float* lse, uint64_t* stamps,
                            uint32_t hold_polls, int nsm, cudaStream_t st);
 

@@ -222,6 +222,12 @@ int fvattn_route_finish(const fvattn_shape* shape, const fvattn_route_cfg* cfg,
  * dtype as Q. lse: optional device float [B,H,S] receiving the natural-log softmax
  * normaliser of each row (NULL to skip). bf16 runs on the tensor cores (tcgen05, fp32
  * accumulation); f32 runs on the CUDA cores in fp32.
+ * The CSR is trusted: this library reads the lists the router wrote. Its checked build
+ * (libfvattn_debug.so, the same sources compiled with -DFVATTN_DEBUG) checks every row's list
+ * before reading it and, on a failure, skips the row's tile and writes FVATTN_ERR_INVALID to
+ * status[0] and the check to status[1]: 101 row offsets decreasing or beyond col_capacity,
+ * 102 a key block outside [0, nb), 103 a list not strictly ascending. A tile index outside the
+ * grid in tile_order is reported as FVATTN_ERR_INVALID (status[1] = 11) by both builds.
  */
 int fvattn_sparse_attn(const void* Q, const void* K, const void* V, const fvattn_shape* shape,
                        const fvattn_csr* csr, void* O, float* lse, fvattn_stream_t stream);

@@ -44,6 +44,15 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, n), n
 
 
+def test_checked_build_exports_every_declared_symbol():
+    # libfvattn_debug.so (-DFVATTN_DEBUG) is a drop-in for the same boundary
+    import ctypes
+    assert os.path.exists(_lib.DEBUG_LIB_PATH), "build it with `python -m block_sparse_top_fvattn_b200.build --debug`"
+    dbg = ctypes.CDLL(_lib.DEBUG_LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(dbg, n), n
+
+
 def test_version_and_status_strings(lib):
     assert lib.fvattn_version() >> 16 == 1
     for code in range(0, -6, -1):
