@@ -41,10 +41,11 @@ CHILD = textwrap.dedent(r"""
     if dtype == "bf16":
         w, q, k, v = small_inputs("single", H=3, S=2500)
         tol = {{}}
+        cfg = fv.RouteConfig(p=0.9)
     else:
         w, q, k, v = small_inputs("tiny")
         tol = dict(max_abs=MAX_ABS_F32, mean_abs=MAX_ABS_F32)
-    cfg = fv.RouteConfig(p=0.9)
+        cfg = fv.RouteConfig(p=0.9, local_window=1)           # rows of at least two blocks
     scale = 1.0 / np.sqrt(w.d)
     csr, gm, r = check_route(q, k, cfg)
     check_attention(q, k, v, csr, r, gm, scale, **tol)        # the checked build against the oracle
