@@ -297,6 +297,17 @@ __device__ __forceinline__ double lane_sum(const float (&e)[NE], const uint32_t 
   return (double)t[0];
 }
 
+// lane_sum(e, k, lo_key, false) and, in `cnt`, the number of the lane's keys >= lo_key.
+template <int NE>
+__device__ __forceinline__ double lane_sum_count(const float (&e)[NE], const uint32_t (&k)[NE], uint32_t lo_key,
+                                                 int& cnt) {
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < NE; ++i) c += k[i] >= lo_key;
+  cnt = c;
+  return lane_sum(e, k, lo_key, false);
+}
+
 // The Top-p cut of one row with its weights in registers (NE per lane, element j = lane + 32 i),
 // the same rule as topp_select: weights e_j = 2^((s_j - max) log2 e) from the SFU on fp64
 // logit differences, masses compared with p * sum(e). Both ways below find the cut key T (the
@@ -304,8 +315,10 @@ __device__ __forceinline__ double lane_sum(const float (&e)[NE], const uint32_t 
 // ascending index, as many keys == T as the mass needs. Peaked rows peel key values from the
 // top (REDUX max over the lanes' largest remaining keys, all copies of a value at once) until
 // the mass reaches p; rows with more than kExtract weights above 1/64, or not done after
-// kExtract values, take a bisection over the 32-bit key space. Lane sums are pairwise in fp32
-// and folded across the warp in fp64 in a fixed order (deterministic).
+// kExtract values, take a bisection over the 32-bit key space, which stops as soon as a single
+// key is left in its bracket (the cut is always one of the row's keys, so that key is the one
+// the full bisection would reach). Lane sums are pairwise in fp32 and folded across the warp in
+// fp64 in a fixed order (deterministic).
 template <int NE>
 __device__ void topp_select_reg(const double* __restrict__ src, int n, double p, uint32_t* w, int lane) {
   const int nw = (n + 31) / 32;
@@ -381,15 +394,37 @@ __device__ void topp_select_reg(const double* __restrict__ src, int n, double p,
     }
   }
   if (!done) {
-    // Bisection: largest T with mass{key >= T} >= P. Weights are at most 1, so keys <= 0x3f800000.
-    uint32_t lo = 0, hi = 0x3f800001u;
-    while (hi - lo > 1) {
+    // Bisection: largest T with mass{key >= T} >= P. Weights are at most 1, so keys <= 0x3f800000;
+    // the bracket starts at the smallest key of the row (its mass is the whole row's). cl / ch
+    // count the keys >= lo / >= hi (elements past n have key 0); [lo, hi) always holds a key.
+    uint32_t kmin = 0xffffffffu;
+#pragma unroll
+    for (int i = 0; i < NE; ++i)
+      if (lane + 32 * i < n) kmin = min(kmin, k[i]);
+    uint32_t lo = __reduce_min_sync(0xffffffffu, kmin), hi = 0x3f800001u;
+    int cl = lo > 0u ? n : 32 * NE, ch = 0;
+    while (hi - lo > 1 && cl - ch > 1) {
       const uint32_t mid = lo + ((hi - lo) >> 1);
-      const double sm = warp_sum_d(lane_sum(e, k, mid, false));
-      if (sm >= P) lo = mid;
-      else hi = mid;
+      int c;
+      const double sm = warp_sum_d(lane_sum_count(e, k, mid, c));
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (sm >= P) {
+        lo = mid;
+        cl = c;
+      } else {
+        hi = mid;
+        ch = c;
+      }
     }
-    T = lo;
+    if (cl - ch == 1) {
+      // one key in [lo, hi): mass{key >= it} = mass{key >= lo} >= P, every larger key is >= hi
+      uint32_t km = 0u;
+#pragma unroll
+      for (int i = 0; i < NE; ++i) km = max(km, k[i] < hi ? k[i] : 0u);
+      T = __reduce_max_sync(0xffffffffu, km);
+    } else {
+      T = lo;
+    }
     above = warp_sum_d(lane_sum(e, k, T, true));
   }
   const double tval = (double)__uint_as_float(T);
