@@ -639,6 +639,33 @@ def run_ours(args, w):
     router_gbs = rbytes / (route_avg * 1e-3) / 1e9
     traffic = traffic_from_profile(os.path.join(ROOT, "block_sparse_top_fvattn_b200", "csrc", "attn_tc.cu"))
 
+    # The same step captured once in a CUDA graph (route + attention, static buffers) and replayed
+    # K times: what a caller that replays graphs sees, without per-call launch work on the host.
+    graph = None
+    if not args.no_graph and args.refresh_every == 1 and plain is None and world == 1:
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step()
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            g0.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            g1.record(stream)
+            torch.cuda.synchronize()
+            if fv.read_status(csr) != 0:
+                raise RuntimeError(f"device status {fv.read_status(csr)}")
+            gms = g0.elapsed_time(g1)
+            graph = {"ms_per_step": gms / args.steps, "value": flops * args.steps / (gms * 1e-3) / 1e12,
+                     "unit": UNIT, "steps": args.steps,
+                     "note": "route + attention captured once in a CUDA graph, replayed; timed after the main region"}
+            del g
+        except Exception as exc:                   # reported, not fatal: the headline is the plain launches
+            graph = {"error": f"{type(exc).__name__}: {exc}"}
+
     # SM busy-time imbalance of the persistent attention grid (outside the timed region): one
     # stamped launch on the router's longest-first order, one on ascending tile ids.
     sm_busy = None
@@ -783,6 +810,7 @@ def run_ours(args, w):
                             "frac": router_gbs / pk["hbm_gbs"], "algorithmic_bytes": rbytes,
                             "peak_kind": f"hbm copy ({pk_src})"},
         "e2e": e2e, "cpu_baseline": cpu,
+        **({"graph_replay": graph} if graph is not None else {}),
         **({"rlb_emulated": rlb_em} if rlb_em is not None else {}),
         "gpu_launches": 5 * routed_steps + args.steps,   # router: 5 kernels, attention: 1
         "clocks": clocks,
@@ -801,6 +829,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sm-busy", action="store_true", help="skip the stamped launches of the SM busy-time imbalance")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing of the step")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling case)")
     ap.add_argument("--p", type=float, default=0.0, help="override the Top-p threshold")
     ap.add_argument("--mode", default="topp", choices=["topp", "frame_topk"])
