@@ -206,11 +206,13 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) select_smem_kernel(const doubl
 // head): the cut of both rows in registers, forced blocks, bitmask rows and counts, the tile's
 // cost, then (sasa.coef > 0) each row augmented from the other's slack. A warp needs no other
 // warp's rows, so the CTA has no barrier and a tile's rows never wait for a slower row of
-// another tile. The kernel is bound by the latency of each warp's rows, so rows of up to 512
-// blocks run at 10 CTAs per SM (48 registers and a 40-byte spill: 20 % faster than 8 CTAs at
-// 64 registers; 12 CTAs at 40 registers spill ten times as much and lose).
+// another tile. The kernel is bound by the latency of each warp's rows, so it runs with more
+// CTAs per SM than its registers alone would allow: rows of up to 512 blocks at 10 (48
+// registers and a 40-byte spill: 20 % faster than 8 CTAs at 64 registers; 12 CTAs at 40
+// registers spill ten times as much and lose), rows of up to 1280 blocks at 5 (96 registers and
+// an 80-byte spill: a third faster than 2 CTAs at 181 registers).
 template <int NE>
-__global__ void __launch_bounds__(SEL_WARPS * 32, NE == 16 ? 10 : 1)
+__global__ void __launch_bounds__(SEL_WARPS * 32, NE == 16 ? 10 : 5)
     select_tile_kernel(const double* __restrict__ logits, Dims m, double p, int kblocks, ForceCfg fc, SasaCfg sasa,
                        uint32_t* __restrict__ bits, int32_t* __restrict__ counts, int32_t* __restrict__ tile_cost) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -588,19 +590,20 @@ __global__ void __launch_bounds__(256) csr_kernel(const uint32_t* __restrict__ b
   for (int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < N; row += nwarps) {
     if ((int64_t)row_ptr[row + 1] > capacity) continue;     // reported by the schedule kernel
     const uint32_t* w = bits + row * m.nw;
-    int64_t base = row_ptr[row];
+    int64_t pos = row_ptr[row];
+    // Lane l holds word q0 + l; the non-zero words are then expanded one at a time by the whole
+    // warp, lane b writing block 32q + b when its bit is set, so that each word's entries go
+    // out as one coalesced store in ascending order.
     for (int q0 = 0; q0 < m.nw; q0 += 32) {
-      const int q = q0 + lane;
-      uint32_t x = q < m.nw ? w[q] : 0u;
-      const int c = __popc(x);
-      const int incl = warp_incl_scan(c, lane);
-      int64_t pos = base + incl - c;
-      while (x) {
-        const int b = __ffs(x) - 1;
-        x &= x - 1;
-        col_idx[pos++] = q * 32 + b;
+      const uint32_t xl = q0 + lane < m.nw ? w[q0 + lane] : 0u;
+      uint32_t nz = __ballot_sync(0xffffffffu, xl != 0u);
+      while (nz) {
+        const int k = __ffs(nz) - 1;
+        nz &= nz - 1;
+        const uint32_t x = __shfl_sync(0xffffffffu, xl, k);
+        if ((x >> lane) & 1u) col_idx[pos + __popc(x & lanemask_lt())] = (q0 + k) * 32 + lane;
+        pos += __popc(x);
       }
-      base += __shfl_sync(0xffffffffu, incl, 31);
     }
   }
 }
