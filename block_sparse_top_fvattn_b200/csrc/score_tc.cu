@@ -13,15 +13,19 @@
 // products the tensor cores compute exactly, in the manner of the Ozaki scheme for accurate
 // matrix products).
 //
-// Work: the 128 x 32 output tiles of all heads in (head, row tile, column tile) order, split into
+// Work: the 128 x 64 output tiles of all heads in (head, row tile, column tile) order, split into
 // one contiguous range per CTA (one persistent CTA per SM), so a CTA loads the five Q slices of a
 // row tile once (80 KB, resident in shared memory; rows of 128 bytes, one 128-byte swizzle
 // span) and only reloads them when its range enters the next row tile. The five K slices of a
 // column tile stream through a ring of three tiles (one barrier per tile); one thread issues
-// tcgen05.mma (kind::i8, K = 32 per instruction) into one of two accumulator sets (5 levels x 32
-// columns at 32-column TMEM offsets); sixteen epilogue warps drain the other set meanwhile (four
-// per TMEM lane quarter, 8 columns each), combine the levels in fp64 and write each thread's 8
-// consecutive logits of its row (64 bytes) straight to global memory.
+// tcgen05.mma (kind::i8, M = 128, N = 64, K = 32 per instruction) into one accumulator set of
+// 5 levels x 64 columns; sixteen epilogue warps (four per TMEM lane quarter, 16 columns each)
+// load the set, release it to the next tile's MMAs, combine the levels in fp64 and write each
+// thread's 16 consecutive logits of its row (128 bytes) straight to global memory. An MMA of
+// N = 64 costs the issuing thread about what one of N = 32 does, so the wider tile halves the
+// instructions per logit; two sets of 5 x 64 columns would not fit the 512 TMEM columns, so the
+// set is single and the next tile's MMAs wait only for the epilogue's TMEM loads (59.8 against
+// 67.8 us per launch at dit for two sets of N = 32).
 #include <cuda.h>
 #include <math.h>
 
@@ -34,12 +38,13 @@ namespace fv {
 
 namespace {
 
-constexpr int kRowsQ = 128, kColsK = 32;
+constexpr int kRowsQ = 128, kColsK = 64;
 constexpr int kKTiles = 3;                              // K ring: three column tiles of five slices
 constexpr int kEpiWarps = 16;
 constexpr int kEpiCols = kColsK / (kEpiWarps / 4);      // columns of a tile per epilogue thread
 constexpr int kThreads = (kEpiWarps + 2) * 32;          // + producer warp + MMA warp
-constexpr int kLevelCols = kScoreSlices * kColsK;       // one accumulator set: 160 TMEM columns
+constexpr int kLevelCols = kScoreSlices * kColsK;       // one accumulator set: 320 TMEM columns
+constexpr int kSets = 2 * kLevelCols <= 512 ? 2 : 1;     // accumulator sets that fit in TMEM
 constexpr uint32_t kWaitLimit = 1u << 22;
 
 template <int D>
@@ -200,14 +205,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       TileCursor tcur(t_begin, nrt, nct);
       for (int64_t t = t_begin; ok && t < t_end; ++t, tcur.next()) {
-        const uint32_t j = (uint32_t)(t - t_begin), buf = j & 1;
+        const uint32_t j = (uint32_t)(t - t_begin), buf = j % kSets, use = j / kSets;
         if (t == t_begin || tcur.ct == 0) {
           if (!tc::mbar_wait(&bars->q_full, qc & 1, abort, kWaitLimit)) { ok = false; break; }
           ++qc;
         }
         // Two waits per tile: every mbarrier wait of this thread stalls the MMA stream for a
         // few hundred cycles even when the phase is already complete.
-        if (!tc::mbar_wait(&bars->acc_empty[buf], ((j >> 1) & 1) ^ 1, abort, kWaitLimit) ||
+        if (!tc::mbar_wait(&bars->acc_empty[buf], (use & 1) ^ 1, abort, kWaitLimit) ||
             !tc::mbar_wait(&bars->k_full[s], kph, abort, kWaitLimit)) {
           ok = false;
           break;
@@ -254,20 +259,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     TileCursor tcur(t_begin, nrt, nct), tnext = tcur;
     int ej_next = t_begin < t_end ? col_exp(tcur) : 0;
     for (int64_t t = t_begin; t < t_end; ++t, tcur.next()) {
-      const uint32_t j = (uint32_t)(t - t_begin), buf = j & 1;
+      const uint32_t j = (uint32_t)(t - t_begin), buf = j % kSets, use = j / kSets;
       const int64_t bh = tcur.bh;
       const int i0 = tcur.rt * kRowsQ, j0 = tcur.ct * kColsK;
       if (t == t_begin || tcur.ct == 0) ei = i0 + r < m.nb ? eq[bh * m.nb + i0 + r] : 0;
       const int ej_l = ej_next;
       tnext.next();
       if (t + 1 < t_end) ej_next = col_exp(tnext);
-      const bool ready = tc::mbar_wait(&bars->acc_full[buf], (j >> 1) & 1, abort, kWaitLimit);
+      const bool ready = tc::mbar_wait(&bars->acc_full[buf], use & 1, abort, kWaitLimit);
       if (!ready || *abort) break;
       tc::fence_after_sync();
       uint32_t acc[kScoreSlices][kEpiCols];
 #pragma unroll
       for (int l = 0; l < kScoreSlices; ++l)
-        tc::tmem_ld8(tbase + lane_off + buf * kLevelCols + l * kColsK + part * kEpiCols, acc[l]);
+#pragma unroll
+        for (int c8 = 0; c8 < kEpiCols; c8 += 8)
+          tc::tmem_ld8(tbase + lane_off + buf * kLevelCols + l * kColsK + part * kEpiCols + c8,
+                       *reinterpret_cast<uint32_t(*)[8]>(&acc[l][c8]));
       tc::tmem_ld_wait();
       tc::fence_before_sync();
       __syncwarp();
